@@ -1,0 +1,269 @@
+// Op-level C ABI: the tied LM head + cross-entropy alone, LayerNorm,
+// attention and the dense contraction, each on caller-owned device buffers
+// and a caller-provided workspace, asynchronous on the caller's stream.
+//
+// Sources: [ZERO] "GPT training" (Zero docs): output layer (fused projection
+// + cross-entropy whose [B*T, V] logits stay out of the saved graph),
+// Transformer Block (LayerNorm), Attention; [LECTURE] "Andrej Karpathy:
+// reproducing GPT-2 from scratch": tied head over the padded vocabulary;
+// [CS336] "CS336 from scratch — pretraining" §1: cross-entropy with the row
+// maximum subtracted.
+
+#include <algorithm>
+#include <string>
+
+#include "kernels.h"
+
+using gpt2_internal::set_error;
+
+namespace {
+
+constexpr int kLmChunk = 2048;
+
+struct Carve {
+  char* p;
+  size_t left;
+  bool ok = true;
+  void* take(size_t bytes) {
+    bytes = (bytes + 255) / 256 * 256;
+    if (bytes > left) {
+      ok = false;
+      return nullptr;
+    }
+    void* r = p;
+    p += bytes;
+    left -= bytes;
+    return r;
+  }
+};
+
+size_t lm_ws(int M, int C, int Vp, int dtype) {
+  const int mc = std::min(kLmChunk, M);
+  const size_t a = dtype == GPT2_BF16 ? 2 : 4;
+  auto r = [](size_t b) { return (b + 255) / 256 * 256; };
+  size_t gw = std::max({gemm_workspace_bytes(mc, Vp, C), gemm_workspace_bytes(mc, C, Vp),
+                        gemm_workspace_bytes(Vp, C, mc)});
+  return r(size_t(mc) * Vp * 4) + r(size_t(mc) * Vp * a) + 2 * r(size_t(M) * 4) + r(gw) + 256;
+}
+
+__device__ int g_op_error;  // bounded-wait timeouts of op-level launches
+
+}  // namespace
+
+int* device_error_word() {
+  static int* addr[64] = {nullptr};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_op_error) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+extern "C" {
+
+int gpt2_lmhead_ce_workspace(int M, int C, int Vp, int dtype, size_t* bytes) {
+  if (!bytes || M < 1 || C < 1 || Vp < 1) return GPT2_ERR_ARG;
+  *bytes = lm_ws(M, C, Vp, dtype);
+  return GPT2_OK;
+}
+
+int gpt2_lmhead_ce(const void* hidden, const void* W, const int32_t* y, int M, int C, int Vp,
+                   int V, int dtype, float grad_scale, float* d_loss, float* d_lse, void* d_dh,
+                   float* d_dw, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!hidden || !W || !y || !d_loss || M < 1 || C < 1 || Vp < V || V < 1 ||
+      (dtype != GPT2_BF16 && dtype != GPT2_F32)) {
+    set_error("lmhead_ce: bad arguments");
+    return GPT2_ERR_ARG;
+  }
+  if (!workspace || workspace_bytes < lm_ws(M, C, Vp, dtype)) {
+    set_error("lmhead_ce: workspace too small");
+    return GPT2_ERR_ARG;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bf = dtype == GPT2_BF16;
+  const size_t a = bf ? 2 : 4;
+  const int mc_max = std::min(kLmChunk, M);
+  Carve cv{static_cast<char*>(workspace), workspace_bytes};
+  float* z = static_cast<float*>(cv.take(size_t(mc_max) * Vp * 4));
+  void* dz = cv.take(size_t(mc_max) * Vp * a);
+  float* lse = d_lse ? d_lse : static_cast<float*>(cv.take(size_t(M) * 4));
+  float* rl = static_cast<float*>(cv.take(size_t(M) * 4));
+  size_t gw = std::max({gemm_workspace_bytes(mc_max, Vp, C), gemm_workspace_bytes(mc_max, C, Vp),
+                        gemm_workspace_bytes(Vp, C, mc_max)});
+  float* gws = static_cast<float*>(cv.take(gw));
+  if (!cv.ok) {
+    set_error("lmhead_ce: workspace too small");
+    return GPT2_ERR_ARG;
+  }
+  const bool bwd = d_dh || d_dw;
+  const float scale = grad_scale / float(M);
+  for (int64_t r0 = 0; r0 < M; r0 += kLmChunk) {
+    const int mc = int(std::min<int64_t>(kLmChunk, M - r0));
+    const void* hr = static_cast<const char*>(hidden) + r0 * C * int64_t(a);
+    EpiParams e;
+    e.kind = EPI_STORE;
+    e.out = z;
+    e.ldo = Vp;
+    GemmArgs g{hr, 1, C, W, 1, C, bf, mc, Vp, C, e, gws, gw};
+    int rc = gemm_launch(g, st);
+    if (rc) return rc;
+    rc = launch_ce_rows_fwd(z, y + r0, mc, Vp, lse + r0, rl + r0, st);
+    if (rc) return rc;
+    if (!bwd) continue;
+    rc = bf ? launch_ce_rows_bwd<bf16>(z, lse + r0, y + r0, mc, Vp, scale, static_cast<bf16*>(dz), st)
+            : launch_ce_rows_bwd<float>(z, lse + r0, y + r0, mc, Vp, scale, static_cast<float*>(dz), st);
+    if (rc) return rc;
+    if (d_dh) {
+      EpiParams e2;
+      e2.kind = EPI_STORE;
+      e2.out = static_cast<char*>(d_dh) + r0 * C * int64_t(a);
+      e2.ldo = C;
+      e2.out_bf16 = bf;
+      GemmArgs g2{dz, 1, Vp, W, 0, C, bf, mc, C, Vp, e2, gws, gw};
+      rc = gemm_launch(g2, st);
+      if (rc) return rc;
+    }
+    if (d_dw) {
+      EpiParams e3;
+      e3.kind = EPI_ACC;
+      e3.out = d_dw;
+      e3.ldo = C;
+      e3.accumulate = 1;
+      GemmArgs g3{dz, 0, Vp, hr, 0, C, bf, Vp, C, mc, e3, gws, gw};
+      rc = gemm_launch(g3, st);
+      if (rc) return rc;
+    }
+  }
+  return launch_mean(rl, M, d_loss, st);
+}
+
+int gpt2_layernorm_fwd(const float* x, const float* gamma, const float* beta, int64_t M, int C,
+                       float eps, void* y, int y_dtype, float* mean, float* rstd, void* stream) {
+  if (!x || !gamma || !beta || !y || M < 1 || C < 1 || C > 1024) {
+    set_error("layernorm_fwd: bad arguments");
+    return GPT2_ERR_ARG;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (y_dtype == GPT2_BF16)
+    return launch_layernorm_fwd<bf16>(x, gamma, beta, static_cast<bf16*>(y), mean, rstd, M, C, eps, st);
+  if (y_dtype == GPT2_F32)
+    return launch_layernorm_fwd<float>(x, gamma, beta, static_cast<float*>(y), mean, rstd, M, C, eps, st);
+  set_error("layernorm_fwd: bad dtype");
+  return GPT2_ERR_ARG;
+}
+
+int gpt2_layernorm_bwd_workspace(int64_t M, int C, size_t* bytes) {
+  if (!bytes || M < 1 || C < 1) return GPT2_ERR_ARG;
+  *bytes = layernorm_bwd_workspace(M, C);
+  return GPT2_OK;
+}
+
+int gpt2_layernorm_bwd(const void* dy, int dy_dtype, const float* x, const float* mean,
+                       const float* rstd, const float* gamma, int64_t M, int C, float* dx,
+                       float* dgamma, float* dbeta, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (!dy || !x || !mean || !rstd || !gamma || !dx || !dgamma || !dbeta || M < 1 || C < 1 ||
+      C > 1024 || !workspace || workspace_bytes < layernorm_bwd_workspace(M, C)) {
+    set_error("layernorm_bwd: bad arguments or workspace too small");
+    return GPT2_ERR_ARG;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  if (dy_dtype == GPT2_BF16)
+    return launch_layernorm_bwd<bf16, bf16>(static_cast<const bf16*>(dy), x, mean, rstd, gamma, M,
+                                            C, dx, nullptr, dgamma, dbeta, 1, ws, st);
+  if (dy_dtype == GPT2_F32)
+    return launch_layernorm_bwd<float, float>(static_cast<const float*>(dy), x, mean, rstd, gamma,
+                                              M, C, dx, nullptr, dgamma, dbeta, 1, ws, st);
+  set_error("layernorm_bwd: bad dtype");
+  return GPT2_ERR_ARG;
+}
+
+int gpt2_attention_fwd(const void* qkv, int dtype, int B, int T, int C, int H, void* out,
+                       float* lse, void* stream) {
+  if (!qkv || !out || !lse || B < 1 || T < 1 || H < 1 || C % H) {
+    set_error("attention_fwd: bad arguments");
+    return GPT2_ERR_ARG;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == GPT2_BF16)
+    return launch_attn_fwd<bf16>(static_cast<const bf16*>(qkv), B, T, C, H, static_cast<bf16*>(out), lse, st);
+  if (dtype == GPT2_F32)
+    return launch_attn_fwd<float>(static_cast<const float*>(qkv), B, T, C, H, static_cast<float*>(out), lse, st);
+  set_error("attention_fwd: bad dtype");
+  return GPT2_ERR_ARG;
+}
+
+int gpt2_attention_bwd_workspace(int B, int T, int C, int H, int dtype, size_t* bytes) {
+  (void)C;
+  (void)dtype;
+  if (!bytes || B < 1 || T < 1 || H < 1) return GPT2_ERR_ARG;
+  *bytes = attn_bwd_workspace(B, T, H);
+  return GPT2_OK;
+}
+
+int gpt2_attention_bwd(const void* dout, const void* qkv, const void* out, const float* lse,
+                       int dtype, int B, int T, int C, int H, void* dqkv, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (!dout || !qkv || !out || !lse || !dqkv || B < 1 || T < 1 || H < 1 || C % H || !workspace ||
+      workspace_bytes < attn_bwd_workspace(B, T, H)) {
+    set_error("attention_bwd: bad arguments or workspace too small");
+    return GPT2_ERR_ARG;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  if (dtype == GPT2_BF16)
+    return launch_attn_bwd<bf16>(static_cast<const bf16*>(dout), static_cast<const bf16*>(qkv),
+                                 static_cast<const bf16*>(out), lse, B, T, C, H,
+                                 static_cast<bf16*>(dqkv), ws, st);
+  if (dtype == GPT2_F32)
+    return launch_attn_bwd<float>(static_cast<const float*>(dout), static_cast<const float*>(qkv),
+                                  static_cast<const float*>(out), lse, B, T, C, H,
+                                  static_cast<float*>(dqkv), ws, st);
+  set_error("attention_bwd: bad dtype");
+  return GPT2_ERR_ARG;
+}
+
+int gpt2_matmul_workspace(int M, int N, int K, size_t* bytes) {
+  if (!bytes || M < 1 || N < 1 || K < 1) return GPT2_ERR_ARG;
+  *bytes = gemm_workspace_bytes(M, N, K);
+  return GPT2_OK;
+}
+
+int gpt2_matmul(const void* A, int a_kmajor, int64_t lda, const void* B, int b_kmajor, int64_t ldb,
+                int dtype, int M, int N, int K, float alpha, int accumulate, void* D, int d_dtype,
+                int64_t ldd, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!A || !B || !D || M < 1 || N < 1 || K < 1 || (dtype != GPT2_BF16 && dtype != GPT2_F32) ||
+      (accumulate && d_dtype != GPT2_F32) || ldd < N) {
+    set_error("matmul: bad arguments");
+    return GPT2_ERR_ARG;
+  }
+  EpiParams e;
+  e.kind = accumulate ? EPI_ACC : EPI_STORE;
+  e.out = D;
+  e.ldo = ldd;
+  e.alpha = alpha;
+  e.accumulate = accumulate;
+  e.out_bf16 = d_dtype == GPT2_BF16;
+  GemmArgs g{A, a_kmajor ? 1 : 0, lda, B, b_kmajor ? 1 : 0, ldb, dtype == GPT2_BF16, M, N, K, e,
+             static_cast<float*>(workspace), workspace_bytes};
+  return gemm_launch(g, static_cast<cudaStream_t>(stream));
+}
+
+int gpt2_device_error(int* code) {
+  if (!code) return GPT2_ERR_ARG;
+  int* w = device_error_word();
+  if (!w) return GPT2_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GPT2_ERR_CUDA;
+  int z = 0;
+  cudaMemcpy(w, &z, sizeof(int), cudaMemcpyHostToDevice);
+  *code = v ? GPT2_ERR_TIMEOUT : GPT2_OK;
+  return GPT2_OK;
+}
+
+}  // extern "C"

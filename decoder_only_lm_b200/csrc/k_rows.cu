@@ -1,0 +1,704 @@
+// Memory-bound kernels of the training step: batch slicing, embedding
+// forward/backward, LayerNorm forward/backward, bias-gradient column sums,
+// cross-entropy rows, gradient norm and the fused clip+AdamW pass.
+//
+// Sources: [CH28] "Chapter 28: data, evaluation and recovery" §28.3 (B*T+1
+// slicing); [ZERO] "GPT training" (Zero docs): Embedding, Transformer Block
+// (pre-LN), output layer; [CS336] "CS336 from scratch — pretraining" §1
+// cross-entropy (max subtracted), §2 AdamW (bias correction folded into the
+// step size, decay before the update) and gradient clipping
+// (min(1, c/(n+1e-6))); [LECTURE] "Andrej Karpathy: reproducing GPT-2 from
+// scratch": tied head gradients add, decay on matrices only, fused AdamW.
+//
+// All reductions are in a fixed order (no floating-point atomics), so two runs
+// on the same inputs give identical bits.
+
+#include <algorithm>
+
+#include "kernels.h"
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// ------------------------------------------------------------ batch slicing
+__global__ void slice_batch_kernel(const uint16_t* __restrict__ s, int64_t off, int64_t n,
+                                   int32_t* __restrict__ x, int32_t* __restrict__ y) {
+  int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i < n) {
+    x[i] = int32_t(s[off + i]);
+    y[i] = int32_t(s[off + i + 1]);
+  }
+}
+
+// ------------------------------------------------------------ embedding
+// out[m, :] = wte[x_m, :] + wpe[t_m, :] in fp32; ids outside [0, V) are
+// recorded in the status word and read as id 0 so no access leaves the table.
+__global__ void embed_fwd_kernel(const int32_t* __restrict__ x, const int32_t* __restrict__ y,
+                                 const float* __restrict__ wte, const float* __restrict__ wpe,
+                                 int T, int C, int V, int64_t M, float* __restrict__ out,
+                                 DevStatus* status) {
+  int64_t m = blockIdx.x;
+  if (m >= M) return;
+  int id = x[m];
+  if (threadIdx.x == 0) {
+    int yy = y ? y[m] : 0;
+    if (id < 0 || id >= V || yy < 0 || yy >= V) atomicExch(&status->token_bad, 1);
+  }
+  if (id < 0 || id >= V) id = 0;
+  const int t = int(m % T);
+  const float* a = wte + int64_t(id) * C;
+  const float* b = wpe + int64_t(t) * C;
+  float* o = out + m * C;
+  if ((C & 3) == 0) {
+    for (int c = threadIdx.x * 4; c < C; c += blockDim.x * 4) {
+      float4 u = *reinterpret_cast<const float4*>(a + c);
+      float4 w = *reinterpret_cast<const float4*>(b + c);
+      *reinterpret_cast<float4*>(o + c) = make_float4(u.x + w.x, u.y + w.y, u.z + w.z, u.w + w.w);
+    }
+  } else {
+    for (int c = threadIdx.x; c < C; c += blockDim.x) o[c] = a[c] + b[c];
+  }
+}
+
+// Embedding backward, deterministic:
+//  1. keys_m = (x_m << 32) | m, padded with ~0 to a power of two, bitonic-sorted
+//     (ties impossible: m is unique), so equal ids are grouped in index order;
+//  2. pieces: every run of equal ids inside an aligned group of 32 sorted
+//     entries is summed (rows of dh in index order) into piece[first entry];
+//  3. every run start adds its pieces (stride 32) in order into dwte[id].
+constexpr int kSortChunk = 2048;  // keys sorted in shared memory by one block
+constexpr int kPiece = 32;
+
+__device__ __forceinline__ void cmp_swap(uint64_t& a, uint64_t& b, bool up) {
+  if ((a > b) == up) {
+    uint64_t t = a;
+    a = b;
+    b = t;
+  }
+}
+
+__global__ void make_keys_kernel(const int32_t* __restrict__ x, int64_t M, int64_t Mp, int V,
+                                 uint64_t* __restrict__ keys) {
+  int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= Mp) return;
+  if (i < M) {
+    int id = x[i];
+    if (id < 0 || id >= V) id = 0;  // recorded by the forward; keep accesses in range
+    keys[i] = (uint64_t(uint32_t(id)) << 32) | uint64_t(i);
+  } else {
+    keys[i] = ~uint64_t(0);
+  }
+}
+
+// Stages k = 2 .. min(kSortChunk, Mp) of the bitonic network inside one chunk,
+// directions taken from the global index.  `k_from` > 2 restarts at a merge
+// level (then only the j < kSortChunk steps of level k_from are done).
+__global__ void bitonic_chunk_kernel(uint64_t* __restrict__ keys, int64_t Mp, int64_t k_only) {
+  __shared__ uint64_t s[kSortChunk];
+  const int64_t base = int64_t(blockIdx.x) * kSortChunk;
+  const int n = int(min64(kSortChunk, Mp));
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s[i] = keys[base + i];
+  __syncthreads();
+  int64_t k_lo = 2, k_hi = n;
+  if (k_only) k_lo = k_hi = k_only;
+  for (int64_t k = k_lo; k <= k_hi; k <<= 1) {
+    for (int j = int(min64(k >> 1, n >> 1)); j > 0; j >>= 1) {
+      for (int t = threadIdx.x; t < n / 2; t += blockDim.x) {
+        int i = 2 * j * (t / j) + (t % j);
+        int64_t gi = base + i;
+        cmp_swap(s[i], s[i + j], (gi & k) == 0);
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[base + i] = s[i];
+}
+
+__global__ void bitonic_global_kernel(uint64_t* __restrict__ keys, int64_t Mp, int64_t j,
+                                      int64_t k) {
+  int64_t t = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (t >= Mp / 2) return;
+  int64_t i = 2 * j * (t / j) + (t % j);
+  uint64_t a = keys[i], b = keys[i + j];
+  bool up = (i & k) == 0;
+  if ((a > b) == up) {
+    keys[i] = b;
+    keys[i + j] = a;
+  }
+}
+
+__global__ void embed_pieces_kernel(const uint64_t* __restrict__ keys, const float* __restrict__ dh,
+                                    int64_t M, int C, float* __restrict__ piece) {
+  const int64_t r0 = int64_t(blockIdx.x) * kPiece;
+  const int64_t r1 = min64(M, r0 + kPiece);
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float acc = 0.f;
+    int64_t start = r0;
+    uint32_t cur = uint32_t(keys[r0] >> 32);
+    for (int64_t r = r0; r < r1; ++r) {
+      uint64_t kk = keys[r];
+      uint32_t id = uint32_t(kk >> 32);
+      if (id != cur) {
+        piece[start * C + c] = acc;
+        acc = 0.f;
+        start = r;
+        cur = id;
+      }
+      acc += dh[int64_t(uint32_t(kk)) * C + c];
+    }
+    piece[start * C + c] = acc;
+  }
+}
+
+__global__ void embed_runs_kernel(const uint64_t* __restrict__ keys, const float* __restrict__ piece,
+                                  int64_t M, int C, float* __restrict__ dwte) {
+  const int64_t r0 = int64_t(blockIdx.x) * kPiece;
+  const int64_t r1 = min64(M, r0 + kPiece);
+  for (int64_t r = r0; r < r1; ++r) {
+    const uint32_t id = uint32_t(keys[r] >> 32);
+    if (r > 0 && uint32_t(keys[r - 1] >> 32) == id) continue;  // not a run start
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      float acc = piece[r * C + c];
+      for (int64_t q = (r / kPiece + 1) * kPiece; q < M && uint32_t(keys[q] >> 32) == id; q += kPiece)
+        acc += piece[q * C + c];
+      dwte[int64_t(id) * C + c] += acc;
+    }
+  }
+}
+
+// dwpe[t, c] (+)= sum_b dh[b, t, c]
+__global__ void embed_wpe_kernel(const float* __restrict__ dh, int B, int T, int C,
+                                 float* __restrict__ dwpe, int accumulate) {
+  int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= int64_t(T) * C) return;
+  float acc = 0.f;
+  for (int b = 0; b < B; ++b) acc += dh[int64_t(b) * T * C + i];
+  dwpe[i] = accumulate ? dwpe[i] + acc : acc;
+}
+
+// ------------------------------------------------------------ LayerNorm
+constexpr int kLnMaxPerLane = 32;  // C <= 1024
+
+template <typename OutT>
+__global__ void layernorm_fwd_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                     const float* __restrict__ b, OutT* __restrict__ y,
+                                     float* __restrict__ mean, float* __restrict__ rstd,
+                                     int64_t M, int C, float eps) {
+  const int64_t row = int64_t(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float* xr = x + row * C;
+  float v[kLnMaxPerLane];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kLnMaxPerLane; ++i) {
+    int c = lane + 32 * i;
+    v[i] = c < C ? xr[c] : 0.f;
+    s += v[i];
+  }
+  const float mu = warp_sum(s) / float(C);
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < kLnMaxPerLane; ++i) {
+    int c = lane + 32 * i;
+    float d = c < C ? v[i] - mu : 0.f;
+    q += d * d;
+  }
+  const float rs = rsqrtf(warp_sum(q) / float(C) + eps);
+  OutT* yr = y + row * C;
+#pragma unroll
+  for (int i = 0; i < kLnMaxPerLane; ++i) {
+    int c = lane + 32 * i;
+    if (c < C) yr[c] = from_f32<OutT>((v[i] - mu) * rs * g[c] + b[c]);
+  }
+  if (lane == 0) {
+    if (mean) mean[row] = mu;
+    if (rstd) rstd[row] = rs;
+  }
+}
+
+// One block = 8 warps; each warp takes rows row0 + warp, row0 + warp + 8, ...
+// (kLnRowsPerBlock rows per block).  dx is ADDED to `dx` (the residual-stream
+// gradient) and, when dx_copy is given, the new dx is also stored rounded to
+// CopyT.  Column partials of dgamma/dbeta go to ws[block][2C].
+constexpr int kLnRowsPerBlock = 64;
+
+template <typename DyT, typename CopyT>
+__global__ void layernorm_bwd_kernel(const DyT* __restrict__ dy, const float* __restrict__ x,
+                                     const float* __restrict__ mean, const float* __restrict__ rstd,
+                                     const float* __restrict__ g, int64_t M, int C,
+                                     float* __restrict__ dx, CopyT* __restrict__ dx_copy,
+                                     float* __restrict__ ws) {
+  __shared__ float red[8][2][kLnMaxPerLane * 32 / 8];  // reused per column slice
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  float pg[kLnMaxPerLane], pb[kLnMaxPerLane];
+#pragma unroll
+  for (int i = 0; i < kLnMaxPerLane; ++i) pg[i] = pb[i] = 0.f;
+  const int64_t row0 = int64_t(blockIdx.x) * kLnRowsPerBlock;
+  for (int rr = warp; rr < kLnRowsPerBlock; rr += 8) {
+    const int64_t row = row0 + rr;
+    if (row >= M) break;
+    const float mu = mean[row], rs = rstd[row];
+    float xh[kLnMaxPerLane], dyv[kLnMaxPerLane];
+    float a = 0.f, bsum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kLnMaxPerLane; ++i) {
+      int c = lane + 32 * i;
+      if (c < C) {
+        xh[i] = (x[row * C + c] - mu) * rs;
+        dyv[i] = to_f32<DyT>(dy[row * C + c]);
+        float dxh = dyv[i] * g[c];
+        a += dxh;
+        bsum += dxh * xh[i];
+        pg[i] += dyv[i] * xh[i];
+        pb[i] += dyv[i];
+      } else {
+        xh[i] = dyv[i] = 0.f;
+      }
+    }
+    a = warp_sum(a) / float(C);
+    bsum = warp_sum(bsum) / float(C);
+#pragma unroll
+    for (int i = 0; i < kLnMaxPerLane; ++i) {
+      int c = lane + 32 * i;
+      if (c < C) {
+        float dxh = dyv[i] * g[c];
+        float nv = dx[row * C + c] + rs * (dxh - a - xh[i] * bsum);
+        dx[row * C + c] = nv;
+        if (dx_copy) dx_copy[row * C + c] = from_f32<CopyT>(nv);
+      }
+    }
+  }
+  // Reduce the 8 warps' column partials in a fixed order, 128 columns at a time.
+  float* out = ws + int64_t(blockIdx.x) * 2 * C;
+#pragma unroll
+  for (int i0 = 0; i0 < kLnMaxPerLane; i0 += 4) {
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      red[warp][0][i * 32 + lane] = pg[i0 + i];
+      red[warp][1][i * 32 + lane] = pb[i0 + i];
+    }
+    __syncthreads();
+    if (threadIdx.x < 128) {
+      const int i = threadIdx.x / 32, l = threadIdx.x & 31;
+      const int c = l + 32 * (i0 + i);
+      if (c < C) {
+        float sg = 0.f, sb = 0.f;
+        for (int w = 0; w < 8; ++w) {
+          sg += red[w][0][threadIdx.x];
+          sb += red[w][1][threadIdx.x];
+        }
+        out[c] = sg;
+        out[C + c] = sb;
+      }
+    }
+  }
+}
+
+// out[c] (+)= sum over `parts` rows of ws[., c], in order.
+__global__ void reduce_partials_kernel(const float* __restrict__ ws, int parts, int n,
+                                       float* __restrict__ out, int accumulate) {
+  int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= n) return;
+  float acc = 0.f;
+  for (int p = 0; p < parts; ++p) acc += ws[int64_t(p) * n + c];
+  out[c] = accumulate ? out[c] + acc : acc;
+}
+
+__global__ void reduce_ln_partials_kernel(const float* __restrict__ ws, int parts, int C,
+                                          float* __restrict__ dg, float* __restrict__ db,
+                                          int accumulate) {
+  int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= 2 * C) return;
+  float acc = 0.f;
+  for (int p = 0; p < parts; ++p) acc += ws[int64_t(p) * 2 * C + c];
+  float* o = c < C ? dg + c : db + (c - C);
+  *o = accumulate ? *o + acc : acc;
+}
+
+// ------------------------------------------------------------ bias-gradient column sums
+constexpr int kColRows = 256;  // rows per partial
+
+template <typename InT>
+__global__ void colsum_partial_kernel(const InT* __restrict__ in, int64_t M, int N,
+                                      float* __restrict__ ws) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  const int64_t r0 = int64_t(blockIdx.y) * kColRows;
+  const int64_t r1 = min64(M, r0 + kColRows);
+  float acc = 0.f;
+  for (int64_t r = r0; r < r1; ++r) acc += to_f32<InT>(in[r * N + n]);
+  ws[int64_t(blockIdx.y) * N + n] = acc;
+}
+
+// ------------------------------------------------------------ cross-entropy rows
+// lse_r = max_v z + log sum_v exp(z - max);  row_loss_r = lse_r - z[r, y_r].
+__global__ void ce_rows_fwd_kernel(const float* __restrict__ z, const int32_t* __restrict__ y,
+                                   int Vp, float* __restrict__ lse, float* __restrict__ row_loss) {
+  __shared__ float sh[32];
+  const int r = blockIdx.x;
+  const float* zr = z + int64_t(r) * Vp;
+  float mx = -INFINITY;
+  for (int v = threadIdx.x; v < Vp; v += blockDim.x) mx = fmaxf(mx, zr[v]);
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x / 32] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < blockDim.x / 32 ? sh[threadIdx.x] : -INFINITY;
+    t = warp_max(t);
+    if (threadIdx.x == 0) sh[0] = t;
+  }
+  __syncthreads();
+  mx = sh[0];
+  __syncthreads();
+  float s = 0.f;
+  for (int v = threadIdx.x; v < Vp; v += blockDim.x) s += expf(zr[v] - mx);
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x / 32] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < int(blockDim.x / 32); ++w) t += sh[w];
+    float l = mx + logf(t);
+    lse[r] = l;
+    row_loss[r] = l - zr[y[r]];
+  }
+}
+
+template <typename OutT>
+__global__ void ce_rows_bwd_kernel(const float* __restrict__ z, const float* __restrict__ lse,
+                                   const int32_t* __restrict__ y, int Vp, float scale,
+                                   OutT* __restrict__ dz) {
+  const int r = blockIdx.x;
+  const float* zr = z + int64_t(r) * Vp;
+  OutT* dr = dz + int64_t(r) * Vp;
+  const float l = lse[r];
+  const int t = y[r];
+  for (int v = threadIdx.x; v < Vp; v += blockDim.x)
+    dr[v] = from_f32<OutT>(scale * (expf(zr[v] - l) - (v == t ? 1.f : 0.f)));
+}
+
+// out = mean of v[0..n), fixed order (one block).
+__global__ void mean_kernel(const float* __restrict__ v, int64_t n, float* __restrict__ out) {
+  __shared__ double sh[kThreads];
+  double acc = 0.0;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) acc += double(v[i]);
+  sh[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) sh[threadIdx.x] += sh[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *out = float(sh[0] / double(n));
+}
+
+// ------------------------------------------------------------ gradient norm, clip + AdamW
+constexpr int kNormBlocks = 1024;
+
+__global__ void sumsq_kernel(const float* __restrict__ g, int64_t n, double* __restrict__ ws) {
+  __shared__ double sh[kThreads];
+  const int64_t chunk = (n + kNormBlocks - 1) / kNormBlocks;
+  const int64_t a = int64_t(blockIdx.x) * chunk, e = min64(n, a + chunk);
+  double acc = 0.0;
+  for (int64_t i = a + threadIdx.x; i < e; i += blockDim.x) {
+    float v = g[i];
+    acc += double(v) * double(v);
+  }
+  sh[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) sh[threadIdx.x] += sh[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) ws[blockIdx.x] = sh[0];
+}
+
+__global__ void norm_finalize_kernel(const double* __restrict__ ws, float* __restrict__ norm) {
+  __shared__ double sh[kNormBlocks];
+  for (int i = threadIdx.x; i < kNormBlocks; i += blockDim.x) sh[i] = ws[i];
+  __syncthreads();
+  for (int s = kNormBlocks / 2; s > 0; s >>= 1) {
+    for (int i = threadIdx.x; i < s; i += blockDim.x) sh[i] += sh[i + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) norm[0] = float(sqrt(sh[0]));
+}
+
+// One fused pass.  Elements [0, n_decay) belong to 2-D tensors (decayed).
+// Every thread reads the same status and norm, so either all of them update
+// or none does; the step counter is advanced by step_advance_kernel.
+__global__ void clip_adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
+                                  float* __restrict__ m, float* __restrict__ v,
+                                  bf16* __restrict__ pb, int64_t n, int64_t n_decay,
+                                  const float* __restrict__ norm, const DevStatus* __restrict__ st,
+                                  float lr, float b1, float b2, float eps, float wd,
+                                  float max_norm) {
+  const float nrm = *norm;
+  if (st->token_bad || !isfinite(nrm)) return;
+  const int t = st->step + 1;
+  const float s = fminf(1.f, max_norm / (nrm + 1e-6f));
+  const float alpha = lr * sqrtf(1.f - powf(b2, float(t))) / (1.f - powf(b1, float(t)));
+  const float dec = 1.f - lr * wd;
+  const int64_t n4 = n / 4;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n4;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    float4 P = reinterpret_cast<float4*>(p)[i];
+    float4 G = reinterpret_cast<const float4*>(g)[i];
+    float4 Mo = reinterpret_cast<float4*>(m)[i];
+    float4 Vo = reinterpret_cast<float4*>(v)[i];
+    const float d = (i * 4 < n_decay) ? dec : 1.f;  // n_decay is a multiple of 4
+    float* pp = &P.x;
+    float* gg = &G.x;
+    float* mm = &Mo.x;
+    float* vv = &Vo.x;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float gk = s * gg[k];
+      mm[k] = b1 * mm[k] + (1.f - b1) * gk;
+      vv[k] = b2 * vv[k] + (1.f - b2) * gk * gk;
+      pp[k] = pp[k] * d;
+      pp[k] -= alpha * mm[k] / (sqrtf(vv[k]) + eps);
+    }
+    reinterpret_cast<float4*>(p)[i] = P;
+    reinterpret_cast<float4*>(m)[i] = Mo;
+    reinterpret_cast<float4*>(v)[i] = Vo;
+    if (pb) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(P.x, P.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(P.z, P.w);
+      reinterpret_cast<__nv_bfloat162*>(pb)[2 * i] = lo;
+      reinterpret_cast<__nv_bfloat162*>(pb)[2 * i + 1] = hi;
+    }
+  }
+}
+
+__global__ void step_advance_kernel(const float* __restrict__ norm, DevStatus* st) {
+  if (st->token_bad) return;
+  if (!isfinite(*norm)) {
+    st->nonfinite = 1;
+    return;
+  }
+  st->step += 1;
+}
+
+__global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, int64_t n) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
+       i += int64_t(gridDim.x) * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+__global__ void fill_kernel(float* __restrict__ p, float v, int64_t n) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
+       i += int64_t(gridDim.x) * blockDim.x)
+    p[i] = v;
+}
+
+int grid_for(int64_t n, int threads) {
+  int64_t b = (n + threads - 1) / threads;
+  int cap = gpt2_internal::sm_count() * 8;
+  return int(max64(1, min64(b, cap)));
+}
+
+int64_t next_pow2(int64_t n) {
+  int64_t p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
+}  // namespace
+
+// ============================================================ launchers
+
+int launch_slice_batch(const uint16_t* s, int64_t off, int64_t n, int32_t* x, int32_t* y,
+                       cudaStream_t st) {
+  if (n <= 0) return GPT2_OK;
+  slice_batch_kernel<<<int(cdiv64(n, kThreads)), kThreads, 0, st>>>(s, off, n, x, y);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int launch_embed_fwd(const int32_t* x, const int32_t* y, const float* wte, const float* wpe, int B,
+                     int T, int C, int V, float* out, DevStatus* status, cudaStream_t st) {
+  const int64_t M = int64_t(B) * T;
+  embed_fwd_kernel<<<int(M), 192, 0, st>>>(x, y, wte, wpe, T, C, V, M, out, status);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+size_t embed_bwd_workspace(int64_t M, int C) {
+  int64_t Mp = max64(next_pow2(M), 2);
+  return size_t(Mp) * sizeof(uint64_t) + size_t(M) * C * sizeof(float) + 256;
+}
+
+int launch_embed_bwd(const int32_t* x, const float* dh, int B, int T, int C, int V, float* dwte,
+                     float* dwpe, int wpe_accumulate, void* ws, cudaStream_t st) {
+  const int64_t M = int64_t(B) * T;
+  const int64_t Mp = max64(next_pow2(M), 2);
+  uint64_t* keys = reinterpret_cast<uint64_t*>(ws);
+  float* piece = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) +
+                                          ((size_t(Mp) * sizeof(uint64_t) + 255) / 256) * 256);
+  make_keys_kernel<<<int(cdiv64(Mp, kThreads)), kThreads, 0, st>>>(x, M, Mp, V, keys);
+  COUNT_LAUNCH(1);
+  const int nchunks = int(max64(1, Mp / kSortChunk));
+  bitonic_chunk_kernel<<<nchunks, 1024, 0, st>>>(keys, Mp, 0);
+  COUNT_LAUNCH(1);
+  for (int64_t k = 2 * kSortChunk; k <= Mp; k <<= 1) {
+    for (int64_t j = k >> 1; j >= kSortChunk; j >>= 1) {
+      bitonic_global_kernel<<<int(cdiv64(Mp / 2, kThreads)), kThreads, 0, st>>>(keys, Mp, j, k);
+      COUNT_LAUNCH(1);
+    }
+    bitonic_chunk_kernel<<<nchunks, 1024, 0, st>>>(keys, Mp, k);
+    COUNT_LAUNCH(1);
+  }
+  const int nb = int(cdiv64(M, kPiece));
+  embed_pieces_kernel<<<nb, std::min(C, 256), 0, st>>>(keys, dh, M, C, piece);
+  COUNT_LAUNCH(1);
+  embed_runs_kernel<<<nb, std::min(C, 256), 0, st>>>(keys, piece, M, C, dwte);
+  COUNT_LAUNCH(1);
+  embed_wpe_kernel<<<int(cdiv64(int64_t(T) * C, kThreads)), kThreads, 0, st>>>(dh, B, T, C, dwpe,
+                                                                               wpe_accumulate);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+template <typename OutT>
+int launch_layernorm_fwd(const float* x, const float* g, const float* b, OutT* y, float* mean,
+                         float* rstd, int64_t M, int C, float eps, cudaStream_t st) {
+  if (C > kLnMaxPerLane * 32) {
+    gpt2_internal::set_error("layernorm: C above 1024");
+    return GPT2_ERR_ARG;
+  }
+  layernorm_fwd_kernel<OutT><<<int(cdiv64(M, 8)), 256, 0, st>>>(x, g, b, y, mean, rstd, M, C, eps);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+template int launch_layernorm_fwd<float>(const float*, const float*, const float*, float*, float*,
+                                         float*, int64_t, int, float, cudaStream_t);
+template int launch_layernorm_fwd<bf16>(const float*, const float*, const float*, bf16*, float*,
+                                        float*, int64_t, int, float, cudaStream_t);
+
+size_t layernorm_bwd_workspace(int64_t M, int C) {
+  return size_t(cdiv64(M, kLnRowsPerBlock)) * 2 * C * sizeof(float);
+}
+
+template <typename DyT, typename CopyT>
+int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const float* rstd,
+                         const float* g, int64_t M, int C, float* dx, CopyT* dx_copy, float* dg,
+                         float* db, int accumulate, float* ws, cudaStream_t st) {
+  if (C > kLnMaxPerLane * 32) {
+    gpt2_internal::set_error("layernorm: C above 1024");
+    return GPT2_ERR_ARG;
+  }
+  const int nb = int(cdiv64(M, kLnRowsPerBlock));
+  layernorm_bwd_kernel<DyT, CopyT><<<nb, 256, 0, st>>>(dy, x, mean, rstd, g, M, C, dx, dx_copy, ws);
+  COUNT_LAUNCH(1);
+  // ws rows hold [dgamma | dbeta]; both halves are reduced in one pass
+  reduce_ln_partials_kernel<<<cdiv(2 * C, 256), 256, 0, st>>>(ws, nb, C, dg, db, accumulate);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+template int launch_layernorm_bwd<float, float>(const float*, const float*, const float*,
+                                                const float*, const float*, int64_t, int, float*,
+                                                float*, float*, float*, int, float*, cudaStream_t);
+template int launch_layernorm_bwd<bf16, bf16>(const bf16*, const float*, const float*, const float*,
+                                              const float*, int64_t, int, float*, bf16*, float*,
+                                              float*, int, float*, cudaStream_t);
+template int launch_layernorm_bwd<float, bf16>(const float*, const float*, const float*,
+                                               const float*, const float*, int64_t, int, float*,
+                                               bf16*, float*, float*, int, float*, cudaStream_t);
+
+size_t colsum_workspace(int64_t M, int N) { return size_t(cdiv64(M, kColRows)) * N * sizeof(float); }
+
+template <typename InT>
+int launch_colsum(const InT* in, int64_t M, int N, float* out, int accumulate, float* ws,
+                  cudaStream_t st) {
+  const int parts = int(cdiv64(M, kColRows));
+  dim3 grid(cdiv(N, kThreads), parts);
+  colsum_partial_kernel<InT><<<grid, kThreads, 0, st>>>(in, M, N, ws);
+  COUNT_LAUNCH(1);
+  reduce_partials_kernel<<<cdiv(N, kThreads), kThreads, 0, st>>>(ws, parts, N, out, accumulate);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+template int launch_colsum<float>(const float*, int64_t, int, float*, int, float*, cudaStream_t);
+template int launch_colsum<bf16>(const bf16*, int64_t, int, float*, int, float*, cudaStream_t);
+
+size_t gradnorm_workspace() { return kNormBlocks * sizeof(double); }
+
+int launch_gradnorm(const float* g, int64_t n, double* ws, float* norm, cudaStream_t st) {
+  sumsq_kernel<<<kNormBlocks, kThreads, 0, st>>>(g, n, ws);
+  COUNT_LAUNCH(1);
+  norm_finalize_kernel<<<1, 1024, 0, st>>>(ws, norm);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int launch_clip_adamw(float* p, const float* g, float* m, float* v, bf16* pb, int64_t n,
+                      int64_t n_decay, const float* norm, DevStatus* status, float lr, float b1,
+                      float b2, float eps, float wd, float max_norm, cudaStream_t st) {
+  if ((n & 3) || (n_decay & 3)) {
+    gpt2_internal::set_error("clip_adamw: arena sizes must be multiples of 4");
+    return GPT2_ERR_ARG;
+  }
+  clip_adamw_kernel<<<grid_for(n / 4, kThreads), kThreads, 0, st>>>(
+      p, g, m, v, pb, n, n_decay, norm, status, lr, b1, b2, eps, wd, max_norm);
+  COUNT_LAUNCH(1);
+  step_advance_kernel<<<1, 1, 0, st>>>(norm, status);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int launch_ce_rows_fwd(const float* z, const int32_t* y, int rows, int Vp, float* lse,
+                       float* row_loss, cudaStream_t st) {
+  if (rows <= 0) return GPT2_OK;
+  ce_rows_fwd_kernel<<<rows, 512, 0, st>>>(z, y, Vp, lse, row_loss);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+template <typename OutT>
+int launch_ce_rows_bwd(const float* z, const float* lse, const int32_t* y, int rows, int Vp,
+                       float scale, OutT* dz, cudaStream_t st) {
+  if (rows <= 0) return GPT2_OK;
+  ce_rows_bwd_kernel<OutT><<<rows, 512, 0, st>>>(z, lse, y, Vp, scale, dz);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+template int launch_ce_rows_bwd<float>(const float*, const float*, const int32_t*, int, int, float,
+                                       float*, cudaStream_t);
+template int launch_ce_rows_bwd<bf16>(const float*, const float*, const int32_t*, int, int, float,
+                                      bf16*, cudaStream_t);
+
+int launch_mean(const float* v, int64_t n, float* out, cudaStream_t st) {
+  mean_kernel<<<1, kThreads, 0, st>>>(v, n, out);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int launch_to_bf16(const float* src, bf16* dst, int64_t n, cudaStream_t st) {
+  if (n <= 0) return GPT2_OK;
+  to_bf16_kernel<<<grid_for(n, kThreads), kThreads, 0, st>>>(src, dst, n);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int launch_fill(float* p, float v, int64_t n, cudaStream_t st) {
+  if (n <= 0) return GPT2_OK;
+  fill_kernel<<<grid_for(n, kThreads), kThreads, 0, st>>>(p, v, n);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}

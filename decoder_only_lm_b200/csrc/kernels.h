@@ -1,0 +1,94 @@
+// Host-side launchers of the library's kernels (internal, C++ linkage).
+#pragma once
+
+#include "common.cuh"
+
+// ---------------------------------------------------------------- GEMM
+// D[m,n] = epilogue(sum_k A(m,k) B(n,k)).
+// A(m,k) = A[m*lda+k] (K-major) or A[k*lda+m] (MN-major); B(n,k) likewise.
+enum EpiKind {
+  EPI_STORE = 0,     // out = alpha*acc (+ bias[n])                  -> out type
+  EPI_GELU = 1,      // u = acc + bias -> out; g = gelu(u) -> out2    (act type)
+  EPI_RESID = 2,     // rout = rin + acc + bias                       (fp32)
+  EPI_ACC = 3,       // out = (accumulate ? out : 0) + alpha*acc      (fp32)
+  EPI_GELU_BWD = 4,  // out = acc * gelu'(aux[m,n])                   (act type)
+  EPI_CE_GRAD = 5,   // out = scale*(exp(acc - lse[m]) - [n == tgt[m]]) (act type)
+};
+
+struct EpiParams {
+  int kind = EPI_STORE;
+  void* out = nullptr;
+  int64_t ldo = 0;
+  int out_bf16 = 0;        // element type of out / out2 / aux
+  void* out2 = nullptr;
+  const float* bias = nullptr;
+  const float* rin = nullptr;
+  float* rout = nullptr;
+  const void* aux = nullptr;
+  float alpha = 1.f;
+  int accumulate = 0;
+  const int32_t* tgt = nullptr;
+  const float* lse = nullptr;
+  float ce_scale = 0.f;
+};
+
+struct GemmArgs {
+  const void* A; int a_kmajor; int64_t lda;
+  const void* B; int b_kmajor; int64_t ldb;
+  int bf16_in;  // A and B are bf16 (else fp32)
+  int M, N, K;
+  EpiParams ep;
+  float* ws; size_t ws_bytes;  // split-K partial sums (EPI_ACC only)
+};
+
+size_t gemm_workspace_bytes(int M, int N, int K);
+int gemm_launch(const GemmArgs& g, cudaStream_t st);
+
+// ---------------------------------------------------------------- elementwise / rows
+int launch_slice_batch(const uint16_t* s, int64_t off, int64_t n, int32_t* x, int32_t* y,
+                       cudaStream_t st);
+int launch_embed_fwd(const int32_t* x, const int32_t* y, const float* wte, const float* wpe,
+                     int B, int T, int C, int V, float* out, DevStatus* status, cudaStream_t st);
+// dwte[x_m] += dh[m] (deterministic: sort by id, segmented sums); dwpe[t] (+)= sum_b dh[b,t].
+size_t embed_bwd_workspace(int64_t M, int C);
+int launch_embed_bwd(const int32_t* x, const float* dh, int B, int T, int C, int V, float* dwte,
+                     float* dwpe, int wpe_accumulate, void* ws, cudaStream_t st);
+template <typename OutT>
+int launch_layernorm_fwd(const float* x, const float* g, const float* b, OutT* y, float* mean,
+                         float* rstd, int64_t M, int C, float eps, cudaStream_t st);
+size_t layernorm_bwd_workspace(int64_t M, int C);
+template <typename DyT, typename CopyT>
+int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const float* rstd,
+                         const float* g, int64_t M, int C, float* dx, CopyT* dx_copy,
+                         float* dg, float* db, int accumulate, float* ws, cudaStream_t st);
+size_t colsum_workspace(int64_t M, int N);
+template <typename InT>
+int launch_colsum(const InT* in, int64_t M, int N, float* out, int accumulate, float* ws,
+                  cudaStream_t st);
+// gradient norm (deterministic two-stage, double accumulation) into *norm (device)
+size_t gradnorm_workspace();
+int launch_gradnorm(const float* g, int64_t n, double* ws, float* norm, cudaStream_t st);
+int launch_clip_adamw(float* p, const float* g, float* m, float* v, bf16* pb, int64_t n,
+                      int64_t n_decay, const float* norm, DevStatus* status, float lr, float b1,
+                      float b2, float eps, float wd, float max_norm, cudaStream_t st);
+int launch_to_bf16(const float* src, bf16* dst, int64_t n, cudaStream_t st);
+int launch_fill(float* p, float v, int64_t n, cudaStream_t st);
+// cross-entropy over a chunk of logits rows z [rows, Vp] (fp32)
+int launch_ce_rows_fwd(const float* z, const int32_t* y, int rows, int Vp, float* lse,
+                       float* row_loss, cudaStream_t st);
+template <typename OutT>
+int launch_ce_rows_bwd(const float* z, const float* lse, const int32_t* y, int rows, int Vp,
+                       float scale, OutT* dz, cudaStream_t st);
+int launch_mean(const float* v, int64_t n, float* out, cudaStream_t st);
+
+// ---------------------------------------------------------------- attention
+template <typename T>
+int launch_attn_fwd(const T* qkv, int B, int Tn, int C, int H, T* out, float* lse,
+                    cudaStream_t st);
+size_t attn_bwd_workspace(int B, int Tn, int H);
+template <typename T>
+int launch_attn_bwd(const T* dout, const T* qkv, const T* out, const float* lse, int B, int Tn,
+                    int C, int H, T* dqkv, float* ws, cudaStream_t st);
+
+// device error word of the op-level calls (bounded waits)
+int* device_error_word();

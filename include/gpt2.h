@@ -1,0 +1,310 @@
+/*
+ * gpt2.h — C ABI of the B200 GPT-2 training-step library (libgpt2_b200.so).
+ *
+ * One training step of a decoder-only GPT-2: token + position embedding,
+ * pre-LN transformer blocks (LayerNorm, QKV projection with bias, causal
+ * multi-head attention, output projection, 4x feed-forward with tanh GELU,
+ * residual adds), a final LayerNorm, an LM head tied to the token embedding,
+ * mean next-token cross-entropy, the backward pass, global grad-norm clipping
+ * and AdamW with decoupled weight decay and bias correction.  Every step runs
+ * in hand-written sm_100a CUDA kernels; there is no CPU path.
+ *
+ * Sources the operations follow (cited by page and section):
+ *   [LECTURE] "Andrej Karpathy: reproducing GPT-2 from scratch" (lecture
+ *             summary, youtublog.net): architecture, tied head, padded
+ *             vocabulary, mixed precision, decay groups, clipping.
+ *   [CH28]    "Chapter 28: data, evaluation and recovery" (book.ozine.me),
+ *             §28.3 batches of B*T+1 tokens, §28.4 validation loss.
+ *   [CS336]   "CS336 from scratch — pretraining" (fengye404.top), §1
+ *             cross-entropy, §2 AdamW and gradient clipping.
+ *   [ZERO]    "GPT training" (Zero framework docs, ismantic.github.io):
+ *             autoregressive objective, model sections, training loop.
+ *
+ * Conventions for every entry point
+ *   - Return value: GPT2_OK (0) or one of the GPT2_ERR_* codes below.  No C++
+ *     exception crosses the ABI.  gpt2_last_error() gives a message.
+ *   - "device" pointers are CUDA device (or managed) addresses on the device
+ *     that was current at gpt2_create; "host" pointers are CPU addresses
+ *     (pinned or pageable).  The caller keeps ownership of every pointer it
+ *     passes; the library never frees them.
+ *   - Work is enqueued on the caller's stream (gpt2_config.stream) and is
+ *     asynchronous, except where a host scalar is returned (loss, grad norm)
+ *     or a host buffer is read/written: those calls synchronise that stream.
+ *   - Matrices are row-major.  Linear weights are [out, in] and a linear
+ *     layer computes y = x W^T + b.
+ *   - Not thread-safe: one handle is used by one host thread at a time.
+ */
+#ifndef GPT2_B200_H
+#define GPT2_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status */
+#define GPT2_OK 0
+#define GPT2_ERR_ARG 1          /* bad config/argument, size above capacity */
+#define GPT2_ERR_TOKEN 2        /* a token or target id outside [0, vocab_size) */
+#define GPT2_ERR_NONFINITE 3    /* non-finite loss or gradient norm: update skipped */
+#define GPT2_ERR_CUDA 4         /* a CUDA runtime call failed */
+#define GPT2_ERR_OOM 5          /* device allocation failed */
+#define GPT2_ERR_TIMEOUT 6      /* a bounded device wait gave up (kernel reported it) */
+#define GPT2_ERR_STATE 7        /* calls out of order (e.g. backward without forward) */
+
+/* tensor selectors for gpt2_get_tensor / gpt2_set_tensor */
+#define GPT2_PARAM 0            /* fp32 master weights */
+#define GPT2_GRAD 1             /* fp32 gradients */
+#define GPT2_ADAM_M 2           /* fp32 first moment */
+#define GPT2_ADAM_V 3           /* fp32 second moment */
+
+/* element types of op-level buffers */
+#define GPT2_F32 0
+#define GPT2_BF16 1
+
+typedef struct gpt2_handle gpt2_handle;
+
+/* Device allocator hooks: when alloc is non-NULL every device buffer the
+ * handle owns comes from alloc(bytes, ctx) and goes back through
+ * free(ptr, ctx) (e.g. PyTorch's caching allocator); otherwise cudaMalloc. */
+typedef void* (*gpt2_alloc_fn)(size_t bytes, void* ctx);
+typedef void (*gpt2_free_fn)(void* ptr, void* ctx);
+
+typedef struct {
+  int n_layer;       /* L  (12 for GPT-2 124M) */
+  int n_embd;        /* C  (768); must be a multiple of n_head and of 8 */
+  int n_head;        /* H  (12); head size D = C/H must be 16, 32, 64 or 128 */
+  int vocab_size;    /* V  (50257): ids a token or target may take */
+  int padded_vocab;  /* Vp >= V (50304): rows of the tied matrix; the extra
+                        rows are real columns of the output softmax [LECTURE:
+                        vocabulary padding] */
+  int max_T;         /* rows of the position-embedding matrix (1024) */
+  int bf16;          /* 1: bf16 GEMM operands and activations with fp32
+                        accumulation, statistics, loss, gradients, master
+                        weights and Adam state [LECTURE: mixed precision];
+                        0: fp32 everywhere (parity mode, SIMT kernels) */
+  float ln_eps;      /* LayerNorm epsilon (1e-5) */
+  int max_B;         /* activation capacity: every call needs B <= max_B ... */
+  int max_Tseq;      /* ... and T <= max_Tseq <= max_T */
+  int resid_init_scale; /* reserved, must be 0 (initial values come from the caller) */
+  void* stream;      /* cudaStream_t owned by the caller; NULL = default stream */
+  gpt2_alloc_fn alloc; /* optional device allocator, see above */
+  gpt2_free_fn free;
+  void* alloc_ctx;
+} gpt2_config;
+
+/* ---------------------------------------------------------------- handle */
+
+/* Creates a model: validates cfg, allocates the fp32 parameter, gradient and
+ * AdamW arenas (zeroed; parameters must then be set with gpt2_set_tensor),
+ * the bf16 weight mirrors and the activation/workspace memory for
+ * max_B x max_Tseq tokens.  *out receives the handle (NULL on failure; the
+ * message is then in gpt2_last_error(NULL)).  Adam's step counter starts at 0. */
+int gpt2_create(const gpt2_config* cfg, gpt2_handle** out);
+
+/* Synchronises the stream and frees everything the handle owns. */
+int gpt2_destroy(gpt2_handle* h);
+
+/* Last error message of h (or of the last failed gpt2_create when h is NULL).
+ * The string lives until the next call on h. */
+const char* gpt2_last_error(const gpt2_handle* h);
+
+/* Parameter tensors, in the order [LECTURE: module naming]:
+ *   wte [Vp,C], wpe [max_T,C], then for l in 0..L-1: h.l.ln1.w [C], h.l.ln1.b [C],
+ *   h.l.attn.qkv.w [3C,C], h.l.attn.qkv.b [3C], h.l.attn.proj.w [C,C],
+ *   h.l.attn.proj.b [C], h.l.ln2.w [C], h.l.ln2.b [C], h.l.mlp.fc.w [4C,C],
+ *   h.l.mlp.fc.b [4C], h.l.mlp.proj.w [C,4C], h.l.mlp.proj.b [C]; then
+ *   lnf.w [C], lnf.b [C].
+ * The QKV rows stack q, k, v; head h owns channels [hD, (h+1)D).
+ * decay = 1 for 2-D tensors (weight decay applies), 0 for vectors [LECTURE:
+ * weight decay on matrices, not on biases or other 1-D parameters].
+ * *name stays valid for the handle's lifetime; shape[1] = 1 for vectors. */
+int gpt2_num_tensors(const gpt2_handle* h, int* n);
+int gpt2_tensor_info(const gpt2_handle* h, int i, const char** name, int* ndim,
+                     int64_t shape[2], int* decay);
+int gpt2_param_count(const gpt2_handle* h, int64_t* n);
+
+/* Copies tensor i of the selected arena (GPT2_PARAM/GRAD/ADAM_M/ADAM_V) from /
+ * to a dense row-major fp32 buffer of the tensor's shape, on the host
+ * (on_device = 0; the call synchronises) or on the device (on_device = 1).
+ * Setting parameters refreshes the bf16 mirrors before the next forward.
+ * Reading GPT2_GRAD after gpt2_zero_grad returns zeros. */
+int gpt2_set_tensor(gpt2_handle* h, int i, int which, const float* src, int on_device);
+int gpt2_get_tensor(gpt2_handle* h, int i, int which, float* dst, int on_device);
+
+/* AdamW step counter t (number of updates done; the next update uses t+1). */
+int gpt2_get_step(const gpt2_handle* h, int* t);
+int gpt2_set_step(gpt2_handle* h, int t);
+
+/* ---------------------------------------------------------------- data */
+
+/* Cuts one batch from a device stream of uint16 token ids [CH28 §28.3]:
+ *   x[b,t] = stream[offset + b*T + t],  y[b,t] = stream[offset + b*T + t + 1]
+ * for b < B, t < T (B*T+1 consecutive ids; every row is its own causal
+ * window).  d_x, d_y are device int32 [B*T].  Needs offset >= 0 and
+ * offset + B*T + 1 <= stream_len, else GPT2_ERR_ARG.  Bit-exact. */
+int gpt2_batch_from_stream(gpt2_handle* h, const uint16_t* d_stream, int64_t stream_len,
+                           int64_t offset, int B, int T, int32_t* d_x, int32_t* d_y);
+
+/* ---------------------------------------------------------------- step */
+
+/* Forward pass and mean loss [ZERO: autoregressive objective]:
+ *   L = -1/(B*T) * sum_{b,t} log P(y[b,t] | x[b, 0..t])
+ * x, y: int32 [B*T] ids in [0, vocab_size), device (tokens_on_device = 1) or
+ * host (0; copied on the stream inside the call).  Saves the activations the
+ * backward needs.  loss_out (host, nullable): when given the call
+ * synchronises and writes L.  d_row_loss (device fp32 [B*T], nullable)
+ * receives the per-position losses.  An id out of range is caught on the
+ * device: the call (or the next synchronising call) returns GPT2_ERR_TOKEN
+ * and the next gpt2_clip_adamw_step is refused.  Needs 1 <= B <= max_B,
+ * 1 <= T <= max_Tseq. */
+int gpt2_forward_loss(gpt2_handle* h, const int32_t* x, const int32_t* y, int B, int T,
+                      int tokens_on_device, float* loss_out, float* d_row_loss);
+
+/* Backward pass of the last gpt2_forward_loss: adds grad_scale * dL/dtheta
+ * into the fp32 gradients (grad_scale = 1/accumulation steps for gradient
+ * accumulation [LECTURE: gradient accumulation]).  The tied matrix receives
+ * both the head and the embedding contributions.  GPT2_ERR_STATE if no
+ * forward with saved activations precedes it. */
+int gpt2_backward(gpt2_handle* h, float grad_scale);
+
+/* Sets every gradient to zero (lazily: the next backward overwrites). */
+int gpt2_zero_grad(gpt2_handle* h);
+
+/* Global-norm clipping and AdamW over every parameter, one fused pass
+ * [CS336 §2 AdamW, gradient clipping; ZERO: training loop]:
+ *   n = sqrt(sum g^2);  s = min(1, max_norm / (n + 1e-6));  g' = s*g;  t += 1
+ *   m = b1 m + (1-b1) g';  v = b2 v + (1-b2) g'^2
+ *   p *= 1 - lr*wd (decay tensors only)
+ *   p -= lr * sqrt(1-b2^t)/(1-b1^t) * m / (sqrt(v) + eps)
+ * then refreshes the bf16 mirrors.  The stored gradients are read, not
+ * rewritten.  grad_norm_out (host, nullable): the pre-clip n; when given the
+ * call synchronises.  A non-finite n, or a token error in the forward, leaves
+ * parameters, moments and t untouched (GPT2_ERR_NONFINITE / GPT2_ERR_TOKEN,
+ * reported by this call when it synchronises, else by gpt2_synchronize). */
+int gpt2_clip_adamw_step(gpt2_handle* h, float lr, float beta1, float beta2, float eps,
+                         float weight_decay, float max_norm, float* grad_norm_out);
+
+/* One whole step: zero_grad, forward_loss, backward(1), clip_adamw_step.
+ * loss_out / grad_norm_out (host, nullable) as above. */
+int gpt2_train_step(gpt2_handle* h, const int32_t* x, const int32_t* y, int B, int T,
+                    int tokens_on_device, float lr, float beta1, float beta2, float eps,
+                    float weight_decay, float max_norm, float* loss_out, float* grad_norm_out);
+
+/* Forward-only mean loss (no activations saved; the saved state of a
+ * previous forward is invalidated) [CH28 §28.4: validation loss].  loss_out
+ * (host) is required; the call synchronises. */
+int gpt2_eval_loss(gpt2_handle* h, const int32_t* x, const int32_t* y, int B, int T,
+                   int tokens_on_device, float* loss_out);
+
+/* Waits for the stream and reports a device-side error recorded since the
+ * last check (token range, non-finite norm, bounded-wait timeout). */
+int gpt2_synchronize(gpt2_handle* h);
+
+/* Raw device address and length (elements) of one fp32 arena (GPT2_PARAM,
+ * GPT2_GRAD, GPT2_ADAM_M, GPT2_ADAM_V).  The arena holds every tensor at its
+ * own 64-element aligned offset (the padding stays 0), so it can be handed as
+ * one buffer to a collective (e.g. a data-parallel gradient all-reduce) or a
+ * checkpoint writer.  The pointer is owned by the handle.  Reading GPT2_GRAD
+ * right after gpt2_zero_grad first materialises the zeros. */
+int gpt2_arena(gpt2_handle* h, int which, float** ptr, int64_t* n_elems);
+
+/* ---------------------------------------------------------------- profiling */
+/* Kernel groups timed by the built-in profiler. */
+#define GPT2_PROF_GEMM 0        /* linear-layer contractions (fwd, dX, dW) */
+#define GPT2_PROF_LMHEAD 1      /* tied-head contractions + cross-entropy rows */
+#define GPT2_PROF_ATTN_FWD 2
+#define GPT2_PROF_ATTN_BWD 3
+#define GPT2_PROF_LN_FWD 4
+#define GPT2_PROF_LN_BWD 5
+#define GPT2_PROF_EMBED 6       /* embedding forward and backward */
+#define GPT2_PROF_OPTIM 7       /* gradient norm + clip + AdamW */
+#define GPT2_PROF_OTHER 8       /* column sums, copies, loss mean */
+#define GPT2_PROF_NCAT 9
+
+/* When enabled, every kernel group the handle launches is bracketed by CUDA
+ * events on the handle's stream.  gpt2_profile_read synchronises and returns,
+ * for group `cat` since the last reset: launches (kernels), summed device
+ * time in ms, and the algorithmic FLOPs and HBM bytes of those launches
+ * (nullable outputs).  cat = -1 returns the total launch count of the handle
+ * (counted whether or not profiling is enabled). */
+int gpt2_profile_enable(gpt2_handle* h, int enable);
+int gpt2_profile_reset(gpt2_handle* h);
+int gpt2_profile_read(gpt2_handle* h, int cat, int64_t* launches, double* ms, double* flops,
+                      double* bytes);
+
+/* ---------------------------------------------------------------- ops */
+
+/* Tied LM head + mean cross-entropy alone [ZERO: output layer, fused
+ * projection + cross-entropy; LECTURE: tied head over the padded vocabulary]:
+ *   z = hidden W^T over all Vp rows; loss_m = logsumexp(z_m) - z_{m,y_m};
+ *   *d_loss = mean_m loss_m;  dz = grad_scale/M * (softmax(z) - onehot(y))
+ *   d_dh = dz W (overwritten), d_dw += dz^T hidden.
+ * hidden: [M,C], W: [Vp,C] of type `dtype` (GPT2_BF16 or GPT2_F32), device.
+ * y: device int32 [M] in [0, V).  d_loss: device fp32 [1].  d_lse (nullable):
+ * device fp32 [M] log-normalisers.  d_dh (nullable, same type as hidden) and
+ * d_dw (nullable, fp32 [Vp,C]) request the backward.  The [M,Vp] logits are
+ * never stored: at most a bounded row chunk lives in the workspace.
+ * workspace: device memory of at least gpt2_lmhead_ce_workspace() bytes.
+ * C must be a multiple of 64 for GPT2_BF16.  Asynchronous on `stream`. */
+int gpt2_lmhead_ce_workspace(int M, int C, int Vp, int dtype, size_t* bytes);
+int gpt2_lmhead_ce(const void* hidden, const void* W, const int32_t* y, int M, int C, int Vp,
+                   int V, int dtype, float grad_scale, float* d_loss, float* d_lse, void* d_dh,
+                   float* d_dw, void* workspace, size_t workspace_bytes, void* stream);
+
+/* LayerNorm forward over rows of x fp32 [M,C] (biased variance)
+ * [ZERO: Transformer Block]:  y = gamma*(x-mu)*rstd + beta, written as
+ * `y_dtype`; mean, rstd fp32 [M] (nullable).  Device buffers. */
+int gpt2_layernorm_fwd(const float* x, const float* gamma, const float* beta, int64_t M, int C,
+                       float eps, void* y, int y_dtype, float* mean, float* rstd, void* stream);
+
+/* LayerNorm backward: with xh = (x-mu)*rstd, dxh = dy*gamma,
+ *   dx += rstd*(dxh - mean(dxh) - xh*mean(dxh*xh)),
+ *   dgamma += sum_m dy*xh, dbeta += sum_m dy   (deterministic column sums).
+ * dy of type dy_dtype [M,C]; x, dx fp32 [M,C]; mean, rstd fp32 [M];
+ * gamma, dgamma, dbeta fp32 [C].  workspace >= gpt2_layernorm_bwd_workspace(). */
+int gpt2_layernorm_bwd_workspace(int64_t M, int C, size_t* bytes);
+int gpt2_layernorm_bwd(const void* dy, int dy_dtype, const float* x, const float* mean,
+                       const float* rstd, const float* gamma, int64_t M, int C, float* dx,
+                       float* dgamma, float* dbeta, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* Causal multi-head attention [ZERO: Attention; LECTURE: causal attention]:
+ * qkv [B,T,3C] (q | k | v, head h = channels [hD,(h+1)D)) of type `dtype`;
+ * out [B,T,C] = per head softmax(q k^T / sqrt(D) with j > i excluded) v;
+ * lse fp32 [B,H,T] = the softmax log-normaliser of each row (for the backward).
+ * The [B,H,T,T] scores are never stored. */
+int gpt2_attention_fwd(const void* qkv, int dtype, int B, int T, int C, int H, void* out,
+                       float* lse, void* stream);
+
+/* Backward of gpt2_attention_fwd: dqkv [B,T,3C] (overwritten) from dout
+ * [B,T,C], qkv, out and lse of the forward.  workspace >=
+ * gpt2_attention_bwd_workspace(). */
+int gpt2_attention_bwd_workspace(int B, int T, int C, int H, int dtype, size_t* bytes);
+int gpt2_attention_bwd(const void* dout, const void* qkv, const void* out, const float* lse,
+                       int dtype, int B, int T, int C, int H, void* dqkv, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Dense contraction used by every linear layer (no counterpart on the pages
+ * beyond "linear layer"; exported so it can be tested alone):
+ *   D[m,n] = alpha * sum_k A(m,k) B(n,k)  (+ beta_accumulate * D[m,n] when
+ *   accumulate = 1; D fp32 then)
+ * A(m,k) = A[m*lda + k] when a_kmajor, else A[k*lda + m]; B likewise with ldb.
+ * A, B of type `dtype`; D of type d_dtype (fp32, or bf16 when accumulate = 0).
+ * workspace >= gpt2_matmul_workspace() (split-K partial sums). */
+int gpt2_matmul_workspace(int M, int N, int K, size_t* bytes);
+int gpt2_matmul(const void* A, int a_kmajor, int64_t lda, const void* B, int b_kmajor, int64_t ldb,
+                int dtype, int M, int N, int K, float alpha, int accumulate, void* D, int d_dtype,
+                int64_t ldd, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Reads and clears the device error word shared by the op-level calls
+ * (bounded-wait timeouts).  *code = GPT2_OK when nothing was recorded.
+ * Synchronises the device. */
+int gpt2_device_error(int* code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT2_B200_H */

@@ -1,0 +1,78 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/gpt2.h declares, the binding covers them, and host-side validation
+rejects bad configurations before any device call."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gpt2.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gpt2_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def g():
+    import decoder_only_lm_b200 as g
+    return g
+
+
+def test_header_declares_the_step_entry_points():
+    names = declared_functions()
+    for n in ("gpt2_create", "gpt2_forward_loss", "gpt2_backward", "gpt2_clip_adamw_step",
+              "gpt2_eval_loss", "gpt2_batch_from_stream", "gpt2_lmhead_ce"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(g):
+    out = subprocess.run(["nm", "-D", "--defined-only", g.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (gpt2_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    # and nothing with C linkage beyond the header
+    assert exported <= set(declared_functions())
+
+
+def test_binding_covers_the_header(g):
+    assert set(g.SIGNATURES) == set(declared_functions())
+    for n in declared_functions():
+        assert callable(getattr(g, n))
+
+
+def _cfg(g, **kw):
+    base = dict(n_layer=2, n_embd=64, n_head=4, vocab_size=512, padded_vocab=512, max_T=64, bf16=0,
+                ln_eps=1e-5, max_B=4, max_Tseq=32, resid_init_scale=0, stream=None)
+    base.update(kw)
+    c = g.Config()
+    for k, v in base.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("bad", [dict(n_embd=66), dict(n_head=5), dict(padded_vocab=500),
+                                 dict(max_Tseq=128), dict(ln_eps=0.0), dict(n_layer=0),
+                                 dict(n_embd=256, n_head=2), dict(resid_init_scale=1)])
+def test_create_rejects_bad_config_on_the_host(g, bad):
+    h = C.c_void_p()
+    rc = g.lib.gpt2_create(C.byref(_cfg(g, **bad)), C.byref(h))
+    assert rc == g.ERR_ARG and not h.value
+    assert g.lib.gpt2_last_error(None)
+
+
+def test_null_arguments_are_refused(g):
+    assert g.lib.gpt2_create(None, None) == g.ERR_ARG
+    assert g.lib.gpt2_backward(None, 1.0) == g.ERR_ARG
+    assert g.lib.gpt2_zero_grad(None) == g.ERR_ARG
+    ws = C.c_size_t()
+    assert g.lib.gpt2_lmhead_ce_workspace(0, 64, 64, g.BF16, C.byref(ws)) == g.ERR_ARG
+    assert g.lib.gpt2_lmhead_ce_workspace(128, 768, 50304, g.BF16, C.byref(ws)) == g.OK
+    assert ws.value > 128 * 50304 * 4  # holds one bounded chunk of logits, not all of them
+    assert ws.value < 8192 * 50304 * 2  # ... and less than the full [8192, 50304] bf16 logits

@@ -1,0 +1,208 @@
+"""GPU path vs the CPU oracle, through the C ABI, on seeded inputs.
+
+Bars: bit-exact for slicing; fp32 mode loss within 1e-4 nats and per-tensor
+gradient (and AdamW update) relative L2 within 1e-3; bf16 mode 2e-2 nats and
+3e-2.  The oracle runs in float64.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.parity_util import RAGGED, TINY, TOL, gpu_model, inputs, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+HP = dict(lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, max_norm=1.0)
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch
+    assert torch.cuda.is_available()
+    return torch
+
+
+def run_both(shape, bf16, torch, grad_scale=1.0):
+    om, named, stream, x, y = inputs(shape)
+    gm = gpu_model(shape, bf16)
+    gm.set_params(named)
+    flat = om.pack(named)
+    loss_o, rl_o, g_o, _ = om.fwd_bwd(flat, x, y, row_loss=True, grad_scale=grad_scale)
+    rl = torch.empty(shape.B * shape.T, dtype=torch.float32, device="cuda")
+    gm.zero_grad()
+    loss_g = gm.forward_loss(torch.from_numpy(x).cuda(), torch.from_numpy(y).cuda(), row_loss=rl)
+    gm.backward(grad_scale)
+    gm.synchronize()
+    return om, gm, named, flat, (loss_o, rl_o, g_o), (loss_g, rl.cpu().numpy(), x, y)
+
+
+@pytest.mark.parametrize("shape", [TINY, RAGGED], ids=["tiny", "ragged"])
+@pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
+def test_step_matches_oracle(shape, bf16, torch):
+    tol = TOL[bf16]
+    om, gm, named, flat, (lo, rlo, go), (lg, rlg, x, y) = run_both(shape, bf16, torch)
+    assert abs(lg - lo) <= tol["loss"], (lg, lo)
+    assert np.max(np.abs(rlg - rlo)) <= 10 * tol["loss"]
+    G = om.unpack(go)
+    for name, shp in om.shapes():
+        gg = gm.get_tensor(name, which=1)
+        assert rel_l2(gg, G[name]) <= tol["grad"], (name, rel_l2(gg, G[name]))
+    # one clip + AdamW step: compare the parameter updates
+    norm_g = gm.clip_adamw_step(**HP)
+    p_o, m_o, v_o = flat.copy(), np.zeros_like(flat), np.zeros_like(flat)
+    norm_o = om.clip_adamw(p_o, go, m_o, v_o, 1, HP["lr"], HP["beta1"], HP["beta2"], HP["eps"],
+                           HP["weight_decay"], HP["max_norm"])
+    assert abs(norm_g - norm_o) <= tol["grad"] * norm_o
+    P_o = om.unpack(p_o)
+    for name, shp in om.shapes():
+        pg = gm.get_tensor(name).astype(np.float64)
+        d_g = pg - named[name].astype(np.float64)
+        d_o = P_o[name] - named[name].astype(np.float64)
+        # Adam normalises each element's step: elements whose gradient is at the
+        # rounding level of the comparison may flip sign, so the bar is on the
+        # update as a whole.
+        assert rel_l2(d_g, d_o) <= max(tol["grad"], 0.05 if bf16 else 2e-3), name
+    assert gm.step == 1
+
+
+def test_batch_slicing_bit_exact(torch):
+    import decoder_only_lm_b200 as g
+    gm = gpu_model(TINY, False)
+    s = synth.token_stream(5, 50_000)
+    ds = torch.from_numpy(s.astype(np.int16).view(np.int16)).cuda()
+    for off, B, T in [(0, 4, 32), (12345, 3, 17), (50_000 - 4 * 32 - 1, 4, 32)]:
+        x, y = gm.batch_from_stream(ds, off, B, T)
+        xo, yo = oracle.batch_from_stream(s, off, B, T)
+        assert np.array_equal(x.cpu().numpy(), xo) and np.array_equal(y.cpu().numpy(), yo)
+    with pytest.raises(g.GPT2Error):
+        gm.batch_from_stream(ds, 50_000 - 4 * 32, 4, 32)
+
+
+def test_ln_vocab_at_zero_logits(torch):
+    om, named, stream, x, y = inputs(TINY)
+    named["wte"][:] = 0
+    for bf16 in (False, True):
+        gm = gpu_model(TINY, bf16)
+        gm.set_params(named)
+        loss = gm.forward_loss(x, y)  # host tokens
+        assert abs(loss - math.log(512)) < (1e-5 if not bf16 else 1e-3)
+
+
+def test_causal_invariance_gpu(torch):
+    om, named, stream, x, y = inputs(TINY)
+    gm = gpu_model(TINY, True)
+    gm.set_params(named)
+    rl1 = torch.empty(TINY.B * TINY.T, device="cuda")
+    rl2 = torch.empty_like(rl1)
+    gm.forward_loss(x, y, row_loss=rl1)
+    x2, y2 = x.copy(), y.copy()
+    x2[:, 20:] = (x2[:, 20:] + 7) % 512
+    y2[:, 20:] = (y2[:, 20:] + 3) % 512
+    gm.forward_loss(x2, y2, row_loss=rl2)
+    keep = (np.arange(TINY.B * TINY.T) % TINY.T) < 20
+    a, b = rl1.cpu().numpy(), rl2.cpu().numpy()
+    assert np.array_equal(a[keep], b[keep]) and not np.array_equal(a[~keep], b[~keep])
+
+
+def test_deterministic(torch):
+    outs = []
+    for _ in range(2):
+        om, gm, *_ = run_both(RAGGED, True, torch)
+        outs.append({n: gm.get_tensor(n, which=1) for n, _ in om.shapes()})
+    for n in outs[0]:
+        assert np.array_equal(outs[0][n], outs[1][n]), n
+
+
+@pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
+def test_gradient_accumulation(bf16, torch):
+    om, named, stream, x, y = inputs(TINY)
+    gm = gpu_model(TINY, bf16)
+    gm.set_params(named)
+    gm.zero_grad()
+    gm.forward_loss(x, y, loss=False)
+    gm.backward(1.0)
+    full = {n: gm.get_tensor(n, which=1) for n, _ in om.shapes()}
+    gm.zero_grad()
+    for half in (slice(0, 2), slice(2, 4)):
+        gm.forward_loss(x[half], y[half], loss=False)
+        gm.backward(0.5)
+    for n, _ in om.shapes():
+        assert rel_l2(gm.get_tensor(n, which=1), full[n]) <= (1e-5 if not bf16 else 1e-2), n
+
+
+def test_backward_needs_forward(torch):
+    import decoder_only_lm_b200 as g
+    gm = gpu_model(TINY, True)
+    with pytest.raises(g.GPT2Error) as e:
+        gm.backward()
+    assert e.value.code == g.ERR_STATE
+
+
+def test_token_out_of_range_refused(torch):
+    import decoder_only_lm_b200 as g
+    om, named, stream, x, y = inputs(TINY)
+    gm = gpu_model(TINY, True)
+    gm.set_params(named)
+    x = x.copy()
+    x[2, 5] = 512
+    with pytest.raises(g.GPT2Error) as e:
+        gm.forward_loss(x, y)
+    assert e.value.code == g.ERR_TOKEN
+    # a forward with a bad id, then backward + step: the step is refused
+    gm.zero_grad()
+    gm.forward_loss(x, y, loss=False)
+    gm.backward()
+    with pytest.raises(g.GPT2Error) as e:
+        gm.clip_adamw_step(**HP)
+    assert e.value.code == g.ERR_TOKEN
+    assert np.array_equal(gm.get_tensor("h.0.mlp.fc.w"), named["h.0.mlp.fc.w"])
+    assert gm.step == 0
+
+
+def test_nonfinite_gradient_skips_update(torch):
+    import decoder_only_lm_b200 as g
+    om, named, stream, x, y = inputs(TINY)
+    gm = gpu_model(TINY, True)
+    gm.set_params(named)
+    gm.zero_grad()
+    gm.forward_loss(x, y, loss=False)
+    gm.backward()
+    bad = gm.get_tensor("h.1.attn.qkv.b", which=1)
+    bad[3] = np.nan
+    gm.set_tensor("h.1.attn.qkv.b", bad, which=1)
+    with pytest.raises(g.GPT2Error) as e:
+        gm.clip_adamw_step(**HP)
+    assert e.value.code == g.ERR_NONFINITE
+    for n in ("wte", "h.0.ln1.w", "lnf.b"):
+        assert np.array_equal(gm.get_tensor(n), named[n])
+    assert gm.step == 0
+    # the handle stays usable
+    gm.zero_grad()
+    gm.forward_loss(x, y, loss=False)
+    gm.backward()
+    assert math.isfinite(gm.clip_adamw_step(**HP)) and gm.step == 1
+
+
+def test_eval_loss_matches_forward(torch):
+    om, named, stream, x, y = inputs(RAGGED)
+    gm = gpu_model(RAGGED, True)
+    gm.set_params(named)
+    a = gm.forward_loss(x, y)
+    b = gm.eval_loss(x, y)
+    assert a == b
+    lo = om.fwd_bwd(om.pack(named), x, y, grads=False)[0]
+    assert abs(b - lo) <= TOL[True]["loss"]
+
+
+def test_overfit_one_batch_gpu(torch):
+    om, named, stream, x, y = inputs(TINY)
+    gm = gpu_model(TINY, True)
+    gm.set_params(named)
+    first = None
+    for _ in range(30):
+        loss, norm = gm.train_step(x, y, lr=3e-3)
+        first = first if first is not None else loss
+    assert loss < 0.5 * first
