@@ -63,7 +63,6 @@ struct LayerOff {
 };
 
 constexpr int64_t kAlign = 64;  // elements (256 B of fp32)
-constexpr int kLmChunk = 2048;  // rows of logits held at once by the tied head
 
 int64_t align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
@@ -92,8 +91,8 @@ struct gpt2_handle {
   float* dres = nullptr;
   void *dres_a = nullptr, *dln = nullptr, *datt = nullptr, *dqkv = nullptr, *du = nullptr,
        *dhf = nullptr;
-  float* zchunk = nullptr;
-  void* dzchunk = nullptr;
+  void* lm_ws = nullptr;
+  size_t lm_ws_bytes = 0;
   float* ws = nullptr;
   size_t ws_bytes = 0;
   void* ws_emb = nullptr;
@@ -428,15 +427,10 @@ int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save) {
                                      h->muf, h->rsf, M, C, h->cfg.ln_eps, h->st));
   }
   {
-    // tied head + cross-entropy, one bounded chunk of logit rows at a time
+    // tied head + cross-entropy: no logits are stored (see lmhead_fwd)
     PROF(GPT2_PROF_LMHEAD, gemm_flops(M, Vp, C), a * (M * C + double(Vp) * C) + 8.0 * M);
-    for (int64_t r0 = 0; r0 < M; r0 += kLmChunk) {
-      const int mc = int(std::min<int64_t>(kLmChunk, M - r0));
-      EpiParams e = epi(EPI_STORE, h->zchunk, Vp, 0);
-      H_TRY(h, gemm(h, hf + r0 * C, 1, C, wptr(h, h->off_wte), 1, C, mc, Vp, C, e));
-      H_TRY(h, launch_ce_rows_fwd(h->zchunk, h->ybuf + r0, mc, Vp, h->hlse + r0,
-                                  h->row_loss + r0, h->st));
-    }
+    H_TRY(h, lmhead_fwd(hf, wptr(h, h->off_wte), h->ybuf, int(M), C, Vp, h->use_bf16, h->hlse,
+                        h->row_loss, h->lm_ws, h->lm_ws_bytes, h->st));
   }
   {
     PROF(GPT2_PROF_OTHER, 0, 4.0 * M);
@@ -472,18 +466,8 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     // (algorithmic work: the dH and dW contractions; the logits are recomputed)
     PROF(GPT2_PROF_LMHEAD, 2 * gemm_flops(M, Vp, C),
          a * (2.0 * M * C + double(Vp) * C) + 8.0 * double(Vp) * C);
-    for (int64_t r0 = 0; r0 < M; r0 += kLmChunk) {
-      const int mc = int(std::min<int64_t>(kLmChunk, M - r0));
-      EpiParams e = epi(EPI_STORE, h->zchunk, Vp, 0);
-      H_TRY(h, gemm(h, hf + r0 * C, 1, C, wptr(h, h->off_wte), 1, C, mc, Vp, C, e));
-      H_TRY(h, launch_ce_rows_bwd<A>(h->zchunk, h->hlse + r0, h->ybuf + r0, mc, Vp, scale,
-                                     static_cast<A*>(h->dzchunk), h->st));
-      e = epi(EPI_STORE, dhf + r0 * C, C, ab);
-      H_TRY(h, gemm(h, h->dzchunk, 1, Vp, wptr(h, h->off_wte), 0, C, mc, C, Vp, e));
-      e = epi(EPI_ACC, G + h->off_wte, C, 0);
-      e.accumulate = (acc || r0 > 0) ? 1 : 0;
-      H_TRY(h, gemm(h, h->dzchunk, 0, Vp, hf + r0 * C, 0, C, Vp, C, mc, e));
-    }
+    H_TRY(h, lmhead_bwd(hf, wptr(h, h->off_wte), h->ybuf, h->hlse, int(M), C, Vp, h->use_bf16,
+                        scale, dhf, G + h->off_wte, acc, h->lm_ws, h->lm_ws_bytes, h->st));
   }
   A* copy = ab ? dres_a : nullptr;
   const double lnb_bytes = M * C * (4.0 + 8.0 + 2.0 * a) + 8.0 * M;
@@ -679,17 +663,15 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
   h->dqkv = A(M * 3 * C * a);
   h->du = A(M * F * a);
   h->dhf = A(M * C * a);
-  const int64_t mc = std::min<int64_t>(kLmChunk, M);
-  h->zchunk = static_cast<float*>(A(mc * Vp * sizeof(float)));
-  h->dzchunk = A(mc * Vp * a);
+  h->lm_ws_bytes = lmhead_workspace(int(M), int(C), int(Vp), h->use_bf16);
+  h->lm_ws = A(h->lm_ws_bytes);
   // general fp32 workspace: max of every user's need
   size_t ws = 0;
   ws = std::max(ws, layernorm_bwd_workspace(M, int(C)));
   ws = std::max(ws, colsum_workspace(M, int(std::max(F, 3 * C))));
   ws = std::max(ws, attn_bwd_workspace(c.max_B, c.max_Tseq, H));
-  const int shapes[][3] = {{int(C), int(F), int(M)},     {int(F), int(C), int(M)},
-                           {int(C), int(C), int(M)},     {int(3 * C), int(C), int(M)},
-                           {int(Vp), int(C), int(mc)}};
+  const int shapes[][3] = {{int(C), int(F), int(M)}, {int(F), int(C), int(M)},
+                           {int(C), int(C), int(M)}, {int(3 * C), int(C), int(M)}};
   for (auto& s : shapes) ws = std::max(ws, gemm_workspace_bytes(s[0], s[1], s[2]));
   h->ws_bytes = ws;
   h->ws = static_cast<float*>(A(ws));

@@ -18,34 +18,6 @@ using gpt2_internal::set_error;
 
 namespace {
 
-constexpr int kLmChunk = 2048;
-
-struct Carve {
-  char* p;
-  size_t left;
-  bool ok = true;
-  void* take(size_t bytes) {
-    bytes = (bytes + 255) / 256 * 256;
-    if (bytes > left) {
-      ok = false;
-      return nullptr;
-    }
-    void* r = p;
-    p += bytes;
-    left -= bytes;
-    return r;
-  }
-};
-
-size_t lm_ws(int M, int C, int Vp, int dtype) {
-  const int mc = std::min(kLmChunk, M);
-  const size_t a = dtype == GPT2_BF16 ? 2 : 4;
-  auto r = [](size_t b) { return (b + 255) / 256 * 256; };
-  size_t gw = std::max({gemm_workspace_bytes(mc, Vp, C), gemm_workspace_bytes(mc, C, Vp),
-                        gemm_workspace_bytes(Vp, C, mc)});
-  return r(size_t(mc) * Vp * 4) + r(size_t(mc) * Vp * a) + 2 * r(size_t(M) * 4) + r(gw) + 256;
-}
-
 __device__ int g_op_error;  // bounded-wait timeouts of op-level launches
 
 }  // namespace
@@ -66,8 +38,9 @@ int* device_error_word() {
 extern "C" {
 
 int gpt2_lmhead_ce_workspace(int M, int C, int Vp, int dtype, size_t* bytes) {
-  if (!bytes || M < 1 || C < 1 || Vp < 1) return GPT2_ERR_ARG;
-  *bytes = lm_ws(M, C, Vp, dtype);
+  if (!bytes || M < 1 || C < 1 || Vp < 1 || (dtype != GPT2_BF16 && dtype != GPT2_F32))
+    return GPT2_ERR_ARG;
+  *bytes = lmhead_workspace(M, C, Vp, dtype == GPT2_BF16) + 2 * ((size_t(M) * 4 + 255) / 256 * 256);
   return GPT2_OK;
 }
 
@@ -79,64 +52,26 @@ int gpt2_lmhead_ce(const void* hidden, const void* W, const int32_t* y, int M, i
     set_error("lmhead_ce: bad arguments");
     return GPT2_ERR_ARG;
   }
-  if (!workspace || workspace_bytes < lm_ws(M, C, Vp, dtype)) {
+  size_t need = 0;
+  gpt2_lmhead_ce_workspace(M, C, Vp, dtype, &need);
+  if (!workspace || workspace_bytes < need) {
     set_error("lmhead_ce: workspace too small");
     return GPT2_ERR_ARG;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int bf = dtype == GPT2_BF16;
-  const size_t a = bf ? 2 : 4;
-  const int mc_max = std::min(kLmChunk, M);
-  Carve cv{static_cast<char*>(workspace), workspace_bytes};
-  float* z = static_cast<float*>(cv.take(size_t(mc_max) * Vp * 4));
-  void* dz = cv.take(size_t(mc_max) * Vp * a);
-  float* lse = d_lse ? d_lse : static_cast<float*>(cv.take(size_t(M) * 4));
-  float* rl = static_cast<float*>(cv.take(size_t(M) * 4));
-  size_t gw = std::max({gemm_workspace_bytes(mc_max, Vp, C), gemm_workspace_bytes(mc_max, C, Vp),
-                        gemm_workspace_bytes(Vp, C, mc_max)});
-  float* gws = static_cast<float*>(cv.take(gw));
-  if (!cv.ok) {
-    set_error("lmhead_ce: workspace too small");
-    return GPT2_ERR_ARG;
-  }
-  const bool bwd = d_dh || d_dw;
-  const float scale = grad_scale / float(M);
-  for (int64_t r0 = 0; r0 < M; r0 += kLmChunk) {
-    const int mc = int(std::min<int64_t>(kLmChunk, M - r0));
-    const void* hr = static_cast<const char*>(hidden) + r0 * C * int64_t(a);
-    EpiParams e;
-    e.kind = EPI_STORE;
-    e.out = z;
-    e.ldo = Vp;
-    GemmArgs g{hr, 1, C, W, 1, C, bf, mc, Vp, C, e, gws, gw};
-    int rc = gemm_launch(g, st);
+  char* w = static_cast<char*>(workspace);
+  const size_t rows = (size_t(M) * 4 + 255) / 256 * 256;
+  float* lse = d_lse ? d_lse : reinterpret_cast<float*>(w);
+  float* rl = reinterpret_cast<float*>(w + rows);
+  void* lw = w + 2 * rows;
+  const size_t lw_bytes = workspace_bytes - 2 * rows;
+  int rc = lmhead_fwd(hidden, W, y, M, C, Vp, bf, lse, rl, lw, lw_bytes, st);
+  if (rc) return rc;
+  if (d_dh || d_dw) {
+    rc = lmhead_bwd(hidden, W, y, lse, M, C, Vp, bf, grad_scale / float(M), d_dh, d_dw, 1, lw,
+                    lw_bytes, st);
     if (rc) return rc;
-    rc = launch_ce_rows_fwd(z, y + r0, mc, Vp, lse + r0, rl + r0, st);
-    if (rc) return rc;
-    if (!bwd) continue;
-    rc = bf ? launch_ce_rows_bwd<bf16>(z, lse + r0, y + r0, mc, Vp, scale, static_cast<bf16*>(dz), st)
-            : launch_ce_rows_bwd<float>(z, lse + r0, y + r0, mc, Vp, scale, static_cast<float*>(dz), st);
-    if (rc) return rc;
-    if (d_dh) {
-      EpiParams e2;
-      e2.kind = EPI_STORE;
-      e2.out = static_cast<char*>(d_dh) + r0 * C * int64_t(a);
-      e2.ldo = C;
-      e2.out_bf16 = bf;
-      GemmArgs g2{dz, 1, Vp, W, 0, C, bf, mc, C, Vp, e2, gws, gw};
-      rc = gemm_launch(g2, st);
-      if (rc) return rc;
-    }
-    if (d_dw) {
-      EpiParams e3;
-      e3.kind = EPI_ACC;
-      e3.out = d_dw;
-      e3.ldo = C;
-      e3.accumulate = 1;
-      GemmArgs g3{dz, 0, Vp, hr, 0, C, bf, Vp, C, mc, e3, gws, gw};
-      rc = gemm_launch(g3, st);
-      if (rc) return rc;
-    }
   }
   return launch_mean(rl, M, d_loss, st);
 }

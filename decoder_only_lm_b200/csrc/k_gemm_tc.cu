@@ -1,0 +1,658 @@
+// Tensor-core GEMM for sm_100a: tcgen05.mma (kind::f16, bf16 operands, fp32
+// accumulation in TMEM) fed by TMA, with the linear-layer epilogues fused.
+//
+//   D[m,n] = epilogue( sum_k A(m,k) B(n,k) )
+//
+// Design
+//   - persistent CTAs (one per SM), static round-robin over output tiles of
+//     128 x BN (BN = 256 or 128), m fastest so co-resident CTAs share B tiles;
+//   - warp-specialised: warp 0 issues TMA loads (one elected lane), warp 1
+//     issues tcgen05.mma (one elected lane), warp 2 owns the TMEM allocation,
+//     warps 4-7 (one warpgroup) drain the accumulator with tcgen05.ld and run
+//     the epilogue;
+//   - STAGES-deep shared-memory ring of (A, B) k-blocks of 64 elements with
+//     128-byte swizzle, full/empty mbarriers; two TMEM accumulators so the
+//     epilogue of tile i overlaps the MMAs of tile i+1;
+//   - operands may be K-major (rows of K contiguous) or MN-major (rows of M or
+//     N contiguous: the weight-gradient and transposed-weight contractions of
+//     the backward pass), described to the MMA by the smem descriptors;
+//   - split-K for weight gradients with few output tiles: split s writes its
+//     partial tile to a workspace, a reduction adds the splits in order;
+//   - every mbarrier wait is bounded by a global-timer budget: on expiry the
+//     kernel records a timeout in the error word, every role leaves its loop,
+//     in-flight copies and MMAs are waited for (again bounded) and TMEM is
+//     freed before the CTA exits.  No trap, no unbounded spin.
+//
+// No TMA multicast is used anywhere (each CTA loads its own tiles).
+
+#include <cuda.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "epilogue.cuh"
+
+namespace {
+
+constexpr int BM = 128, BK = 64, UMMA_K = 16;
+constexpr int kThreads = 256;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
+
+template <int BN>
+struct TcCfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = STAGES * STAGE + BAR_BYTES + 1024;
+};
+
+struct TcParams {
+  int M, N, K;
+  int a_mn, b_mn;
+  int tiles_m, tiles_n, splits, kb_per_split, num_kb, total_tiles;
+  EpiParams ep;
+  float* ws;
+  int* err;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait on one phase; false (and the error word set) on expiry.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int where) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try(bar, parity)) return true;
+    if (global_ns() - t0 > kTimeoutNs) {
+      atomicExch(err, where);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Shared-memory matrix descriptor (sm_100 format, version 1, 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return uint64_t((addr & 0x3FFFF) >> 4) | (uint64_t((lbo >> 4) & 0x3FFF) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+// K-major, 128-byte rows of 64 bf16 along K, 8-row swizzle atoms of 1024 B;
+// the k-th 16-element slice starts 32 B further.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int k) {
+  return smem_desc(tile + k * 32, 16, 1024);
+}
+// MN-major: chunks of 64 MN-elements x BK rows (8 KB) side by side (LBO), rows
+// of 128 B along MN, 8-row groups 1024 B apart (SBO); k-th slice 16 rows on.
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int k) {
+  return smem_desc(tile + k * 16 * 128, BK * 128, 1024);
+}
+
+// Instruction descriptor: kind::f16, bf16 A and B, fp32 D, M = 128, N = BN.
+template <int BN>
+__device__ __forceinline__ uint32_t idesc_bf16(int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) |
+         (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+}
+
+// ------------------------------------------------------------ vector helpers
+template <typename T>
+__device__ __forceinline__ void store32(T* p, const float (&v)[32]);
+template <>
+__device__ __forceinline__ void store32<float>(float* p, const float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4)
+    *reinterpret_cast<float4*>(p + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+}
+template <>
+__device__ __forceinline__ void store32<bf16>(bf16* p, const float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 8) {
+    uint4 u;
+    __nv_bfloat162 t0 = __floats2bfloat162_rn(v[j], v[j + 1]);
+    __nv_bfloat162 t1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
+    __nv_bfloat162 t2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]);
+    __nv_bfloat162 t3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
+    u.x = *reinterpret_cast<uint32_t*>(&t0);
+    u.y = *reinterpret_cast<uint32_t*>(&t1);
+    u.z = *reinterpret_cast<uint32_t*>(&t2);
+    u.w = *reinterpret_cast<uint32_t*>(&t3);
+    *reinterpret_cast<uint4*>(p + j) = u;
+  }
+}
+template <typename T>
+__device__ __forceinline__ void load32(const T* p, float (&v)[32]);
+template <>
+__device__ __forceinline__ void load32<float>(const float* p, float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    float4 f = *reinterpret_cast<const float4*>(p + j);
+    v[j] = f.x;
+    v[j + 1] = f.y;
+    v[j + 2] = f.z;
+    v[j + 3] = f.w;
+  }
+}
+template <>
+__device__ __forceinline__ void load32<bf16>(const bf16* p, float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 8) {
+    uint4 u = *reinterpret_cast<const uint4*>(p + j);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float2 f = __bfloat1622float2(h[q]);
+      v[j + 2 * q] = f.x;
+      v[j + 2 * q + 1] = f.y;
+    }
+  }
+}
+
+// Epilogue of 32 consecutive columns n .. n+31 of row m (all in range).
+template <int EPI, typename OutT>
+__device__ __forceinline__ void epi_chunk32(const EpiParams& e, int m, int n, float (&v)[32],
+                                            float row_lse, int row_tgt) {
+  const int64_t i = int64_t(m) * e.ldo + n;
+  if (EPI == EPI_STORE) {
+    if (e.bias) {
+      float b[32];
+      load32<float>(e.bias + n, b);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = v[j] * e.alpha + b[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
+    }
+    store32<OutT>(reinterpret_cast<OutT*>(e.out) + i, v);
+  } else if (EPI == EPI_GELU) {
+    float b[32];
+    load32<float>(e.bias + n, b);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = round_through<OutT>(v[j] + b[j]);
+    store32<OutT>(reinterpret_cast<OutT*>(e.out) + i, v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+    store32<OutT>(reinterpret_cast<OutT*>(e.out2) + i, v);
+  } else if (EPI == EPI_RESID) {
+    float r[32];
+    load32<float>(e.rin + i, r);
+    if (e.bias) {
+      float b[32];
+      load32<float>(e.bias + n, b);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] += b[j];
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] += r[j];
+    store32<float>(e.rout + i, v);
+  } else if (EPI == EPI_ACC) {
+    float* o = reinterpret_cast<float*>(e.out) + i;
+    if (e.accumulate) {
+      float r[32];
+      load32<float>(o, r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = r[j] + e.alpha * v[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
+    }
+    store32<float>(o, v);
+  } else if (EPI == EPI_GELU_BWD) {
+    float u[32];
+    load32<OutT>(reinterpret_cast<const OutT*>(e.aux) + i, u);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] *= gelu_tanh_grad(u[j]);
+    store32<OutT>(reinterpret_cast<OutT*>(e.out) + i, v);
+  } else if (EPI == EPI_CE_GRAD) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = e.ce_scale * (__expf(v[j] - row_lse) - (n + j == row_tgt ? 1.f : 0.f));
+    store32<OutT>(reinterpret_cast<OutT*>(e.out) + i, v);
+  }
+}
+
+template <int BN, int EPI, typename OutT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
+                   const __grid_constant__ CUtensorMap tma_b, const TcParams p) {
+  using Cfg = TcCfg<BN>;
+  constexpr int S = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cfg::STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  const uint32_t sbase = smem_u32(smem);
+  auto full = [&](int s) { return smem_u32(bars + s); };
+  auto empty = [&](int s) { return smem_u32(bars + S + s); };
+  auto tfull = [&](int a) { return smem_u32(bars + 2 * S + a); };
+  auto tempty = [&](int a) { return smem_u32(bars + 2 * S + 2 + a); };
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), 128);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 2) tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.total_tiles && ok; tile += gridDim.x) {
+      const int tm = tile % p.tiles_m;
+      const int rest = tile / p.tiles_m;
+      const int tn = rest % p.tiles_n, sp = rest / p.tiles_n;
+      const int kb0 = sp * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(empty(stage), phase ^ 1, p.err, 1)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(full(stage), Cfg::STAGE);
+        const uint32_t sa = sbase + stage * Cfg::STAGE, sb = sa + Cfg::A_BYTES;
+        const int k0 = kb * BK;
+        if (!p.a_mn) {
+          tma_load_2d(sa, &tma_a, full(stage), k0, tm * BM);
+        } else {
+          tma_load_2d(sa, &tma_a, full(stage), tm * BM, k0);
+          tma_load_2d(sa + BK * 128, &tma_a, full(stage), tm * BM + 64, k0);
+        }
+        if (!p.b_mn) {
+          tma_load_2d(sb, &tma_b, full(stage), k0, tn * BN);
+        } else {
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_2d(sb + j * BK * 128, &tma_b, full(stage), tn * BN + 64 * j, k0);
+        }
+        ++issued;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    // wait until the copies of the last (up to S) issued stages have landed
+    for (int q = 1; q <= min(issued, S); ++q) {
+      const int idx = issued - q;
+      mbar_wait(full(idx % S), uint32_t((idx / S) & 1), p.err, 5);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------ MMA issuer
+    const uint32_t idesc = idesc_bf16<BN>(p.a_mn, p.b_mn);
+    int stage = 0;
+    uint32_t phase = 0;
+    int t_local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.total_tiles && ok; tile += gridDim.x, ++t_local) {
+      const int rest = tile / p.tiles_m;
+      const int sp = rest / p.tiles_n;
+      const int kb0 = sp * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+      const int acc = t_local & 1;
+      if (!mbar_wait(tempty(acc), ((t_local >> 1) & 1) ^ 1, p.err, 2)) break;
+      tc_fence_after();
+      const uint32_t d = tmem_base + uint32_t(acc * BN);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(full(stage), phase, p.err, 3)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = sbase + stage * Cfg::STAGE, sb = sa + Cfg::A_BYTES;
+#pragma unroll
+        for (int k = 0; k < BK / UMMA_K; ++k) {
+          const uint64_t ad = p.a_mn ? desc_mnmajor(sa, k) : desc_kmajor(sa, k);
+          const uint64_t bd = p.b_mn ? desc_mnmajor(sb, k) : desc_kmajor(sb, k);
+          umma_bf16(d, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(empty(stage));
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      umma_commit(tfull(acc));
+    }
+    // all issued MMAs complete before TMEM is released
+    if (t_local > 0) {
+      const int last = t_local - 1;
+      mbar_wait(tfull(last & 1), uint32_t((last >> 1) & 1), p.err, 6);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------ epilogue warpgroup
+    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    int t_local = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++t_local) {
+      const int tm = tile % p.tiles_m;
+      const int rest = tile / p.tiles_m;
+      const int tn = rest % p.tiles_n, sp = rest / p.tiles_n;
+      const int acc = t_local & 1;
+      bool ok = mbar_wait(tfull(acc), (t_local >> 1) & 1, p.err, 4);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int m = tm * BM + q * 32 + lane;
+      float row_lse = 0.f;
+      int row_tgt = -1;
+      if ((EPI == EPI_CE_GRAD || EPI == EPI_LSE_PARTIAL) && m < p.M) {
+        if (EPI == EPI_CE_GRAD) row_lse = p.ep.lse[m];
+        row_tgt = p.ep.tgt[m];
+      }
+      float run_m = -INFINITY, run_s = 0.f, zt = 0.f;
+      bool has_t = false;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        __syncwarp();
+        float v[32];
+        tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c0), v);
+        const int n = tn * BN + c0;
+        if (m >= p.M || n >= p.N) continue;
+        if (EPI == EPI_LSE_PARTIAL) {
+          // running max / sum of exp over this tile's valid columns
+          float cm = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (n + j < p.N) cm = fmaxf(cm, v[j]);
+          const float nm = fmaxf(run_m, cm);
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (n + j < p.N) s += __expf(v[j] - nm);
+          run_s = run_s * __expf(run_m - nm) + s;
+          run_m = nm;
+          if (row_tgt >= n && row_tgt < n + 32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j == row_tgt) zt = v[j];
+            has_t = true;
+          }
+          continue;
+        }
+        const int nc = min(32, p.N - n);
+        if (p.ws) {
+          float* w = p.ws + (int64_t(sp) * p.M + m) * p.N + n;
+          if (nc == 32 && (p.N & 3) == 0) {
+            store32<float>(w, v);
+          } else {
+            for (int j = 0; j < nc; ++j) w[j] = v[j];
+          }
+        } else if (nc == 32) {
+          epi_chunk32<EPI, OutT>(p.ep, m, n, v, row_lse, row_tgt);
+        } else {
+          for (int j = 0; j < nc; ++j) epi_apply<OutT>(p.ep, EPI, m, n + j, v[j]);
+        }
+      }
+      if (EPI == EPI_LSE_PARTIAL && m < p.M) {
+        p.ep.part_max[int64_t(m) * p.ep.part_ld + tn] = run_m;
+        p.ep.part_sum[int64_t(m) * p.ep.part_ld + tn] = run_s;
+        if (has_t) p.ep.tgt_logit[m] = zt;
+      }
+      tc_fence_before();
+      mbar_arrive(tempty(acc));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+__global__ void tc_splitk_reduce_kernel(const float* __restrict__ ws, int splits, int M, int N,
+                                        float* __restrict__ out, int64_t ldo, float alpha,
+                                        int accumulate) {
+  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= int64_t(M) * N) return;
+  const int m = int(i / N), n = int(i % N);
+  float acc = 0.f;
+  for (int z = 0; z < splits; ++z) acc += ws[int64_t(z) * M * N + i];
+  float* o = out + int64_t(m) * ldo + n;
+  *o = (accumulate ? *o : 0.f) + alpha * acc;
+}
+
+// ------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [outer, inner] view with row stride ld
+// (elements), box {64, box_outer}, 128-byte swizzle, zero fill out of range.
+bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
+              int box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(outer)};
+  cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
+  cuuint32_t box[2] = {64, cuuint32_t(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int choose_splits_tc(int tiles, int num_kb) {
+  const int sms = gpt2_internal::sm_count();
+  int s = 1;
+  while (tiles * s * 2 <= sms && num_kb / (s * 2) >= 8) s *= 2;
+  return s;
+}
+
+template <int BN, int EPI, typename OutT>
+int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
+  using Cfg = TcCfg<BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, OutT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) {
+      gpt2_internal::set_error(std::string("tc gemm smem attribute: ") + cudaGetErrorString(e));
+      return GPT2_ERR_CUDA;
+    }
+    attr_set = true;
+  }
+  CUtensorMap ma, mb;
+  const bool okA = g.a_kmajor ? make_map(&ma, g.A, g.K, g.M, g.lda, BM)
+                              : make_map(&ma, g.A, g.M, g.K, g.lda, BK);
+  const bool okB = g.b_kmajor ? make_map(&mb, g.B, g.K, g.N, g.ldb, BN)
+                              : make_map(&mb, g.B, g.N, g.K, g.ldb, BK);
+  if (!okA || !okB) {
+    gpt2_internal::set_error("tc gemm: tensor map encoding failed");
+    return GPT2_ERR_CUDA;
+  }
+  TcParams p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.a_mn = g.a_kmajor ? 0 : 1;
+  p.b_mn = g.b_kmajor ? 0 : 1;
+  p.tiles_m = cdiv(g.M, BM);
+  p.tiles_n = cdiv(g.N, BN);
+  p.num_kb = cdiv(g.K, BK);
+  p.kb_per_split = cdiv(p.num_kb, splits);
+  p.splits = cdiv(p.num_kb, p.kb_per_split);
+  p.total_tiles = p.tiles_m * p.tiles_n * p.splits;
+  p.ep = g.ep;
+  p.ws = p.splits > 1 ? g.ws : nullptr;
+  p.err = device_error_word();
+  const int grid = std::min(p.total_tiles, gpt2_internal::sm_count());
+  gemm_tc_kernel<BN, EPI, OutT><<<grid, kThreads, Cfg::SMEM, st>>>(ma, mb, p);
+  COUNT_LAUNCH(1);
+  if (p.splits > 1) {
+    const int64_t n = int64_t(g.M) * g.N;
+    tc_splitk_reduce_kernel<<<int(cdiv64(n, 256)), 256, 0, st>>>(
+        g.ws, p.splits, g.M, g.N, reinterpret_cast<float*>(g.ep.out), g.ep.ldo, g.ep.alpha,
+        g.ep.accumulate);
+    COUNT_LAUNCH(1);
+  }
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+template <int BN>
+int dispatch_epi(const GemmArgs& g, int splits, cudaStream_t st) {
+  const bool ob = g.ep.out_bf16;
+  switch (g.ep.kind) {
+    case EPI_STORE:
+      return ob ? launch_tc<BN, EPI_STORE, bf16>(g, splits, st)
+                : launch_tc<BN, EPI_STORE, float>(g, splits, st);
+    case EPI_GELU: return launch_tc<BN, EPI_GELU, bf16>(g, splits, st);
+    case EPI_RESID: return launch_tc<BN, EPI_RESID, float>(g, splits, st);
+    case EPI_ACC: return launch_tc<BN, EPI_ACC, float>(g, splits, st);
+    case EPI_GELU_BWD: return launch_tc<BN, EPI_GELU_BWD, bf16>(g, splits, st);
+    case EPI_CE_GRAD: return launch_tc<BN, EPI_CE_GRAD, bf16>(g, splits, st);
+    case EPI_LSE_PARTIAL: return launch_tc<BN, EPI_LSE_PARTIAL, float>(g, splits, st);
+  }
+  gpt2_internal::set_error("tc gemm: unknown epilogue");
+  return GPT2_ERR_ARG;
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const GemmArgs& g) {
+  if (!g.bf16_in || !encode_fn()) return false;
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  if (!al16(g.A) || !al16(g.B) || (g.lda & 7) || (g.ldb & 7)) return false;
+  if (g.ep.out && (!al16(g.ep.out) || (g.ep.ldo & 7))) return false;
+  if (g.ep.kind == EPI_LSE_PARTIAL && (!g.ep.part_max || !g.ep.part_sum || !g.ep.tgt_logit))
+    return false;
+  if ((g.ep.kind == EPI_GELU || g.ep.kind == EPI_GELU_BWD || g.ep.kind == EPI_CE_GRAD) &&
+      !g.ep.out_bf16)
+    return false;
+  if (g.ep.kind == EPI_RESID && (!al16(g.ep.rin) || !al16(g.ep.rout) || (g.ep.ldo & 7)))
+    return false;
+  if (g.ep.bias && !al16(g.ep.bias)) return false;
+  return true;
+}
+
+int gemm_tc_tile_n() { return 256; }
+
+size_t gemm_tc_workspace_bytes(int M, int N, int K) {
+  const int tiles = cdiv(M, BM) * cdiv(N, 256);
+  const int s = choose_splits_tc(tiles, cdiv(K, BK));
+  return s > 1 ? size_t(s) * M * N * sizeof(float) : 0;
+}
+
+int gemm_tc_launch(const GemmArgs& g, cudaStream_t st) {
+  constexpr int BN = 256;
+  int splits = 1;
+  if (g.ep.kind == EPI_ACC) {
+    splits = choose_splits_tc(cdiv(g.M, BM) * cdiv(g.N, BN), cdiv(g.K, BK));
+    if (!g.ws || size_t(splits) * g.M * g.N * sizeof(float) > g.ws_bytes) splits = 1;
+  }
+  return dispatch_epi<BN>(g, splits, st);
+}

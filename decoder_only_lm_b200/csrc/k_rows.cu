@@ -318,6 +318,174 @@ __global__ void reduce_ln_partials_kernel(const float* __restrict__ ws, int part
   *o = accumulate ? *o + acc : acc;
 }
 
+// Vectorised LayerNorm for C = 128 * NV (one warp per row, lane l owns the
+// float4 column groups 4l + 128i): the row lives in registers.
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, float (&v)[4]);
+template <>
+__device__ __forceinline__ void load4<float>(const float* p, float (&v)[4]) {
+  float4 f = *reinterpret_cast<const float4*>(p);
+  v[0] = f.x;
+  v[1] = f.y;
+  v[2] = f.z;
+  v[3] = f.w;
+}
+template <>
+__device__ __forceinline__ void load4<bf16>(const bf16* p, float (&v)[4]) {
+  uint2 u = *reinterpret_cast<const uint2*>(p);
+  float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
+  float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
+  v[0] = a.x;
+  v[1] = a.y;
+  v[2] = b.x;
+  v[3] = b.y;
+}
+template <typename T>
+__device__ __forceinline__ void store4(T* p, const float (&v)[4]);
+template <>
+__device__ __forceinline__ void store4<float>(float* p, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+__device__ __forceinline__ void store4<bf16>(bf16* p, const float (&v)[4]) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+template <int NV, typename OutT>
+__global__ void __launch_bounds__(256) layernorm_fwd_vec_kernel(
+    const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b,
+    OutT* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd, int64_t M,
+    float eps) {
+  constexpr int C = NV * 128;
+  const int64_t row = int64_t(blockIdx.x) * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float* xr = x + row * C;
+  float v[NV][4];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    load4<float>(xr + 4 * lane + 128 * i, v[i]);
+    s += (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
+  }
+  const float mu = warp_sum(s) / float(C);
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float d = v[i][k] - mu;
+      q += d * d;
+    }
+  const float rs = rsqrtf(warp_sum(q) / float(C) + eps);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = 4 * lane + 128 * i;
+    float gg[4], bb[4], o[4];
+    load4<float>(g + c, gg);
+    load4<float>(b + c, bb);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[k] = (v[i][k] - mu) * rs * gg[k] + bb[k];
+    store4<OutT>(y + row * C + c, o);
+  }
+  if (lane == 0) {
+    if (mean) mean[row] = mu;
+    if (rstd) rstd[row] = rs;
+  }
+}
+
+constexpr int kLnVecRows = 8;  // rows per warp in the vectorised backward
+
+// Each warp owns rows [w*8, w*8+8): dx is added into `dx` (and the new value
+// optionally stored rounded to CopyT); its dgamma/dbeta column partials go to
+// ws[w][0..C) and ws[w][C..2C).
+template <int NV, typename DyT, typename CopyT>
+__global__ void __launch_bounds__(256) layernorm_bwd_vec_kernel(
+    const DyT* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ mean,
+    const float* __restrict__ rstd, const float* __restrict__ g, int64_t M,
+    float* __restrict__ dx, CopyT* __restrict__ dx_copy, float* __restrict__ ws) {
+  constexpr int C = NV * 128;
+  const int64_t w = int64_t(blockIdx.x) * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t r0 = w * kLnVecRows;
+  if (r0 >= M) return;
+  float gam[NV][4], pg[NV][4], pb[NV][4];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    load4<float>(g + 4 * lane + 128 * i, gam[i]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) pg[i][k] = pb[i][k] = 0.f;
+  }
+  for (int r = 0; r < kLnVecRows; ++r) {
+    const int64_t row = r0 + r;
+    if (row >= M) break;
+    const float mu = mean[row], rs = rstd[row];
+    float xh[NV][4], d[NV][4];
+    float a = 0.f, bsum = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = 4 * lane + 128 * i;
+      load4<float>(x + row * C + c, xh[i]);
+      load4<DyT>(dy + row * C + c, d[i]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        xh[i][k] = (xh[i][k] - mu) * rs;
+        const float dxh = d[i][k] * gam[i][k];
+        a += dxh;
+        bsum += dxh * xh[i][k];
+        pg[i][k] += d[i][k] * xh[i][k];
+        pb[i][k] += d[i][k];
+      }
+    }
+    a = warp_sum(a) / float(C);
+    bsum = warp_sum(bsum) / float(C);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = 4 * lane + 128 * i;
+      float cur[4];
+      load4<float>(dx + row * C + c, cur);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) cur[k] += rs * (d[i][k] * gam[i][k] - a - xh[i][k] * bsum);
+      store4<float>(dx + row * C + c, cur);
+      if (dx_copy) store4<CopyT>(dx_copy + row * C + c, cur);
+    }
+  }
+  float* out = ws + w * 2 * C;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    store4<float>(out + 4 * lane + 128 * i, pg[i]);
+    store4<float>(out + C + 4 * lane + 128 * i, pb[i]);
+  }
+}
+
+// out[c] (+)= sum_p ws[p][c] for c < n (c >= split goes to out1[c - split]),
+// in a fixed order: 8 interleaved row slices per column, then the 8 slices.
+__global__ void __launch_bounds__(256) reduce_rows_kernel(const float* __restrict__ ws, int parts,
+                                                          int n, float* __restrict__ out0,
+                                                          float* __restrict__ out1, int split,
+                                                          int accumulate) {
+  __shared__ float sh[8][33];
+  const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + cx;
+  float acc = 0.f;
+  if (c < n)
+    for (int p = ry; p < parts; p += 8) acc += ws[int64_t(p) * n + c];
+  sh[ry][cx] = acc;
+  __syncthreads();
+  if (ry == 0 && c < n) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += sh[k][cx];
+    float* o = c < split ? out0 + c : out1 + (c - split);
+    *o = accumulate ? *o + t : t;
+  }
+}
+
 // ------------------------------------------------------------ bias-gradient column sums
 constexpr int kColRows = 256;  // rows per partial
 
@@ -572,7 +740,18 @@ int launch_layernorm_fwd(const float* x, const float* g, const float* b, OutT* y
     gpt2_internal::set_error("layernorm: C above 1024");
     return GPT2_ERR_ARG;
   }
-  layernorm_fwd_kernel<OutT><<<int(cdiv64(M, 8)), 256, 0, st>>>(x, g, b, y, mean, rstd, M, C, eps);
+  switch (C) {
+#define LNF(NV)                                                                                  \
+  case NV * 128:                                                                               \
+    layernorm_fwd_vec_kernel<NV, OutT><<<int(cdiv64(M, 8)), 256, 0, st>>>(x, g, b, y, mean, rstd, \
+                                                                          M, eps);             \
+    break;
+    LNF(1) LNF(2) LNF(3) LNF(4) LNF(5) LNF(6) LNF(7) LNF(8)
+#undef LNF
+    default:
+      layernorm_fwd_kernel<OutT><<<int(cdiv64(M, 8)), 256, 0, st>>>(x, g, b, y, mean, rstd, M, C,
+                                                                    eps);
+  }
   COUNT_LAUNCH(1);
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;
@@ -583,7 +762,9 @@ template int launch_layernorm_fwd<bf16>(const float*, const float*, const float*
                                         float*, int64_t, int, float, cudaStream_t);
 
 size_t layernorm_bwd_workspace(int64_t M, int C) {
-  return size_t(cdiv64(M, kLnRowsPerBlock)) * 2 * C * sizeof(float);
+  const int64_t parts =
+      (C % 128 == 0 && C <= 1024) ? cdiv64(M, kLnVecRows) : cdiv64(M, kLnRowsPerBlock);
+  return size_t(parts) * 2 * C * sizeof(float);
 }
 
 template <typename DyT, typename CopyT>
@@ -594,12 +775,31 @@ int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const
     gpt2_internal::set_error("layernorm: C above 1024");
     return GPT2_ERR_ARG;
   }
-  const int nb = int(cdiv64(M, kLnRowsPerBlock));
-  layernorm_bwd_kernel<DyT, CopyT><<<nb, 256, 0, st>>>(dy, x, mean, rstd, g, M, C, dx, dx_copy, ws);
-  COUNT_LAUNCH(1);
-  // ws rows hold [dgamma | dbeta]; both halves are reduced in one pass
-  reduce_ln_partials_kernel<<<cdiv(2 * C, 256), 256, 0, st>>>(ws, nb, C, dg, db, accumulate);
-  COUNT_LAUNCH(1);
+  if (C % 128 == 0 && C <= 1024) {
+    const int64_t warps = cdiv64(M, kLnVecRows);
+    const int nb = int(cdiv64(warps, 8));
+    switch (C / 128) {
+#define LNB(NV)                                                                              \
+  case NV:                                                                                   \
+    layernorm_bwd_vec_kernel<NV, DyT, CopyT><<<nb, 256, 0, st>>>(dy, x, mean, rstd, g, M, dx, \
+                                                                 dx_copy, ws);               \
+    break;
+      LNB(1) LNB(2) LNB(3) LNB(4) LNB(5) LNB(6) LNB(7) LNB(8)
+#undef LNB
+    }
+    COUNT_LAUNCH(1);
+    reduce_rows_kernel<<<cdiv(2 * C, 32), 256, 0, st>>>(ws, int(warps), 2 * C, dg, db, C,
+                                                        accumulate);
+    COUNT_LAUNCH(1);
+  } else {
+    const int nb = int(cdiv64(M, kLnRowsPerBlock));
+    layernorm_bwd_kernel<DyT, CopyT><<<nb, 256, 0, st>>>(dy, x, mean, rstd, g, M, C, dx, dx_copy,
+                                                         ws);
+    COUNT_LAUNCH(1);
+    // ws rows hold [dgamma | dbeta]; both halves are reduced in one pass
+    reduce_ln_partials_kernel<<<cdiv(2 * C, 256), 256, 0, st>>>(ws, nb, C, dg, db, accumulate);
+    COUNT_LAUNCH(1);
+  }
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;
 }

@@ -13,6 +13,9 @@ enum EpiKind {
   EPI_ACC = 3,       // out = (accumulate ? out : 0) + alpha*acc      (fp32)
   EPI_GELU_BWD = 4,  // out = acc * gelu'(aux[m,n])                   (act type)
   EPI_CE_GRAD = 5,   // out = scale*(exp(acc - lse[m]) - [n == tgt[m]]) (act type)
+  EPI_LSE_PARTIAL = 6,  // per row and column tile: max and sum of exp over the tile's
+                        // columns -> part_max/part_sum[m*part_ld + tile]; z[m, tgt[m]] ->
+                        // tgt_logit[m] (tensor-core path only)
 };
 
 struct EpiParams {
@@ -30,6 +33,10 @@ struct EpiParams {
   const int32_t* tgt = nullptr;
   const float* lse = nullptr;
   float ce_scale = 0.f;
+  float* part_max = nullptr;
+  float* part_sum = nullptr;
+  float* tgt_logit = nullptr;
+  int part_ld = 0;
 };
 
 struct GemmArgs {
@@ -89,6 +96,19 @@ size_t attn_bwd_workspace(int B, int Tn, int H);
 template <typename T>
 int launch_attn_bwd(const T* dout, const T* qkv, const T* out, const float* lse, int B, int Tn,
                     int C, int H, T* dqkv, float* ws, cudaStream_t st);
+
+// ---------------------------------------------------------------- tied LM head + CE
+// Forward: lse[m] = logsumexp_v (h[m] . W[v]) over all Vp rows of W,
+// row_loss[m] = lse[m] - h[m] . W[y[m]].  Backward: with dz = scale (softmax -
+// onehot(y)): dh = dz W (overwritten), dW (+)= dz^T h.  At most a bounded row
+// chunk of dz (never the whole [M, Vp]) lives in the workspace.
+size_t lmhead_workspace(int M, int C, int Vp, int bf16);
+int lmhead_fwd(const void* h, const void* W, const int32_t* y, int M, int C, int Vp, int bf16,
+               float* lse, float* row_loss, void* ws, size_t ws_bytes, cudaStream_t st);
+int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse, int M, int C,
+               int Vp, int bf16, float scale, void* dh, float* dW, int dw_accumulate, void* ws,
+               size_t ws_bytes, cudaStream_t st);
+bool gemm_tc_supported(const GemmArgs& g);
 
 // device error word of the op-level calls (bounded waits)
 int* device_error_word();

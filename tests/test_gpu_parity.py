@@ -1,8 +1,8 @@
 """GPU path vs the CPU oracle, through the C ABI, on seeded inputs.
 
 Bars: bit-exact for slicing; fp32 mode loss within 1e-4 nats and per-tensor
-gradient (and AdamW update) relative L2 within 1e-3; bf16 mode 2e-2 nats and
-3e-2.  The oracle runs in float64.
+gradient relative L2 within 1e-3; bf16 mode 2e-2 nats and 3e-2; the same bars
+for the parameters after one clip + AdamW step.  The oracle runs in float64.
 """
 import math
 
@@ -50,21 +50,34 @@ def test_step_matches_oracle(shape, bf16, torch):
     for name, shp in om.shapes():
         gg = gm.get_tensor(name, which=1)
         assert rel_l2(gg, G[name]) <= tol["grad"], (name, rel_l2(gg, G[name]))
-    # one clip + AdamW step: compare the parameter updates
+    # one clip + AdamW step
+    g_gpu = om.pack({n: gm.get_tensor(n, which=1) for n, _ in om.shapes()})
     norm_g = gm.clip_adamw_step(**HP)
     p_o, m_o, v_o = flat.copy(), np.zeros_like(flat), np.zeros_like(flat)
     norm_o = om.clip_adamw(p_o, go, m_o, v_o, 1, HP["lr"], HP["beta1"], HP["beta2"], HP["eps"],
                            HP["weight_decay"], HP["max_norm"])
     assert abs(norm_g - norm_o) <= tol["grad"] * norm_o
-    P_o = om.unpack(p_o)
+    # the optimizer kernel alone: the oracle's clip + AdamW applied to the GPU's own
+    # gradients must give the GPU's update (fp32 arithmetic vs float64)
+    p_x = flat.copy()
+    om.clip_adamw(p_x, g_gpu, np.zeros_like(flat), np.zeros_like(flat), 1, HP["lr"], HP["beta1"],
+                  HP["beta2"], HP["eps"], HP["weight_decay"], HP["max_norm"])
+    P_o, P_x = om.unpack(p_o), om.unpack(p_x)
     for name, shp in om.shapes():
+        p0 = named[name].astype(np.float64)
         pg = gm.get_tensor(name).astype(np.float64)
-        d_g = pg - named[name].astype(np.float64)
-        d_o = P_o[name] - named[name].astype(np.float64)
-        # Adam normalises each element's step: elements whose gradient is at the
-        # rounding level of the comparison may flip sign, so the bar is on the
-        # update as a whole.
-        assert rel_l2(d_g, d_o) <= max(tol["grad"], 0.05 if bf16 else 2e-3), name
+        # parameters after the step, within the stated bar
+        assert rel_l2(pg, P_o[name]) <= tol["grad"], name
+        # the update itself, exactly the optimizer's arithmetic on the GPU gradients
+        assert rel_l2(pg - p0, P_x[name] - p0) <= 1e-4, name
+        # the update against the oracle's: AdamW's first step is about lr * sign(g),
+        # so it is compared where the gradient is resolved above the path's
+        # rounding (|g| above 5% of the tensor's RMS gradient in bf16 mode)
+        g_ref = G[name]
+        rms = np.sqrt(np.mean(g_ref ** 2))
+        keep = np.abs(g_ref) > (0.05 if bf16 else 1e-3) * rms
+        if keep.any():
+            assert rel_l2((pg - p0)[keep], (P_o[name] - p0)[keep]) <= tol["grad"], name
     assert gm.step == 1
 
 
