@@ -74,5 +74,5 @@ def test_null_arguments_are_refused(g):
     ws = C.c_size_t()
     assert g.lib.gpt2_lmhead_ce_workspace(0, 64, 64, g.BF16, C.byref(ws)) == g.ERR_ARG
     assert g.lib.gpt2_lmhead_ce_workspace(128, 768, 50304, g.BF16, C.byref(ws)) == g.OK
-    assert ws.value > 128 * 50304 * 4  # holds one bounded chunk of logits, not all of them
+    assert ws.value >= 128 * 50304 * 2  # holds one bounded chunk of dz (bf16), not all of them
     assert ws.value < 8192 * 50304 * 2  # ... and less than the full [8192, 50304] bf16 logits
