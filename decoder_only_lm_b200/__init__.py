@@ -83,7 +83,7 @@ SIGNATURES = {
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m decoder_only_lm_b200.build`"
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python decoder_only_lm_b200/build.py`"
                           " (this package has no CPU fallback)")
     L = C.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():

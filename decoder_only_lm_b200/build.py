@@ -1,6 +1,8 @@
 """Build libgpt2_b200.so (all CUDA sources, sm_100a) in-tree.
 
-    python -m decoder_only_lm_b200.build [--force] [--verbose]
+    python decoder_only_lm_b200/build.py [--force] [--verbose]
+
+(run it as a script: importing the package loads the library it builds)
 
 Each .cu under csrc/ is compiled by nvcc for sm_100a with -lineinfo and the
 objects are linked into decoder_only_lm_b200/libgpt2_b200.so with the CUDA

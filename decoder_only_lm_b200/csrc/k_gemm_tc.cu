@@ -46,7 +46,9 @@ struct TcCfg {
   static constexpr int STAGES = BN == 256 ? 4 : 6;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = STAGES * STAGE + BAR_BYTES + 1024;
+  static constexpr int STAGE_ROW = 36;  // fp32 per staged accumulator row (32 + 4 pad)
+  static constexpr int EPI_BYTES = BM * STAGE_ROW * 4;
+  static constexpr int SMEM = STAGES * STAGE + EPI_BYTES + BAR_BYTES + 1024;
 };
 
 struct TcParams {
@@ -181,118 +183,179 @@ __device__ __forceinline__ uint32_t idesc_bf16(int a_mn, int b_mn) {
 }
 
 // ------------------------------------------------------------ vector helpers
-template <typename T>
-__device__ __forceinline__ void store32(T* p, const float (&v)[32]);
+template <typename T, int W>
+__device__ __forceinline__ void load_vec(const T* p, float (&v)[W]);
+template <typename T, int W>
+__device__ __forceinline__ void store_vec(T* p, const float (&v)[W]);
 template <>
-__device__ __forceinline__ void store32<float>(float* p, const float (&v)[32]) {
+__device__ __forceinline__ void load_vec<float, 4>(const float* p, float (&v)[4]) {
+  const float4 f = *reinterpret_cast<const float4*>(p);
+  v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+}
+template <>
+__device__ __forceinline__ void store_vec<float, 4>(float* p, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+__device__ __forceinline__ void load_vec<bf16, 8>(const bf16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-  for (int j = 0; j < 32; j += 4)
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = __bfloat1622float2(h[q]);
+    v[2 * q] = f.x;
+    v[2 * q + 1] = f.y;
+  }
+}
+template <>
+__device__ __forceinline__ void store_vec<bf16, 8>(bf16* p, const float (&v)[8]) {
+  uint4 u;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+    w[q] = *reinterpret_cast<uint32_t*>(&t);
+  }
+  *reinterpret_cast<uint4*>(p) = u;
+}
+template <>
+__device__ __forceinline__ void load_vec<float, 8>(const float* p, float (&v)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; j += 4) {
+    const float4 f = *reinterpret_cast<const float4*>(p + j);
+    v[j] = f.x; v[j + 1] = f.y; v[j + 2] = f.z; v[j + 3] = f.w;
+  }
+}
+template <>
+__device__ __forceinline__ void store_vec<float, 8>(float* p, const float (&v)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; j += 4)
     *reinterpret_cast<float4*>(p + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
 }
 template <>
-__device__ __forceinline__ void store32<bf16>(bf16* p, const float (&v)[32]) {
-#pragma unroll
-  for (int j = 0; j < 32; j += 8) {
-    uint4 u;
-    __nv_bfloat162 t0 = __floats2bfloat162_rn(v[j], v[j + 1]);
-    __nv_bfloat162 t1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
-    __nv_bfloat162 t2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]);
-    __nv_bfloat162 t3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
-    u.x = *reinterpret_cast<uint32_t*>(&t0);
-    u.y = *reinterpret_cast<uint32_t*>(&t1);
-    u.z = *reinterpret_cast<uint32_t*>(&t2);
-    u.w = *reinterpret_cast<uint32_t*>(&t3);
-    *reinterpret_cast<uint4*>(p + j) = u;
-  }
-}
-template <typename T>
-__device__ __forceinline__ void load32(const T* p, float (&v)[32]);
-template <>
-__device__ __forceinline__ void load32<float>(const float* p, float (&v)[32]) {
-#pragma unroll
-  for (int j = 0; j < 32; j += 4) {
-    float4 f = *reinterpret_cast<const float4*>(p + j);
-    v[j] = f.x;
-    v[j + 1] = f.y;
-    v[j + 2] = f.z;
-    v[j + 3] = f.w;
-  }
+__device__ __forceinline__ void load_vec<bf16, 4>(const bf16* p, float (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
 }
 template <>
-__device__ __forceinline__ void load32<bf16>(const bf16* p, float (&v)[32]) {
+__device__ __forceinline__ void store_vec<bf16, 4>(bf16* p, const float (&v)[4]) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+template <int W>
+__device__ __forceinline__ void load_bias(const float* b, int n, float (&v)[W]) {
 #pragma unroll
-  for (int j = 0; j < 32; j += 8) {
-    uint4 u = *reinterpret_cast<const uint4*>(p + j);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float2 f = __bfloat1622float2(h[q]);
-      v[j + 2 * q] = f.x;
-      v[j + 2 * q + 1] = f.y;
-    }
+  for (int j = 0; j < W; j += 4) {
+    const float4 f = *reinterpret_cast<const float4*>(b + n + j);
+    v[j] = f.x; v[j + 1] = f.y; v[j + 2] = f.z; v[j + 3] = f.w;
   }
 }
 
-// Epilogue of 32 consecutive columns n .. n+31 of row m (all in range).
-template <int EPI, typename OutT>
-__device__ __forceinline__ void epi_chunk32(const EpiParams& e, int m, int n, float (&v)[32],
-                                            float row_lse, int row_tgt) {
+// The epilogue op on W consecutive columns n .. n+W-1 of row m, s = the
+// accumulators (all W columns in range, 16-byte aligned addresses).
+template <int EPI, typename OutT, int W>
+__device__ __forceinline__ void epi_vec(const EpiParams& e, int m, int n, float (&s)[W]) {
   const int64_t i = int64_t(m) * e.ldo + n;
   if (EPI == EPI_STORE) {
     if (e.bias) {
-      float b[32];
-      load32<float>(e.bias + n, b);
+      float b[W];
+      load_bias<W>(e.bias, n, b);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = v[j] * e.alpha + b[j];
+      for (int j = 0; j < W; ++j) s[j] = s[j] * e.alpha + b[j];
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
+      for (int j = 0; j < W; ++j) s[j] *= e.alpha;
     }
-    store32<OutT>(reinterpret_cast<OutT*>(e.out) + i, v);
+    store_vec<OutT, W>(reinterpret_cast<OutT*>(e.out) + i, s);
   } else if (EPI == EPI_GELU) {
-    float b[32];
-    load32<float>(e.bias + n, b);
+    float b[W];
+    load_bias<W>(e.bias, n, b);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = round_through<OutT>(v[j] + b[j]);
-    store32<OutT>(reinterpret_cast<OutT*>(e.out) + i, v);
+    for (int j = 0; j < W; ++j) s[j] = round_through<OutT>(s[j] + b[j]);
+    store_vec<OutT, W>(reinterpret_cast<OutT*>(e.out) + i, s);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
-    store32<OutT>(reinterpret_cast<OutT*>(e.out2) + i, v);
+    for (int j = 0; j < W; ++j) s[j] = gelu_tanh(s[j]);
+    store_vec<OutT, W>(reinterpret_cast<OutT*>(e.out2) + i, s);
   } else if (EPI == EPI_RESID) {
-    float r[32];
-    load32<float>(e.rin + i, r);
+    float r[W];
+    load_vec<float, W>(e.rin + i, r);
     if (e.bias) {
-      float b[32];
-      load32<float>(e.bias + n, b);
+      float b[W];
+      load_bias<W>(e.bias, n, b);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) r[j] += b[j];
+      for (int j = 0; j < W; ++j) r[j] += b[j];
     }
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] += r[j];
-    store32<float>(e.rout + i, v);
+    for (int j = 0; j < W; ++j) s[j] += r[j];
+    store_vec<float, W>(e.rout + i, s);
   } else if (EPI == EPI_ACC) {
     float* o = reinterpret_cast<float*>(e.out) + i;
     if (e.accumulate) {
-      float r[32];
-      load32<float>(o, r);
+      float r[W];
+      load_vec<float, W>(o, r);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = r[j] + e.alpha * v[j];
+      for (int j = 0; j < W; ++j) s[j] = r[j] + e.alpha * s[j];
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
+      for (int j = 0; j < W; ++j) s[j] *= e.alpha;
     }
-    store32<float>(o, v);
+    store_vec<float, W>(o, s);
   } else if (EPI == EPI_GELU_BWD) {
-    float u[32];
-    load32<OutT>(reinterpret_cast<const OutT*>(e.aux) + i, u);
+    float u[W];
+    load_vec<OutT, W>(reinterpret_cast<const OutT*>(e.aux) + i, u);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] *= gelu_tanh_grad(u[j]);
-    store32<OutT>(reinterpret_cast<OutT*>(e.out) + i, v);
+    for (int j = 0; j < W; ++j) s[j] *= gelu_tanh_grad(u[j]);
+    store_vec<OutT, W>(reinterpret_cast<OutT*>(e.out) + i, s);
   } else if (EPI == EPI_CE_GRAD) {
+    const float l = e.lse[m];
+    const int t = e.tgt[m];
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      v[j] = e.ce_scale * (__expf(v[j] - row_lse) - (n + j == row_tgt ? 1.f : 0.f));
-    store32<OutT>(reinterpret_cast<OutT*>(e.out) + i, v);
+    for (int j = 0; j < W; ++j) s[j] = e.ce_scale * (__expf(s[j] - l) - (n + j == t ? 1.f : 0.f));
+    store_vec<OutT, W>(reinterpret_cast<OutT*>(e.out) + i, s);
+  }
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Store phase of one staged 128 x 32 chunk: W consecutive columns per item,
+// items spread so that a warp covers whole row segments (coalesced).
+template <int EPI, typename OutT, int W>
+__device__ __forceinline__ void epi_store_chunk(const TcParams& p, const float* S, int stage_row,
+                                                int e, int m0, int n0, int sp) {
+  constexpr int SEGS = 32 / W;  // segments per row; 128 rows x SEGS items, SEGS per thread
+#pragma unroll
+  for (int k = 0; k < SEGS; ++k) {
+    const int item = e + 128 * k;
+    const int row = item / SEGS, seg = item % SEGS;
+    const int m = m0 + row, n = n0 + seg * W;
+    if (m >= p.M || n >= p.N) continue;
+    float s[W];
+#pragma unroll
+    for (int j = 0; j < W; j += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(S + row * stage_row + seg * W + j);
+      s[j] = f.x; s[j + 1] = f.y; s[j + 2] = f.z; s[j + 3] = f.w;
+    }
+    const bool full = n + W <= p.N;
+    if (p.ws) {
+      float* w = p.ws + (int64_t(sp) * p.M + m) * p.N + n;
+      if (full && W == 4 && (p.N & 3) == 0) {
+        *reinterpret_cast<float4*>(w) = make_float4(s[0], s[1], s[2], s[3]);
+      } else {
+        for (int j = 0; j < W; ++j)
+          if (n + j < p.N) w[j] = s[j];
+      }
+    } else if (full) {
+      epi_vec<EPI, OutT, W>(p.ep, m, n, s);
+    } else {
+      for (int j = 0; j < W; ++j)
+        if (n + j < p.N) epi_apply<OutT>(p.ep, EPI, m, n + j, s[j]);
+    }
   }
 }
 
@@ -420,7 +483,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------ epilogue warpgroup
+    // TMEM phase: thread e (= tile row e, TMEM lane e) loads 32 accumulator
+    // columns and stages them in shared memory; store phase: the 128 threads
+    // apply the epilogue op to row segments and write them coalesced.
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    const int e = threadIdx.x - 128;
+    float* stg = reinterpret_cast<float*>(smem + S * Cfg::STAGE);
+    constexpr int SR = Cfg::STAGE_ROW;
     int t_local = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++t_local) {
       const int tm = tile % p.tiles_m;
@@ -431,13 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int m = tm * BM + q * 32 + lane;
-      float row_lse = 0.f;
+      const int m_row = tm * BM + e;
       int row_tgt = -1;
-      if ((EPI == EPI_CE_GRAD || EPI == EPI_LSE_PARTIAL) && m < p.M) {
-        if (EPI == EPI_CE_GRAD) row_lse = p.ep.lse[m];
-        row_tgt = p.ep.tgt[m];
-      }
+      if (EPI == EPI_LSE_PARTIAL && m_row < p.M) row_tgt = p.ep.tgt[m_row];
       float run_m = -INFINITY, run_s = 0.f, zt = 0.f;
       bool has_t = false;
 #pragma unroll 1
@@ -445,47 +510,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         float v[32];
         tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c0), v);
-        const int n = tn * BN + c0;
-        if (m >= p.M || n >= p.N) continue;
+        const int n0 = tn * BN + c0;
         if (EPI == EPI_LSE_PARTIAL) {
+          if (m_row >= p.M || n0 >= p.N) continue;
           // running max / sum of exp over this tile's valid columns
           float cm = -INFINITY;
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (n + j < p.N) cm = fmaxf(cm, v[j]);
+            if (n0 + j < p.N) cm = fmaxf(cm, v[j]);
           const float nm = fmaxf(run_m, cm);
-          float s = 0.f;
+          float sacc = 0.f;
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (n + j < p.N) s += __expf(v[j] - nm);
-          run_s = run_s * __expf(run_m - nm) + s;
+            if (n0 + j < p.N) sacc += __expf(v[j] - nm);
+          run_s = run_s * __expf(run_m - nm) + sacc;
           run_m = nm;
-          if (row_tgt >= n && row_tgt < n + 32) {
+          if (row_tgt >= n0 && row_tgt < n0 + 32) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (n + j == row_tgt) zt = v[j];
+              if (n0 + j == row_tgt) zt = v[j];
             has_t = true;
           }
           continue;
         }
-        const int nc = min(32, p.N - n);
-        if (p.ws) {
-          float* w = p.ws + (int64_t(sp) * p.M + m) * p.N + n;
-          if (nc == 32 && (p.N & 3) == 0) {
-            store32<float>(w, v);
-          } else {
-            for (int j = 0; j < nc; ++j) w[j] = v[j];
-          }
-        } else if (nc == 32) {
-          epi_chunk32<EPI, OutT>(p.ep, m, n, v, row_lse, row_tgt);
-        } else {
-          for (int j = 0; j < nc; ++j) epi_apply<OutT>(p.ep, EPI, m, n + j, v[j]);
-        }
+        if (n0 >= p.N) continue;  // uniform over the warpgroup
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(stg + e * SR + j) =
+              make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        epi_bar();
+        if (p.ws || sizeof(OutT) == 4)
+          epi_store_chunk<EPI, OutT, 4>(p, stg, SR, e, tm * BM, n0, sp);
+        else
+          epi_store_chunk<EPI, OutT, 8>(p, stg, SR, e, tm * BM, n0, sp);
+        epi_bar();
       }
-      if (EPI == EPI_LSE_PARTIAL && m < p.M) {
-        p.ep.part_max[int64_t(m) * p.ep.part_ld + tn] = run_m;
-        p.ep.part_sum[int64_t(m) * p.ep.part_ld + tn] = run_s;
-        if (has_t) p.ep.tgt_logit[m] = zt;
+      if (EPI == EPI_LSE_PARTIAL && m_row < p.M) {
+        p.ep.part_max[int64_t(m_row) * p.ep.part_ld + tn] = run_m;
+        p.ep.part_sum[int64_t(m_row) * p.ep.part_ld + tn] = run_s;
+        if (has_t) p.ep.tgt_logit[m_row] = zt;
       }
       tc_fence_before();
       mbar_arrive(tempty(acc));
@@ -497,16 +560,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
 }
 
+// Split-K reduction, splits added in order:
+//   EPI_ACC:   out = (accumulate ? out : 0) + alpha * sum_z ws[z]      (fp32)
+//   EPI_STORE: out = alpha * sum_z ws[z] + bias[n]                    (OutT)
+template <typename OutT>
 __global__ void tc_splitk_reduce_kernel(const float* __restrict__ ws, int splits, int M, int N,
-                                        float* __restrict__ out, int64_t ldo, float alpha,
-                                        int accumulate) {
+                                        EpiParams e) {
   const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
   if (i >= int64_t(M) * N) return;
   const int m = int(i / N), n = int(i % N);
   float acc = 0.f;
   for (int z = 0; z < splits; ++z) acc += ws[int64_t(z) * M * N + i];
-  float* o = out + int64_t(m) * ldo + n;
-  *o = (accumulate ? *o : 0.f) + alpha * acc;
+  const int64_t o = int64_t(m) * e.ldo + n;
+  if (e.kind == EPI_ACC) {
+    float* out = reinterpret_cast<float*>(e.out);
+    out[o] = (e.accumulate ? out[o] : 0.f) + e.alpha * acc;
+  } else {
+    reinterpret_cast<OutT*>(e.out)[o] = from_f32<OutT>(e.alpha * acc + (e.bias ? e.bias[n] : 0.f));
+  }
 }
 
 // ------------------------------------------------------------ host side
@@ -545,10 +616,13 @@ bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, 
   return r == CUDA_SUCCESS;
 }
 
+// Splits of K for outputs with fewer tiles than SMs: as many as fit in one
+// wave, each split keeping at least 4 k-blocks.
 int choose_splits_tc(int tiles, int num_kb) {
   const int sms = gpt2_internal::sm_count();
-  int s = 1;
-  while (tiles * s * 2 <= sms && num_kb / (s * 2) >= 8) s *= 2;
+  if (tiles * 2 > sms) return 1;
+  int s = std::min(16, sms / tiles);
+  while (s > 1 && num_kb / s < 4) --s;
   return s;
 }
 
@@ -594,9 +668,8 @@ int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
   COUNT_LAUNCH(1);
   if (p.splits > 1) {
     const int64_t n = int64_t(g.M) * g.N;
-    tc_splitk_reduce_kernel<<<int(cdiv64(n, 256)), 256, 0, st>>>(
-        g.ws, p.splits, g.M, g.N, reinterpret_cast<float*>(g.ep.out), g.ep.ldo, g.ep.alpha,
-        g.ep.accumulate);
+    tc_splitk_reduce_kernel<OutT><<<int(cdiv64(n, 256)), 256, 0, st>>>(g.ws, p.splits, g.M, g.N,
+                                                                       g.ep);
     COUNT_LAUNCH(1);
   }
   GPT2_LAUNCH_CHECK();
@@ -650,7 +723,7 @@ size_t gemm_tc_workspace_bytes(int M, int N, int K) {
 int gemm_tc_launch(const GemmArgs& g, cudaStream_t st) {
   constexpr int BN = 256;
   int splits = 1;
-  if (g.ep.kind == EPI_ACC) {
+  if (g.ep.kind == EPI_ACC || g.ep.kind == EPI_STORE) {
     splits = choose_splits_tc(cdiv(g.M, BM) * cdiv(g.N, BN), cdiv(g.K, BK));
     if (!g.ws || size_t(splits) * g.M * g.N * sizeof(float) > g.ws_bytes) splits = 1;
   }

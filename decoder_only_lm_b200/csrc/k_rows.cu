@@ -402,18 +402,20 @@ __global__ void __launch_bounds__(256) layernorm_fwd_vec_kernel(
 constexpr int kLnVecRows = 8;  // rows per warp in the vectorised backward
 
 // Each warp owns rows [w*8, w*8+8): dx is added into `dx` (and the new value
-// optionally stored rounded to CopyT); its dgamma/dbeta column partials go to
-// ws[w][0..C) and ws[w][C..2C).
+// optionally stored rounded to CopyT).  The 8 warps' dgamma/dbeta column
+// partials are summed in warp order in shared memory and the block's partial
+// goes to ws[block][0..C) and ws[block][C..2C).
 template <int NV, typename DyT, typename CopyT>
 __global__ void __launch_bounds__(256) layernorm_bwd_vec_kernel(
     const DyT* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ mean,
     const float* __restrict__ rstd, const float* __restrict__ g, int64_t M,
     float* __restrict__ dx, CopyT* __restrict__ dx_copy, float* __restrict__ ws) {
   constexpr int C = NV * 128;
-  const int64_t w = int64_t(blockIdx.x) * 8 + threadIdx.x / 32;
+  __shared__ __align__(16) float red[8][C];
+  const int warp = threadIdx.x / 32;
+  const int64_t w = int64_t(blockIdx.x) * 8 + warp;
   const int lane = threadIdx.x & 31;
   const int64_t r0 = w * kLnVecRows;
-  if (r0 >= M) return;
   float gam[NV][4], pg[NV][4], pb[NV][4];
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
@@ -423,15 +425,19 @@ __global__ void __launch_bounds__(256) layernorm_bwd_vec_kernel(
   }
   for (int r = 0; r < kLnVecRows; ++r) {
     const int64_t row = r0 + r;
-    if (row >= M) break;
+    if (row >= M) break;  // warp-uniform
     const float mu = mean[row], rs = rstd[row];
-    float xh[NV][4], d[NV][4];
+    float xh[NV][4], d[NV][4], cur[NV][4];
     float a = 0.f, bsum = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c = 4 * lane + 128 * i;
       load4<float>(x + row * C + c, xh[i]);
       load4<DyT>(dy + row * C + c, d[i]);
+      load4<float>(dx + row * C + c, cur[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         xh[i][k] = (xh[i][k] - mu) * rs;
@@ -447,19 +453,25 @@ __global__ void __launch_bounds__(256) layernorm_bwd_vec_kernel(
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c = 4 * lane + 128 * i;
-      float cur[4];
-      load4<float>(dx + row * C + c, cur);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) cur[k] += rs * (d[i][k] * gam[i][k] - a - xh[i][k] * bsum);
-      store4<float>(dx + row * C + c, cur);
-      if (dx_copy) store4<CopyT>(dx_copy + row * C + c, cur);
+      for (int k = 0; k < 4; ++k) cur[i][k] += rs * (d[i][k] * gam[i][k] - a - xh[i][k] * bsum);
+      store4<float>(dx + row * C + c, cur[i]);
+      if (dx_copy) store4<CopyT>(dx_copy + row * C + c, cur[i]);
     }
   }
-  float* out = ws + w * 2 * C;
+  float* out = ws + int64_t(blockIdx.x) * 2 * C;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    store4<float>(out + 4 * lane + 128 * i, pg[i]);
-    store4<float>(out + C + 4 * lane + 128 * i, pb[i]);
+  for (int half = 0; half < 2; ++half) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) store4<float>(&red[warp][4 * lane + 128 * i], half ? pb[i] : pg[i]);
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      float t = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) t += red[k][c];
+      out[half * C + c] = t;
+    }
+    __syncthreads();
   }
 }
 
@@ -763,7 +775,7 @@ template int launch_layernorm_fwd<bf16>(const float*, const float*, const float*
 
 size_t layernorm_bwd_workspace(int64_t M, int C) {
   const int64_t parts =
-      (C % 128 == 0 && C <= 1024) ? cdiv64(M, kLnVecRows) : cdiv64(M, kLnRowsPerBlock);
+      (C % 128 == 0 && C <= 1024) ? cdiv64(M, 8 * kLnVecRows) : cdiv64(M, kLnRowsPerBlock);
   return size_t(parts) * 2 * C * sizeof(float);
 }
 
@@ -788,8 +800,7 @@ int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const
 #undef LNB
     }
     COUNT_LAUNCH(1);
-    reduce_rows_kernel<<<cdiv(2 * C, 32), 256, 0, st>>>(ws, int(warps), 2 * C, dg, db, C,
-                                                        accumulate);
+    reduce_rows_kernel<<<cdiv(2 * C, 32), 256, 0, st>>>(ws, nb, 2 * C, dg, db, C, accumulate);
     COUNT_LAUNCH(1);
   } else {
     const int nb = int(cdiv64(M, kLnRowsPerBlock));

@@ -1,0 +1,110 @@
+"""Time one op-level entry point of the library on synthetic bf16 inputs.
+
+    python -m decoder_only_lm_b200.opbench matmul --M 16384 --N 3072 --K 768 [--a-mn] [--b-mn]
+    python -m decoder_only_lm_b200.opbench lmhead --M 8192 --C 768 --Vp 50304 [--fwd-only]
+    python -m decoder_only_lm_b200.opbench attention --B 16 --T 1024 --C 768 --H 12 [--bwd]
+    python -m decoder_only_lm_b200.opbench layernorm --M 16384 --C 768 [--bwd]
+
+Each call is timed with CUDA events on the current stream after warm-up and
+reported as one JSON line (ms per call, and TFLOP/s or GB/s of algorithmic
+work).  Small fixed cases of this script are what the ncu captures under
+profiles/ run.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+import decoder_only_lm_b200 as g
+
+
+def timed(fn, iters, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("op", choices=["matmul", "lmhead", "attention", "layernorm"])
+    ap.add_argument("--M", type=int, default=16384)
+    ap.add_argument("--N", type=int, default=3072)
+    ap.add_argument("--K", type=int, default=768)
+    ap.add_argument("--C", type=int, default=768)
+    ap.add_argument("--Vp", type=int, default=50304)
+    ap.add_argument("--V", type=int, default=50257)
+    ap.add_argument("--B", type=int, default=16)
+    ap.add_argument("--T", type=int, default=1024)
+    ap.add_argument("--H", type=int, default=12)
+    ap.add_argument("--a-mn", action="store_true")
+    ap.add_argument("--b-mn", action="store_true")
+    ap.add_argument("--accumulate", action="store_true")
+    ap.add_argument("--bwd", action="store_true")
+    ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--iters", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    a = ap.parse_args()
+    torch.manual_seed(0)
+    dev = "cuda"
+    out = {"op": a.op}
+    if a.op == "matmul":
+        A = torch.randn((a.K, a.M) if a.a_mn else (a.M, a.K), device=dev).bfloat16()
+        B = torch.randn((a.K, a.N) if a.b_mn else (a.N, a.K), device=dev).bfloat16()
+        D = torch.zeros((a.M, a.N), device=dev, dtype=torch.float32 if a.accumulate else torch.bfloat16)
+        fn = lambda: g.matmul(A, B, a_kmajor=not a.a_mn, b_kmajor=not a.b_mn, M=a.M, N=a.N, K=a.K,
+                              out=D, accumulate=a.accumulate)
+        ms = timed(fn, a.iters, a.warmup)
+        fl = 2.0 * a.M * a.N * a.K
+        out.update(M=a.M, N=a.N, K=a.K, a_mn=a.a_mn, b_mn=a.b_mn, ms=ms, tflops=fl / ms / 1e9)
+    elif a.op == "lmhead":
+        h = torch.randn((a.M, a.C), device=dev).bfloat16()
+        W = (0.02 * torch.randn((a.Vp, a.C), device=dev)).bfloat16()
+        y = torch.randint(0, a.V, (a.M,), device=dev, dtype=torch.int32)
+        fn = lambda: g.lmhead_ce(h, W, y, a.V, grads=not a.fwd_only)
+        ms = timed(fn, a.iters, a.warmup)
+        n_gemm = 1 if a.fwd_only else 3
+        fl = n_gemm * 2.0 * a.M * a.C * a.Vp
+        out.update(M=a.M, C=a.C, Vp=a.Vp, fwd_only=a.fwd_only, ms=ms, tflops_algorithmic=fl / ms / 1e9)
+    elif a.op == "attention":
+        qkv = torch.randn((a.B, a.T, 3 * a.C), device=dev).bfloat16()
+        o, lse = g.attention_fwd(qkv, a.H)
+        dout = torch.randn_like(o)
+        if a.bwd:
+            fn = lambda: g.attention_bwd(dout, qkv, o, lse, a.H)
+            mult = 4.0
+        else:
+            fn = lambda: g.attention_fwd(qkv, a.H)
+            mult = 2.0
+        ms = timed(fn, a.iters, a.warmup)
+        fl = mult * a.B * a.H * a.T * a.T * (a.C // a.H)  # causal half of 2 (4) full matmuls
+        out.update(B=a.B, T=a.T, C=a.C, H=a.H, bwd=a.bwd, ms=ms, tflops_algorithmic=fl / ms / 1e9)
+    else:
+        x = torch.randn((a.M, a.C), device=dev)
+        gam = torch.randn(a.C, device=dev)
+        bet = torch.randn(a.C, device=dev)
+        y, mean, rstd = g.layernorm_fwd(x, gam, bet, out_dtype=torch.bfloat16)
+        if a.bwd:
+            dy = torch.randn((a.M, a.C), device=dev).bfloat16()
+            dx = torch.zeros_like(x)
+            fn = lambda: g.layernorm_bwd(dy, x, mean, rstd, gam, dx=dx)
+            by = a.M * a.C * (2 + 4 + 8)
+        else:
+            fn = lambda: g.layernorm_fwd(x, gam, bet, out_dtype=torch.bfloat16)
+            by = a.M * a.C * (4 + 2)
+        ms = timed(fn, a.iters, a.warmup)
+        out.update(M=a.M, C=a.C, bwd=a.bwd, ms=ms, gbs=by / ms / 1e6)
+    out["device_error"] = g.device_error()
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -63,16 +63,21 @@ def test_step_matches_oracle(shape, bf16, torch):
     om.clip_adamw(p_x, g_gpu, np.zeros_like(flat), np.zeros_like(flat), 1, HP["lr"], HP["beta1"],
                   HP["beta2"], HP["eps"], HP["weight_decay"], HP["max_norm"])
     P_o, P_x = om.unpack(p_o), om.unpack(p_x)
+    # parameters after the step, within the stated bar (whole model: tensors that
+    # start at zero are all update, and the update is checked per element below)
+    p_gpu = om.pack({n: gm.get_tensor(n) for n, _ in om.shapes()})
+    assert rel_l2(p_gpu, p_o) <= tol["grad"]
     for name, shp in om.shapes():
         p0 = named[name].astype(np.float64)
         pg = gm.get_tensor(name).astype(np.float64)
-        # parameters after the step, within the stated bar
-        assert rel_l2(pg, P_o[name]) <= tol["grad"], name
         # the update itself, exactly the optimizer's arithmetic on the GPU gradients
         assert rel_l2(pg - p0, P_x[name] - p0) <= 1e-4, name
         # the update against the oracle's: AdamW's first step is about lr * sign(g),
         # so it is compared where the gradient is resolved above the path's
-        # rounding (|g| above 5% of the tensor's RMS gradient in bf16 mode)
+        # rounding (|g| above 5% of the tensor's RMS gradient in bf16 mode).  Some
+        # gradients are exactly zero in exact arithmetic (the key bias: softmax
+        # ignores a shift common to all scores), so only rounding decides their
+        # sign and they are excluded by this mask.
         g_ref = G[name]
         rms = np.sqrt(np.mean(g_ref ** 2))
         keep = np.abs(g_ref) > (0.05 if bf16 else 1e-3) * rms
