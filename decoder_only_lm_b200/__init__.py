@@ -74,6 +74,7 @@ SIGNATURES = {
     "gpt2_attention_fwd": (_i, [_P, _i, _i, _i, _i, _i, _P, _P, _P]),
     "gpt2_attention_bwd_workspace": (_i, [_i, _i, _i, _i, _i, C.POINTER(_sz)]),
     "gpt2_attention_bwd": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _i, _P, _P, _sz, _P]),
+    "gpt2_attention_bwd_noalloc": (_i, [_P, _P, _P, _P, _i, _i, _i, _i, _i, _P, _P]),
     "gpt2_matmul_workspace": (_i, [_i, _i, _i, C.POINTER(_sz)]),
     "gpt2_matmul": (_i, [_P, _i, _i64, _P, _i, _i64, _i, _i, _i, _i, _f, _i, _P, _i, _i64, _P,
                          _sz, _P]),
@@ -383,6 +384,17 @@ def attention_bwd(dout, qkv, out, lse, n_head, stream=None):
     _check(lib.gpt2_attention_bwd(_ptr(dout), _ptr(qkv), _ptr(out), _ptr(lse), _dtype_code(qkv), B, T,
                                   C3 // 3, n_head, _ptr(dqkv), _ptr(ws), ws_b.value,
                                   _stream_ptr(stream)))
+    return dqkv
+
+
+def attention_bwd_noalloc(dout, qkv, out, lse, n_head, dqkv=None, stream=None):
+    """gpt2_attention_bwd_noalloc: no workspace, the scratch is the library's own."""
+    import torch
+    B, T, C3 = qkv.shape
+    dqkv = torch.empty_like(qkv) if dqkv is None else dqkv
+    _check(lib.gpt2_attention_bwd_noalloc(_ptr(dout), _ptr(qkv), _ptr(out), _ptr(lse),
+                                          _dtype_code(qkv), B, T, C3 // 3, n_head, _ptr(dqkv),
+                                          _stream_ptr(stream)))
     return dqkv
 
 

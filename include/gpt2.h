@@ -287,6 +287,24 @@ int gpt2_attention_bwd(const void* dout, const void* qkv, const void* out, const
                        int dtype, int B, int T, int C, int H, void* dqkv, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* gpt2_attention_bwd for callers that cannot allocate device memory: a
+ * program that runs under a fixed memory budget already handed to another
+ * allocator, or a loop that must not call cudaMalloc / cudaFree because those
+ * calls can wait for the whole device to go idle.  Same arguments and result
+ * as gpt2_attention_bwd, but no workspace: the per-row scratch lives in a
+ * fixed 4 MiB device array declared by the library (held on every device that
+ * loads the library until the process exits).  No counterpart on the pages:
+ * an interface variant only.
+ *   - Limit: B*H*T <= 1,048,576 rows, else GPT2_ERR_ARG and a message.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call uses the same array, which keeps the last call's contents
+ *     (each call writes what it reads first, so nothing needs clearing):
+ *     calls that overlap on the GPU, e.g. on two streams, race. */
+int gpt2_attention_bwd_noalloc(const void* dout, const void* qkv, const void* out,
+                               const float* lse, int dtype, int B, int T, int C, int H,
+                               void* dqkv, void* stream);
+
 /* Dense contraction used by every linear layer (no counterpart on the pages
  * beyond "linear layer"; exported so it can be tested alone):
  *   D[m,n] = alpha * sum_k A(m,k) B(n,k)  (+ beta_accumulate * D[m,n] when

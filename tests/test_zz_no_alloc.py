@@ -1,0 +1,55 @@
+"""The attention backward that allocates nothing (gpt2_attention_bwd_noalloc).
+
+It serves callers that cannot allocate device memory: a program running
+under a fixed memory budget already given to another allocator, or a loop
+that must not call cudaMalloc / cudaFree because those calls can wait for the
+whole device.  Its result must match the workspace entry point
+(gpt2_attention_bwd) within the attention tolerance of the other GPU tests,
+on two calls in a row (the fixed scratch keeps the previous call's contents),
+and sizes beyond its fixed scratch must be refused with a message.
+
+This file is collected last so that a run stopping at the first failure has
+already run every other test.
+"""
+import numpy as np
+import pytest
+
+from tests.parity_util import rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("bf16", [True, False], ids=["bf16", "fp32"])
+def test_noalloc_matches_workspace_entry_point(bf16):
+    import torch
+
+    import decoder_only_lm_b200 as g
+    assert torch.cuda.is_available()
+    dt = torch.bfloat16 if bf16 else torch.float32
+    tol = 3e-2 if bf16 else 1e-4
+    for call, (B, T, C, H) in enumerate([(2, 200, 128, 2), (3, 77, 128, 2)]):
+        rng = np.random.default_rng(100 + call)
+        qkv = torch.from_numpy(rng.normal(size=(B, T, 3 * C)).astype(np.float32)).cuda().to(dt)
+        dout = torch.from_numpy(rng.normal(size=(B, T, C)).astype(np.float32)).cuda().to(dt)
+        out, lse = g.attention_fwd(qkv, H)
+        ref = g.attention_bwd(dout, qkv, out, lse, H)
+        got = g.attention_bwd_noalloc(dout, qkv, out, lse, H)
+        torch.cuda.synchronize()
+        a, b = got.float().cpu().numpy(), ref.float().cpu().numpy()
+        assert np.isfinite(a).all()
+        assert rel_l2(a, b) <= tol, (call, rel_l2(a, b))
+
+
+def test_noalloc_refuses_sizes_beyond_its_scratch():
+    import torch
+
+    import decoder_only_lm_b200 as g
+    H, C = 16, 1024
+    B, T = 65, 1024  # B*H*T = 1,064,960 > 1,048,576
+    qkv = torch.empty((1, 1, 3 * C), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(g.GPT2Error) as e:
+        g.lib_call = g.lib.gpt2_attention_bwd_noalloc(
+            qkv.data_ptr(), qkv.data_ptr(), qkv.data_ptr(), qkv.data_ptr(), g.BF16, B, T, C, H,
+            qkv.data_ptr(), None)
+        g._check(g.lib_call)
+    assert e.value.code == g.ERR_ARG and "exceeds" in str(e.value)
