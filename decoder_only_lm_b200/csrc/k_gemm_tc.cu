@@ -324,37 +324,80 @@ __device__ __forceinline__ void epi_vec(const EpiParams& e, int m, int n, float 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // Store phase of one staged 128 x 32 chunk: W consecutive columns per item,
-// items spread so that a warp covers whole row segments (coalesced).
+// items spread so that a warp covers whole row segments (coalesced).  All of
+// a thread's global loads (residual, accumulator, GELU input) are issued
+// before any of its stores, so their latencies overlap.
 template <int EPI, typename OutT, int W>
 __device__ __forceinline__ void epi_store_chunk(const TcParams& p, const float* S, int stage_row,
                                                 int e, int m0, int n0, int sp) {
   constexpr int SEGS = 32 / W;  // segments per row; 128 rows x SEGS items, SEGS per thread
+  constexpr bool kLoadF32 = (EPI == EPI_RESID || EPI == EPI_ACC);
+  constexpr bool kLoadAux = (EPI == EPI_GELU_BWD);
+  const EpiParams& ep = p.ep;
+  float s[SEGS][W], r[SEGS][W];
+  bool full[SEGS], live[SEGS];
 #pragma unroll
   for (int k = 0; k < SEGS; ++k) {
     const int item = e + 128 * k;
     const int row = item / SEGS, seg = item % SEGS;
     const int m = m0 + row, n = n0 + seg * W;
-    if (m >= p.M || n >= p.N) continue;
-    float s[W];
+    live[k] = m < p.M && n < p.N;
+    full[k] = live[k] && n + W <= p.N;
 #pragma unroll
     for (int j = 0; j < W; j += 4) {
       const float4 f = *reinterpret_cast<const float4*>(S + row * stage_row + seg * W + j);
-      s[j] = f.x; s[j + 1] = f.y; s[j + 2] = f.z; s[j + 3] = f.w;
+      s[k][j] = f.x; s[k][j + 1] = f.y; s[k][j + 2] = f.z; s[k][j + 3] = f.w;
     }
-    const bool full = n + W <= p.N;
+    if (!p.ws && full[k]) {
+      const int64_t i = int64_t(m) * ep.ldo + n;
+      if (kLoadF32 && (EPI == EPI_RESID || ep.accumulate))
+        load_vec<float, W>((EPI == EPI_RESID ? ep.rin : reinterpret_cast<const float*>(ep.out)) + i,
+                           r[k]);
+      if (kLoadAux) load_vec<OutT, W>(reinterpret_cast<const OutT*>(ep.aux) + i, r[k]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < SEGS; ++k) {
+    if (!live[k]) continue;
+    const int item = e + 128 * k;
+    const int row = item / SEGS, seg = item % SEGS;
+    const int m = m0 + row, n = n0 + seg * W;
     if (p.ws) {
       float* w = p.ws + (int64_t(sp) * p.M + m) * p.N + n;
-      if (full && W == 4 && (p.N & 3) == 0) {
-        *reinterpret_cast<float4*>(w) = make_float4(s[0], s[1], s[2], s[3]);
+      if (full[k] && W == 4 && (p.N & 3) == 0) {
+        *reinterpret_cast<float4*>(w) = make_float4(s[k][0], s[k][1], s[k][2], s[k][3]);
       } else {
         for (int j = 0; j < W; ++j)
-          if (n + j < p.N) w[j] = s[j];
+          if (n + j < p.N) w[j] = s[k][j];
       }
-    } else if (full) {
-      epi_vec<EPI, OutT, W>(p.ep, m, n, s);
-    } else {
+      continue;
+    }
+    if (!full[k]) {
       for (int j = 0; j < W; ++j)
-        if (n + j < p.N) epi_apply<OutT>(p.ep, EPI, m, n + j, s[j]);
+        if (n + j < p.N) epi_apply<OutT>(ep, EPI, m, n + j, s[k][j]);
+      continue;
+    }
+    const int64_t i = int64_t(m) * ep.ldo + n;
+    if (EPI == EPI_RESID) {
+      if (ep.bias) {
+        float b[W];
+        load_bias<W>(ep.bias, n, b);
+#pragma unroll
+        for (int j = 0; j < W; ++j) r[k][j] += b[j];
+      }
+#pragma unroll
+      for (int j = 0; j < W; ++j) s[k][j] += r[k][j];
+      store_vec<float, W>(ep.rout + i, s[k]);
+    } else if (EPI == EPI_ACC) {
+#pragma unroll
+      for (int j = 0; j < W; ++j) s[k][j] = (ep.accumulate ? r[k][j] : 0.f) + ep.alpha * s[k][j];
+      store_vec<float, W>(reinterpret_cast<float*>(ep.out) + i, s[k]);
+    } else if (EPI == EPI_GELU_BWD) {
+#pragma unroll
+      for (int j = 0; j < W; ++j) s[k][j] *= gelu_tanh_grad(r[k][j]);
+      store_vec<OutT, W>(reinterpret_cast<OutT*>(ep.out) + i, s[k]);
+    } else {
+      epi_vec<EPI, OutT, W>(ep, m, n, s[k]);
     }
   }
 }
