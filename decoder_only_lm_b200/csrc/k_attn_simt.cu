@@ -317,13 +317,13 @@ template int launch_attn_simt_bwd<float>(const float*, const float*, const float
 template int launch_attn_simt_bwd<bf16>(const bf16*, const bf16*, const bf16*, const float*, int,
                                         int, int, int, bf16*, float*, cudaStream_t);
 
-// Dispatch: bf16 with head size 64 runs on the tensor-core kernels; fp32 (the
-// parity mode) and other head sizes run on the kernels above.
-bool attn_mma_supported(int C, int H);
-int launch_attn_mma_fwd(const bf16* qkv, int B, int T, int C, int H, bf16* out, float* lse,
-                        cudaStream_t st);
-int launch_attn_mma_bwd(const bf16* dout, const bf16* qkv, const float* lse, const float* delta,
-                        int B, int T, int C, int H, bf16* dqkv, cudaStream_t st);
+// Dispatch: bf16 with head size 64 runs on the tcgen05 kernels (k_attn_tc.cu);
+// fp32 (the parity mode) and other head sizes run on the kernels above.
+bool attn_tc_supported(int B, int T, int C, int H);
+int launch_attn_tc_fwd(const bf16* qkv, int B, int T, int C, int H, bf16* out, float* lse,
+                       cudaStream_t st);
+int launch_attn_tc_bwd(const bf16* dout, const bf16* qkv, const float* lse, const float* delta,
+                       int B, int T, int C, int H, bf16* dqkv, cudaStream_t st);
 
 template <>
 int launch_attn_fwd<float>(const float* qkv, int B, int Tn, int C, int H, float* out, float* lse,
@@ -333,7 +333,7 @@ int launch_attn_fwd<float>(const float* qkv, int B, int Tn, int C, int H, float*
 template <>
 int launch_attn_fwd<bf16>(const bf16* qkv, int B, int Tn, int C, int H, bf16* out, float* lse,
                           cudaStream_t st) {
-  if (attn_mma_supported(C, H)) return launch_attn_mma_fwd(qkv, B, Tn, C, H, out, lse, st);
+  if (attn_tc_supported(B, Tn, C, H)) return launch_attn_tc_fwd(qkv, B, Tn, C, H, out, lse, st);
   return launch_attn_simt_fwd<bf16>(qkv, B, Tn, C, H, out, lse, st);
 }
 template <>
@@ -344,10 +344,10 @@ int launch_attn_bwd<float>(const float* dout, const float* qkv, const float* out
 template <>
 int launch_attn_bwd<bf16>(const bf16* dout, const bf16* qkv, const bf16* out, const float* lse,
                           int B, int Tn, int C, int H, bf16* dqkv, float* ws, cudaStream_t st) {
-  if (!attn_mma_supported(C, H))
+  if (!attn_tc_supported(B, Tn, C, H))
     return launch_attn_simt_bwd<bf16>(dout, qkv, out, lse, B, Tn, C, H, dqkv, ws, st);
   const int64_t rows = int64_t(B) * H * Tn;
   attn_delta64_kernel<<<int(cdiv64(rows, 256)), 256, 0, st>>>(dout, out, B, Tn, C, H, ws);
   COUNT_LAUNCH(1);
-  return launch_attn_mma_bwd(dout, qkv, lse, ws, B, Tn, C, H, dqkv, st);
+  return launch_attn_tc_bwd(dout, qkv, lse, ws, B, Tn, C, H, dqkv, st);
 }

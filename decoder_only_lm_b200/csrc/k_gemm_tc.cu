@@ -31,12 +31,14 @@
 #include <mutex>
 
 #include "epilogue.cuh"
+#include "tc_common.cuh"
+
+using namespace tc;
 
 namespace {
 
-constexpr int BM = 128, BK = 64, UMMA_K = 16;
+constexpr int BM = 128, UMMA_K = 16;
 constexpr int kThreads = 256;
-constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 
 template <int BN>
 struct TcCfg {
@@ -60,124 +62,9 @@ struct TcParams {
   int* err;
 };
 
-// ------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait on one phase; false (and the error word set) on expiry.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int where) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try(bar, parity)) return true;
-    if (global_ns() - t0 > kTimeoutNs) {
-      atomicExch(err, where);
-      return false;
-    }
-  }
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot),
-               "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void umma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-// Shared-memory matrix descriptor (sm_100 format, version 1, 128-byte swizzle).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return uint64_t((addr & 0x3FFFF) >> 4) | (uint64_t((lbo >> 4) & 0x3FFF) << 16) |
-         (uint64_t((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
-}
-// K-major, 128-byte rows of 64 bf16 along K, 8-row swizzle atoms of 1024 B;
-// the k-th 16-element slice starts 32 B further.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int k) {
-  return smem_desc(tile + k * 32, 16, 1024);
-}
-// MN-major: chunks of 64 MN-elements x BK rows (8 KB) side by side (LBO), rows
-// of 128 B along MN, 8-row groups 1024 B apart (SBO); k-th slice 16 rows on.
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int k) {
-  return smem_desc(tile + k * 16 * 128, BK * 128, 1024);
-}
-
 // Instruction descriptor: kind::f16, bf16 A and B, fp32 D, M = 128, N = BN.
 template <int BN>
-__device__ __forceinline__ uint32_t idesc_bf16(int a_mn, int b_mn) {
+__device__ __forceinline__ uint32_t gemm_idesc(int a_mn, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) |
          (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 }
@@ -484,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------ MMA issuer
-    const uint32_t idesc = idesc_bf16<BN>(p.a_mn, p.b_mn);
+    const uint32_t idesc = gemm_idesc<BN>(p.a_mn, p.b_mn);
     int stage = 0;
     uint32_t phase = 0;
     int t_local = 0;
@@ -643,24 +530,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [outer, inner] view with row stride ld
-// (elements), box {64, box_outer}, 128-byte swizzle, zero fill out of range.
-bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
-              int box_outer) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(outer)};
-  cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
-  cuuint32_t box[2] = {64, cuuint32_t(box_outer)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// Splits of K for outputs with fewer tiles than SMs: as many as fit in one
-// wave, each split keeping at least 4 k-blocks.
 int choose_splits_tc(int tiles, int num_kb) {
   const int sms = gpt2_internal::sm_count();
   if (tiles * 2 > sms) return 1;
@@ -683,10 +552,10 @@ int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
     attr_set = true;
   }
   CUtensorMap ma, mb;
-  const bool okA = g.a_kmajor ? make_map(&ma, g.A, g.K, g.M, g.lda, BM)
-                              : make_map(&ma, g.A, g.M, g.K, g.lda, BK);
-  const bool okB = g.b_kmajor ? make_map(&mb, g.B, g.K, g.N, g.ldb, BN)
-                              : make_map(&mb, g.B, g.N, g.K, g.ldb, BK);
+  const bool okA = g.a_kmajor ? tc::make_map_bf16(&ma, g.A, g.K, g.M, g.lda, BM)
+                              : tc::make_map_bf16(&ma, g.A, g.M, g.K, g.lda, BK);
+  const bool okB = g.b_kmajor ? tc::make_map_bf16(&mb, g.B, g.K, g.N, g.ldb, BN)
+                              : tc::make_map_bf16(&mb, g.B, g.N, g.K, g.ldb, BK);
   if (!okA || !okB) {
     gpt2_internal::set_error("tc gemm: tensor map encoding failed");
     return GPT2_ERR_CUDA;
@@ -738,6 +607,22 @@ int dispatch_epi(const GemmArgs& g, int splits, cudaStream_t st) {
 }
 
 }  // namespace
+
+namespace tc {
+bool make_map_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                   int box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(outer)};
+  cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
+  cuuint32_t box[2] = {64, cuuint32_t(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+}  // namespace tc
 
 bool gemm_tc_supported(const GemmArgs& g) {
   if (!g.bf16_in || !encode_fn()) return false;
