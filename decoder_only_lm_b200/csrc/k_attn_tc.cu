@@ -459,11 +459,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         sLD[e] = q < T ? p.lse[(int64_t(b) * p.H + h) * T + q] * kLog2e : 0.f;
         sLD[BS + e] = q < T ? p.delta[(int64_t(b) * p.H + h) * T + q] : 0.f;
       }
-      bool w = mbar_wait(b_sf, i & 1, p.err, 24);
-      if (i >= 1) w = w && mbar_wait(b_mm, (i - 1) & 1, p.err, 24);  // P^T / dS^T free
-      if (!__all_sync(0xffffffffu, w)) {
-        ok = false;
-        break;
+      // an expired wait (error word set) skips later waits but keeps the
+      // warpgroup's named barriers in step, so no warp is left at one
+      if (ok) {
+        bool w = mbar_wait(b_sf, i & 1, p.err, 24);
+        if (i >= 1) w = w && mbar_wait(b_mm, (i - 1) & 1, p.err, 24);  // P^T / dS^T free
+        ok = w;
       }
       tc_fence_after();
       wg_bar();  // sLD of this tile visible
@@ -503,6 +504,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_arrive(b_pf);
       wg_bar();  // sLD may be rewritten for the next tile
     }
+    ok = __all_sync(0xffffffffu, ok);
     if (ok && n > 0) {
       bool w = mbar_wait(b_mm, (n - 1) & 1, p.err, 27);
       if (__all_sync(0xffffffffu, w)) {

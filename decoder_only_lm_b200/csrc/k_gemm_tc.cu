@@ -28,6 +28,8 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "epilogue.cuh"
@@ -37,36 +39,61 @@ using namespace tc;
 
 namespace {
 
-constexpr int BM = 128, UMMA_K = 16;
-constexpr int kThreads = 256;
+// A tile of the output is 256 x BN, computed by a pair of CTAs (a cluster of
+// two): CTA r of the pair owns rows 128 r .. 128 r + 127 of the tile, holds
+// those rows of A and columns BN/2 r .. BN/2 r + BN/2 - 1 of B in its shared
+// memory, and receives its 128 accumulator rows in its own TMEM.
+constexpr int BM = 128;         // rows per CTA
+constexpr int BM2 = 2 * BM;     // rows per tile (CTA pair)
+constexpr int UMMA_K = 16;
+constexpr int kThreads = 384;  // warps 0-3: TMA, MMA, TMEM, idle; 4-7 and 8-11: epilogue
 
-template <int BN>
+constexpr int kSmemLimit = 232448;  // opt-in dynamic shared memory per block
+
+// Shared memory: [STAGES x (A, B) k-block ring | epilogue area | barriers].
+// With the TMA epilogue (TE) the area is a set of 8 KB chunk buffers; GEMMs
+// whose epilogue reads an input (residual, GELU input) give up one k-block
+// stage for more buffers so that more input bytes are in flight.
+template <int BN, bool TE, bool IN>
 struct TcCfg {
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int A_BYTES = BM * BK * 2;        // this CTA's 128 rows of A
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's BN/2 rows of B
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = !TE ? 5 : (IN ? 4 : 5);
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int BAR_BYTES = 512;
   static constexpr int STAGE_ROW = 36;  // fp32 per staged accumulator row (32 + 4 pad)
-  static constexpr int EPI_BYTES = BM * STAGE_ROW * 4;
+  // chunk buffers per epilogue warpgroup (two warpgroups, at most 8 each)
+  static constexpr int NBUF_WG =
+      TE ? ((kSmemLimit - 1024 - BAR_BYTES - STAGES * STAGE) / 16384 > 8
+                ? 8
+                : (kSmemLimit - 1024 - BAR_BYTES - STAGES * STAGE) / 16384)
+         : 0;
+  static constexpr int WG_BYTES = TE ? NBUF_WG * 8192 : BM * STAGE_ROW * 4;
+  static constexpr int EPI_BYTES = 2 * WG_BYTES;
   static constexpr int SMEM = STAGES * STAGE + EPI_BYTES + BAR_BYTES + 1024;
+  static_assert(SMEM <= kSmemLimit, "shared memory");
+  static_assert(!TE || NBUF_WG >= 4, "epilogue buffers");
 };
+template <int EPI>
+__host__ __device__ constexpr bool epi_has_input() {
+  return EPI == EPI_RESID || EPI == EPI_GELU_BWD;
+}
 
 struct TcParams {
   int M, N, K;
   int a_mn, b_mn;
-  int tiles_m, tiles_n, splits, kb_per_split, num_kb, total_tiles;
+  int tiles_m, tiles_n, splits, kb_per_split, num_kb, total_tiles;  // tiles of BM2 x BN
   EpiParams ep;
   float* ws;
   int* err;
 };
 
-// Instruction descriptor: kind::f16, bf16 A and B, fp32 D, M = 128, N = BN.
+// Instruction descriptor: kind::f16, bf16 A and B, fp32 D, M = 256 (pair), N = BN.
 template <int BN>
 __device__ __forceinline__ uint32_t gemm_idesc(int a_mn, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) |
-         (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+         (uint32_t(BN >> 3) << 17) | (uint32_t(BM2 >> 4) << 24);
 }
 
 // ------------------------------------------------------------ vector helpers
@@ -208,7 +235,10 @@ __device__ __forceinline__ void epi_vec(const EpiParams& e, int m, int n, float 
   }
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// named barrier of one epilogue warpgroup (ids 1 and 2)
+__device__ __forceinline__ void epi_bar(int id) {
+  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
 
 // Store phase of one staged 128 x 32 chunk: W consecutive columns per item,
 // items spread so that a warp covers whole row segments (coalesced).  All of
@@ -289,17 +319,320 @@ __device__ __forceinline__ void epi_store_chunk(const TcParams& p, const float* 
   }
 }
 
-template <int BN, int EPI, typename OutT>
+// ------------------------------------------------------------ TMA epilogue
+// GELU of the bf16 tensor-core path with tanh from the hardware tanh.approx
+// instruction (relative error about 2^-11, below the bf16 rounding of the
+// stored activation) [ZERO: OpFFN; the tanh form of GELU].
+__device__ __forceinline__ float tanh_hw(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// 2^x from the hardware ex2.approx instruction (exp(x) = 2^(x log2 e)).
+__device__ __forceinline__ float ex2_hw(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+__device__ __forceinline__ float gelu_hw(float u) {
+  const float k = 0.7978845608028654f, a = 0.044715f;
+  const float t = tanh_hw(u * (k + k * a * u * u));
+  const float h = 0.5f * u;
+  return fmaf(h, t, h);
+}
+__device__ __forceinline__ float gelu_grad_hw(float u) {
+  const float k = 0.7978845608028654f, a = 0.044715f;
+  const float u2 = u * u;
+  const float t = tanh_hw(u * (k + k * a * u2));
+  return 0.5f * (1.f + t) + 0.5f * u * (1.f - t * t) * k * (1.f + 3.f * a * u2);
+}
+
+// Chunks of the TMA epilogue: 128 rows x 64 bytes (32 bf16 or 16 fp32
+// columns) per 8 KB buffer in the 64-byte swizzle of the tensor map: the
+// 16-byte unit u of row r sits at r*64 + 16*(u ^ ((r >> 1) & 3)), so the
+// row-per-thread accesses of a warp are free of bank conflicts.
+template <int EPI, typename OutT, int NBUF>
+struct TeCfg {
+  static constexpr int CW = 64 / int(sizeof(OutT));
+  static constexpr int ARR = EPI == EPI_GELU ? 2 : 1;  // buffers per chunk
+  static constexpr int SLOTS = NBUF / ARR;
+  static constexpr bool HAS_IN = epi_has_input<EPI>();
+  static constexpr int DIST = HAS_IN ? SLOTS - 2 : 0;  // input prefetch distance in chunks
+  // bulk groups that may still be reading their buffers when a chunk is done
+  static constexpr int WAITN = HAS_IN ? SLOTS - 1 - DIST : (SLOTS - 2 < 6 ? SLOTS - 2 : 6);
+  static_assert(SLOTS >= 2 && SLOTS <= 16 && WAITN >= 0, "epilogue slots");
+};
+// tcgen05.ld of CW (32 or 16) accumulator columns without waiting; the
+// registers are valid after tmem_wait_cols(r), which names them so that no
+// use is scheduled before the wait.
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_ld32_async(taddr, r);
+}
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_cols(uint32_t (&r)[32]) { tmem_wait_ld(r); }
+__device__ __forceinline__ void tmem_wait_cols(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])::"memory");
+}
+__device__ __forceinline__ int swz64(int row, int u) {
+  return row * 64 + ((u ^ ((row >> 1) & 3)) << 4);
+}
+template <typename T>
+__device__ __forceinline__ void row_put(uint8_t* buf, int r, const float (&v)[64 / sizeof(T)]);
+template <>
+__device__ __forceinline__ void row_put<bf16>(uint8_t* buf, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint4 w;
+    uint32_t* x = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 t = __floats2bfloat162_rn(v[8 * u + 2 * q], v[8 * u + 2 * q + 1]);
+      x[q] = *reinterpret_cast<uint32_t*>(&t);
+    }
+    *reinterpret_cast<uint4*>(buf + swz64(r, u)) = w;
+  }
+}
+template <>
+__device__ __forceinline__ void row_put<float>(uint8_t* buf, int r, const float (&v)[16]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    *reinterpret_cast<float4*>(buf + swz64(r, u)) =
+        make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+}
+template <typename T>
+__device__ __forceinline__ void row_get(const uint8_t* buf, int r, float (&v)[64 / sizeof(T)]);
+template <>
+__device__ __forceinline__ void row_get<bf16>(const uint8_t* buf, int r, float (&v)[32]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint4 w = *reinterpret_cast<const uint4*>(buf + swz64(r, u));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(h[q]);
+      v[8 * u + 2 * q] = f.x;
+      v[8 * u + 2 * q + 1] = f.y;
+    }
+  }
+}
+template <>
+__device__ __forceinline__ void row_get<float>(const uint8_t* buf, int r, float (&v)[16]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float4 f = *reinterpret_cast<const float4*>(buf + swz64(r, u));
+    v[4 * u] = f.x; v[4 * u + 1] = f.y; v[4 * u + 2] = f.z; v[4 * u + 3] = f.w;
+  }
+}
+// bias[n0 .. n0+CW-1], zero past column N
+template <int CW>
+__device__ __forceinline__ void bias_chunk(const float* bias, int n0, int N, float (&b)[CW]) {
+  if (n0 + CW <= N) {
+#pragma unroll
+    for (int j = 0; j < CW; j += 4) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(bias + n0 + j));
+      b[j] = f.x; b[j + 1] = f.y; b[j + 2] = f.z; b[j + 3] = f.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < CW; ++j) b[j] = n0 + j < N ? bias[n0 + j] : 0.f;
+  }
+}
+
+// Epilogue warpgroup with TMA stores: thread e owns row 128 r + e of the
+// pair's tile (CTA rank r, TMEM lane e).
+// Per chunk it loads CW accumulator columns, applies the epilogue op (inputs
+// such as the residual or the GELU input arrive by TMA in the chunk's own
+// buffer, DIST chunks ahead), writes the row into the swizzled buffer, and
+// after one named barrier a single thread issues the TMA store (or, for
+// gradient accumulation, the TMA reduce-add: one fp32 add per element, so the
+// result does not depend on timing).  Out-of-range rows and columns of edge
+// tiles are clipped by the tensor map.
+template <int BN, int EPI, typename OutT, int NBUF>
+__device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMap* mo,
+                                             const CUtensorMap* mo2, const CUtensorMap* mi,
+                                             uint8_t* ebuf, uint64_t* tb, uint32_t tmem_base,
+                                             int wg) {
+  using T = TeCfg<EPI, OutT, NBUF>;
+  constexpr int CW = T::CW, NCH = BN / CW, SL = T::SLOTS;
+  const int e = threadIdx.x - 128 - 128 * wg;
+  const int bar_id = 1 + wg;
+  const int q = e >> 5;  // TMEM lanes 32q .. 32q+31
+  const bool leader = e == 0;
+  const uint32_t eb = smem_u32(ebuf);
+  const int rank = int(cluster_ctarank());
+  const int pair = int(blockIdx.x) >> 1, npairs = int(gridDim.x) >> 1;
+  auto tfull = [&](int a) { return smem_u32(tb + a); };
+  // the even CTA's accumulator-empty barrier (its MMA issuer waits on it)
+  auto tempty_pair = [&](int a) { return mapa_shared(smem_u32(tb + 2 + a), 0); };
+  auto lbar = [&](int s) { return smem_u32(tb + 4 + 8 * wg + s); };  // one per slot (<= 8)
+  const EpiParams& ep = p.ep;
+  // warpgroup wg drains accumulator wg: the pair's local tiles wg, wg+2, ...
+  const int pair_tiles = pair < p.total_tiles ? (p.total_tiles - 1 - pair) / npairs + 1 : 0;
+  const int my_tiles = pair_tiles > wg ? (pair_tiles - wg + 1) / 2 : 0;
+  const int total_chunks = my_tiles * NCH;
+  int next_load = 0;  // next chunk whose input is to be fetched (leader only)
+  auto issue_load = [&]() {
+    const int tile = pair + (wg + 2 * (next_load / NCH)) * npairs;
+    const int tm = tile % p.tiles_m, tn = (tile / p.tiles_m) % p.tiles_n;
+    const int slot = next_load % SL;
+    mbar_expect_tx(lbar(slot), 8192);
+    tma_load_2d(eb + slot * 8192, mi, lbar(slot), tn * BN + (next_load % NCH) * CW,
+                tm * BM2 + rank * BM);
+    ++next_load;
+  };
+  if (T::HAS_IN && leader)
+    while (next_load < min(T::DIST, total_chunks)) issue_load();
+
+  // A wait that expires (error word set) poisons the thread: later waits are
+  // skipped but every thread still runs the same sequence of named barriers,
+  // so no warp is left waiting at one.
+  int g = 0;  // chunks done by this warpgroup
+  bool ok = true;
+  for (int t_local = wg, tile = pair + wg * npairs; tile < p.total_tiles;
+       t_local += 2, tile += 2 * npairs) {
+    const int tm = tile % p.tiles_m, tn = (tile / p.tiles_m) % p.tiles_n;
+    const int acc = wg;
+    const int m0 = tm * BM2 + rank * BM;  // first row of this CTA's half
+    if (ok) ok = mbar_wait_cluster(tfull(acc), (t_local >> 1) & 1, p.err, 4);
+    tc_fence_after();
+    const int m = m0 + e;
+    float row_l = 0.f;
+    int row_t = -1;
+    if (EPI == EPI_CE_GRAD && m < p.M) {
+      row_l = ep.lse[m];
+      row_t = ep.tgt[m];
+    }
+    const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
+    // the accumulator columns of chunk c+1 are loaded while chunk c is processed
+    uint32_t rn[CW];
+    tmem_ld_cols(tbase, rn);
+    tmem_wait_cols(rn);
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c, ++g) {
+      const int slot = g % SL;
+      uint8_t* b0 = ebuf + slot * T::ARR * 8192;
+      const int n0 = tn * BN + c * CW;
+      float v[CW];
+#pragma unroll
+      for (int j = 0; j < CW; ++j) v[j] = __uint_as_float(rn[j]);
+      if (c + 1 < NCH) {
+        tmem_ld_cols(tbase + uint32_t((c + 1) * CW), rn);
+      } else if (leader) {
+        // every thread's TMEM loads completed before the previous chunk's
+        // barrier: the accumulator is drained, the pair's MMA may reuse it
+        mbar_arrive_cluster(tempty_pair(acc));
+      }
+      if constexpr (EPI == EPI_RESID || EPI == EPI_GELU_BWD) {
+        if (ok) ok = mbar_wait(lbar(slot), uint32_t((g / SL) & 1), p.err, 7);
+        float r[CW];
+        row_get<OutT>(b0, e, r);
+        if constexpr (EPI == EPI_RESID) {
+          if (ep.bias) {
+            float bb[CW];
+            bias_chunk<CW>(ep.bias, n0, p.N, bb);
+#pragma unroll
+            for (int j = 0; j < CW; ++j) r[j] += bb[j];
+          }
+#pragma unroll
+          for (int j = 0; j < CW; ++j) v[j] += r[j];
+        } else {
+#pragma unroll
+          for (int j = 0; j < CW; ++j) v[j] *= gelu_grad_hw(r[j]);
+        }
+        row_put<OutT>(b0, e, v);
+      } else if constexpr (EPI == EPI_GELU) {
+        float bb[CW], w[CW];
+        bias_chunk<CW>(ep.bias, n0, p.N, bb);
+#pragma unroll
+        for (int j = 0; j < CW; ++j) {
+          v[j] = round_through<OutT>(v[j] + bb[j]);
+          w[j] = gelu_hw(v[j]);
+        }
+        row_put<OutT>(b0, e, v);
+        row_put<OutT>(b0 + 8192, e, w);
+      } else if constexpr (EPI == EPI_STORE) {
+        if (ep.bias) {
+          float bb[CW];
+          bias_chunk<CW>(ep.bias, n0, p.N, bb);
+#pragma unroll
+          for (int j = 0; j < CW; ++j) v[j] = v[j] * ep.alpha + bb[j];
+        } else {
+#pragma unroll
+          for (int j = 0; j < CW; ++j) v[j] *= ep.alpha;
+        }
+        row_put<OutT>(b0, e, v);
+      } else if constexpr (EPI == EPI_ACC) {
+#pragma unroll
+        for (int j = 0; j < CW; ++j) v[j] *= ep.alpha;
+        row_put<OutT>(b0, e, v);
+      } else if constexpr (EPI == EPI_CE_GRAD) {
+        const float cs = ep.ce_scale, l2 = row_l * kLog2e;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) v[j] = cs * ex2_hw(fmaf(v[j], kLog2e, -l2));
+        if (row_t >= n0 && row_t < n0 + CW) {  // the target column: - scale
+#pragma unroll
+          for (int j = 0; j < CW; ++j)
+            if (n0 + j == row_t) v[j] -= cs;
+        }
+        row_put<OutT>(b0, e, v);
+      }
+      fence_proxy_async();
+      if (c + 1 < NCH) tmem_wait_cols(rn);
+      if (c + 2 == NCH) tc_fence_before();  // last TMEM load of the tile waited for
+      if (leader) {
+        bulk_wait_read<T::WAITN>();
+        if (T::HAS_IN && next_load < total_chunks) issue_load();
+      }
+      epi_bar(bar_id);
+      if (leader) {
+        const uint32_t src = eb + slot * T::ARR * 8192;
+        if (EPI == EPI_ACC && ep.accumulate)
+          tma_reduce_add_2d(mo, src, n0, m0);
+        else
+          tma_store_2d(mo, src, n0, m0);
+        if (EPI == EPI_GELU) tma_store_2d(mo2, src + 8192, n0, m0);
+        bulk_commit();
+      }
+    }
+  }
+  if (leader) {
+    bulk_wait_all();
+    // after an expired wait some fetched inputs were never waited for: let
+    // the last one of each buffer land before the CTA exits
+    if (!ok)
+      for (int gc = max(0, next_load - SL); gc < next_load; ++gc)
+        mbar_wait(lbar(gc % SL), uint32_t((gc / SL) & 1), p.err, 8);
+  }
+}
+
+template <int BN, int EPI, typename OutT, bool TE>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
-                   const __grid_constant__ CUtensorMap tma_b, const TcParams p) {
-  using Cfg = TcCfg<BN>;
+                   const __grid_constant__ CUtensorMap tma_b,
+                   const __grid_constant__ CUtensorMap tma_o,
+                   const __grid_constant__ CUtensorMap tma_o2,
+                   const __grid_constant__ CUtensorMap tma_i, const TcParams p) {
+  using Cfg = TcCfg<BN, TE, epi_has_input<EPI>()>;
   constexpr int S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cfg::STAGE);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  // [stages | epilogue area | barriers]; both CTAs of the pair use the same
+  // offsets, which the pair's MMA and its multicast commits rely on
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cfg::STAGE + Cfg::EPI_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 20);
   const uint32_t sbase = smem_u32(smem);
   auto full = [&](int s) { return smem_u32(bars + s); };
   auto empty = [&](int s) { return smem_u32(bars + S + s); };
@@ -307,55 +640,64 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto tempty = [&](int a) { return smem_u32(bars + 2 * S + 2 + a); };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = int(blockIdx.x) >> 1, npairs = int(gridDim.x) >> 1;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full(s), 1);
-      mbar_init(empty(s), 1);
+      mbar_init(full(s), 1);   // even CTA: its producer's arrive + both CTAs' bytes
+      mbar_init(empty(s), 1);  // the pair's MMA commit
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull(a), 1);
-      mbar_init(tempty(a), 128);
+      mbar_init(tfull(a), 1);   // the pair's MMA commit
+      mbar_init(tempty(a), 2);  // even CTA: one arrival from each CTA's epilogue
     }
+    for (int s = 0; s < 16; ++s) mbar_init(smem_u32(bars + 2 * S + 4 + s), 1);  // epilogue inputs
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 2) tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+  if (warp == 2) tmem_alloc_pair(smem_u32(tmem_slot), Cfg::TMEM_COLS);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialised before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ------------------------------------------------ TMA producer
+    // ------------------------------------------------ TMA producer (both CTAs)
+    // Loads this CTA's half of A (rows 128 rank ..) and of B (rows BN/2 rank ..)
+    // into its own ring; completion is counted on the even CTA's full barrier,
+    // whose expected byte count (both halves) the even CTA's producer posts.
+    const uint32_t full0 = mapa_shared(full(0), 0);
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < p.total_tiles && ok; tile += gridDim.x) {
+    for (int tile = pair; tile < p.total_tiles && ok; tile += npairs) {
       const int tm = tile % p.tiles_m;
       const int rest = tile / p.tiles_m;
       const int tn = rest % p.tiles_n, sp = rest / p.tiles_n;
       const int kb0 = sp * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+      const int ma = tm * BM2 + int(rank) * BM, nb = tn * BN + int(rank) * (BN / 2);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(empty(stage), phase ^ 1, p.err, 1)) {
+        if (!mbar_wait_cluster(empty(stage), phase ^ 1, p.err, 1)) {
           ok = false;
           break;
         }
-        mbar_expect_tx(full(stage), Cfg::STAGE);
+        if (rank == 0) mbar_expect_tx(full(stage), 2 * Cfg::STAGE);
+        const uint32_t fb = full0 + uint32_t(stage * 8);
         const uint32_t sa = sbase + stage * Cfg::STAGE, sb = sa + Cfg::A_BYTES;
         const int k0 = kb * BK;
         if (!p.a_mn) {
-          tma_load_2d(sa, &tma_a, full(stage), k0, tm * BM);
+          tma_load_2d_pair(sa, &tma_a, fb, k0, ma);
         } else {
-          tma_load_2d(sa, &tma_a, full(stage), tm * BM, k0);
-          tma_load_2d(sa + BK * 128, &tma_a, full(stage), tm * BM + 64, k0);
+          tma_load_2d_pair(sa, &tma_a, fb, ma, k0);
+          tma_load_2d_pair(sa + BK * 128, &tma_a, fb, ma + 64, k0);
         }
         if (!p.b_mn) {
-          tma_load_2d(sb, &tma_b, full(stage), k0, tn * BN);
+          tma_load_2d_pair(sb, &tma_b, fb, k0, nb);
         } else {
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j)
-            tma_load_2d(sb + j * BK * 128, &tma_b, full(stage), tn * BN + 64 * j, k0);
+          for (int j = 0; j < BN / 128; ++j)
+            tma_load_2d_pair(sb + j * BK * 128, &tma_b, fb, nb + 64 * j, k0);
         }
         ++issued;
         if (++stage == S) {
@@ -364,28 +706,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // wait until the copies of the last (up to S) issued stages have landed
+    // the MMA has consumed (so the copies have landed in) the last issued stages
     for (int q = 1; q <= min(issued, S); ++q) {
       const int idx = issued - q;
-      mbar_wait(full(idx % S), uint32_t((idx / S) & 1), p.err, 5);
+      mbar_wait_cluster(empty(idx % S), uint32_t((idx / S) & 1), p.err, 5);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------ MMA issuer
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------ MMA issuer (even CTA)
     const uint32_t idesc = gemm_idesc<BN>(p.a_mn, p.b_mn);
     int stage = 0;
     uint32_t phase = 0;
     int t_local = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < p.total_tiles && ok; tile += gridDim.x, ++t_local) {
+    for (int tile = pair; tile < p.total_tiles && ok; tile += npairs, ++t_local) {
       const int rest = tile / p.tiles_m;
       const int sp = rest / p.tiles_n;
       const int kb0 = sp * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
       const int acc = t_local & 1;
-      if (!mbar_wait(tempty(acc), ((t_local >> 1) & 1) ^ 1, p.err, 2)) break;
+      if (!mbar_wait_cluster(tempty(acc), ((t_local >> 1) & 1) ^ 1, p.err, 2)) break;
       tc_fence_after();
       const uint32_t d = tmem_base + uint32_t(acc * BN);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(full(stage), phase, p.err, 3)) {
+        if (!mbar_wait_cluster(full(stage), phase, p.err, 3)) {
           ok = false;
           break;
         }
@@ -395,42 +737,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < BK / UMMA_K; ++k) {
           const uint64_t ad = p.a_mn ? desc_mnmajor(sa, k) : desc_kmajor(sa, k);
           const uint64_t bd = p.b_mn ? desc_mnmajor(sb, k) : desc_kmajor(sb, k);
-          umma_bf16(d, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          umma_bf16_pair(d, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
         }
-        umma_commit(empty(stage));
+        umma_commit_pair(empty(stage), 3);  // frees the stage in both CTAs
         if (++stage == S) {
           stage = 0;
           phase ^= 1;
         }
       }
       if (!ok) break;
-      umma_commit(tfull(acc));
+      umma_commit_pair(tfull(acc), 3);  // both halves of the accumulator ready
     }
     // all issued MMAs complete before TMEM is released
     if (t_local > 0) {
       const int last = t_local - 1;
-      mbar_wait(tfull(last & 1), uint32_t((last >> 1) & 1), p.err, 6);
+      mbar_wait_cluster(tfull(last & 1), uint32_t((last >> 1) & 1), p.err, 6);
     }
+  } else if (warp >= 4 && TE) {
+    // ------------------------------------------------ epilogue warpgroup (TMA stores)
+    // (instantiated for the staged configuration too, where it never runs)
+    const int wg = (warp - 4) >> 2;  // warpgroup wg drains accumulator wg
+    epilogue_tma<BN, EPI, OutT, (TE ? Cfg::NBUF_WG : 4)>(
+        p, &tma_o, &tma_o2, &tma_i, smem + S * Cfg::STAGE + wg * Cfg::WG_BYTES, bars + 2 * S,
+        tmem_base, wg);
   } else if (warp >= 4) {
     // ------------------------------------------------ epilogue warpgroup
-    // TMEM phase: thread e (= tile row e, TMEM lane e) loads 32 accumulator
-    // columns and stages them in shared memory; store phase: the 128 threads
-    // apply the epilogue op to row segments and write them coalesced.
+    // TMEM phase: thread e (= row 128 rank + e of the tile, TMEM lane e)
+    // loads 32 accumulator columns and stages them in shared memory; store
+    // phase: the 128 threads apply the epilogue op to row segments and write
+    // them coalesced.
+    // Warpgroup wg (warps 4-7 or 8-11) drains accumulator wg: the pair's
+    // local tiles wg, wg+2, ...
+    const int wg = (warp - 4) >> 2;
+    const int bar_id = 1 + wg;
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
-    const int e = threadIdx.x - 128;
-    float* stg = reinterpret_cast<float*>(smem + S * Cfg::STAGE);
+    const int e = threadIdx.x - 128 - 128 * wg;
+    float* stg = reinterpret_cast<float*>(smem + S * Cfg::STAGE + wg * Cfg::WG_BYTES);
     constexpr int SR = Cfg::STAGE_ROW;
-    int t_local = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++t_local) {
+    const uint32_t tempty0 = mapa_shared(tempty(0), 0);
+    bool ok = true;
+    for (int t_local = wg, tile = pair + wg * npairs; tile < p.total_tiles;
+         t_local += 2, tile += 2 * npairs) {
       const int tm = tile % p.tiles_m;
       const int rest = tile / p.tiles_m;
       const int tn = rest % p.tiles_n, sp = rest / p.tiles_n;
-      const int acc = t_local & 1;
-      bool ok = mbar_wait(tfull(acc), (t_local >> 1) & 1, p.err, 4);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+      const int acc = wg;
+      const int m0 = tm * BM2 + int(rank) * BM;
+      // an expired wait (error word set) skips later waits, never the barriers
+      if (ok) ok = mbar_wait_cluster(tfull(acc), (t_local >> 1) & 1, p.err, 4);
       tc_fence_after();
-      const int m_row = tm * BM + e;
+      const int m_row = m0 + e;
       int row_tgt = -1;
       if (EPI == EPI_LSE_PARTIAL && m_row < p.M) row_tgt = p.ep.tgt[m_row];
       float run_m = -INFINITY, run_s = 0.f, zt = 0.f;
@@ -444,16 +800,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (EPI == EPI_LSE_PARTIAL) {
           if (m_row >= p.M || n0 >= p.N) continue;
           // running max / sum of exp over this tile's valid columns
+          const bool whole = n0 + 32 <= p.N;
           float cm = -INFINITY;
+          if (whole) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (n0 + j < p.N) cm = fmaxf(cm, v[j]);
+            for (int j = 0; j < 32; ++j) cm = fmaxf(cm, v[j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + j < p.N) cm = fmaxf(cm, v[j]);
+          }
           const float nm = fmaxf(run_m, cm);
+          const float nml = nm * kLog2e;
           float sacc = 0.f;
+          if (whole) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (n0 + j < p.N) sacc += __expf(v[j] - nm);
-          run_s = run_s * __expf(run_m - nm) + sacc;
+            for (int j = 0; j < 32; ++j) sacc += ex2_hw(fmaf(v[j], kLog2e, -nml));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + j < p.N) sacc += ex2_hw(fmaf(v[j], kLog2e, -nml));
+          }
+          run_s = run_s * ex2_hw((run_m - nm) * kLog2e) + sacc;
           run_m = nm;
           if (row_tgt >= n0 && row_tgt < n0 + 32) {
 #pragma unroll
@@ -468,26 +836,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; j += 4)
           *reinterpret_cast<float4*>(stg + e * SR + j) =
               make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        epi_bar();
+        epi_bar(bar_id);
         if (p.ws || sizeof(OutT) == 4)
-          epi_store_chunk<EPI, OutT, 4>(p, stg, SR, e, tm * BM, n0, sp);
+          epi_store_chunk<EPI, OutT, 4>(p, stg, SR, e, m0, n0, sp);
         else
-          epi_store_chunk<EPI, OutT, 8>(p, stg, SR, e, tm * BM, n0, sp);
-        epi_bar();
+          epi_store_chunk<EPI, OutT, 8>(p, stg, SR, e, m0, n0, sp);
+        epi_bar(bar_id);
       }
       if (EPI == EPI_LSE_PARTIAL && m_row < p.M) {
         p.ep.part_max[int64_t(m_row) * p.ep.part_ld + tn] = run_m;
         p.ep.part_sum[int64_t(m_row) * p.ep.part_ld + tn] = run_s;
         if (has_t) p.ep.tgt_logit[m_row] = zt;
       }
+      // all 128 threads' TMEM loads done: one arrival for this CTA's half
       tc_fence_before();
-      mbar_arrive(tempty(acc));
+      epi_bar(bar_id);
+      if (e == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc * 8));
     }
   }
+  // neither CTA leaves (freeing shared memory and TMEM that the pair's MMA,
+  // commits and arrivals address) before both are done
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  if (warp == 2) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
 }
 
 // Split-K reduction, splits added in order:
@@ -507,6 +879,38 @@ __global__ void tc_splitk_reduce_kernel(const float* __restrict__ ws, int splits
     out[o] = (e.accumulate ? out[o] : 0.f) + e.alpha * acc;
   } else {
     reinterpret_cast<OutT*>(e.out)[o] = from_f32<OutT>(e.alpha * acc + (e.bias ? e.bias[n] : 0.f));
+  }
+}
+
+// Same reduction, four columns per thread (N and ldo multiples of 4), rows
+// strided over blockIdx.y.
+template <typename OutT>
+__global__ void tc_splitk_reduce4_kernel(const float* __restrict__ ws, int splits, int M, int N,
+                                         EpiParams e) {
+  const int n = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (n >= N) return;
+  const int64_t plane = int64_t(M) * N;
+  for (int m = blockIdx.y; m < M; m += gridDim.y) {
+    const int64_t i = int64_t(m) * N + n;
+    float4 a = *reinterpret_cast<const float4*>(ws + i);
+    for (int z = 1; z < splits; ++z) {
+      const float4 b = *reinterpret_cast<const float4*>(ws + z * plane + i);
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    }
+    const int64_t o = int64_t(m) * e.ldo + n;
+    if (e.kind == EPI_ACC) {
+      float4* out = reinterpret_cast<float4*>(reinterpret_cast<float*>(e.out) + o);
+      float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e.accumulate) r = *out;
+      *out = make_float4(r.x + e.alpha * a.x, r.y + e.alpha * a.y, r.z + e.alpha * a.z,
+                         r.w + e.alpha * a.w);
+    } else {
+      float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e.bias) b = *reinterpret_cast<const float4*>(e.bias + n);
+      float v[4] = {e.alpha * a.x + b.x, e.alpha * a.y + b.y, e.alpha * a.z + b.z,
+                    e.alpha * a.w + b.w};
+      store_vec<OutT, 4>(reinterpret_cast<OutT*>(e.out) + o, v);
+    }
   }
 }
 
@@ -530,20 +934,84 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-int choose_splits_tc(int tiles, int num_kb) {
-  const int sms = gpt2_internal::sm_count();
-  if (tiles * 2 > sms) return 1;
-  int s = std::min(16, sms / tiles);
-  while (s > 1 && num_kb / s < 4) --s;
-  return s;
+// Number of CTA pairs that can be resident at once (1 CTA per SM; not every
+// SM need have a partner in its cluster domain).
+int pair_slots();
+
+// Split-K count for 256 x 256 pair tiles: the estimated time is the rounds of
+// persistent tiles over the resident pairs times the MMA time of one tile,
+// plus, with split-K, the traffic of the partial sums and one more launch.
+// Only plain stores and gradient accumulation may split.
+int choose_splits_tc(int M, int N, int K, bool splittable, size_t ws_bytes) {
+  const int pairs = pair_slots();
+  const int kb = cdiv(K, BK);
+  const int tiles = cdiv(M, BM2) * cdiv(N, 256);
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= (splittable ? 16 : 1); ++s) {
+    if (s > 1 && kb / s < 4) break;
+    const int kbs = cdiv(kb, s), se = cdiv(kb, kbs);
+    if (se > 1 && size_t(se) * M * N * sizeof(float) > ws_bytes) break;
+    const double tile_s = 2.0 * BM2 * 256 * kbs * BK / (2 * 15.5e12) + 0.5e-6;
+    double cost = cdiv(tiles * se, pairs) * tile_s;
+    if (se > 1) cost += double(M) * N * 4.0 * (se + 1) / 4.0e12 + 5e-6;
+    if (cost < best_cost * 0.97) {
+      best_cost = cost;
+      best = se;
+    }
+  }
+  return best;
 }
 
-template <int BN, int EPI, typename OutT>
+int pair_slots() {
+  static int slots = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    using Cfg = TcCfg<256, true, false>;
+    auto kern = gemm_tc_kernel<256, EPI_STORE, bf16, true>;
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * gpt2_internal::sm_count());
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = Cfg::SMEM;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+    }
+    (void)cudaGetLastError();  // no device (build hosts): fall back to SMs / 2
+    slots = n > 0 ? n : std::max(1, gpt2_internal::sm_count() / 2);
+  });
+  return slots;
+}
+
+// The TMA epilogue needs 16-byte aligned arrays and rows (tensor-map rules);
+// split-K partial tiles and the LSE-partial epilogue use the staged path.
+bool te_eligible(const GemmArgs& g, int splits) {
+  if (splits != 1 || g.ep.kind == EPI_LSE_PARTIAL) return false;
+  auto al16 = [](const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  const int eb = (g.ep.kind == EPI_RESID || g.ep.kind == EPI_ACC || !g.ep.out_bf16) ? 4 : 2;
+  if ((g.ep.ldo * eb) % 16 != 0) return false;
+  switch (g.ep.kind) {
+    case EPI_RESID: return al16(g.ep.rin) && al16(g.ep.rout);
+    case EPI_GELU: return al16(g.ep.out) && al16(g.ep.out2);
+    case EPI_GELU_BWD: return al16(g.ep.out) && al16(g.ep.aux);
+    default: return al16(g.ep.out);
+  }
+}
+
+template <int BN, int EPI, typename OutT, bool TE>
 int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
-  using Cfg = TcCfg<BN>;
+  using Cfg = TcCfg<BN, TE, epi_has_input<EPI>()>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, OutT>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, OutT, TE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) {
       gpt2_internal::set_error(std::string("tc gemm smem attribute: ") + cudaGetErrorString(e));
@@ -551,12 +1019,24 @@ int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
     }
     attr_set = true;
   }
-  CUtensorMap ma, mb;
-  const bool okA = g.a_kmajor ? tc::make_map_bf16(&ma, g.A, g.K, g.M, g.lda, BM)
-                              : tc::make_map_bf16(&ma, g.A, g.M, g.K, g.lda, BK);
-  const bool okB = g.b_kmajor ? tc::make_map_bf16(&mb, g.B, g.K, g.N, g.ldb, BN)
-                              : tc::make_map_bf16(&mb, g.B, g.N, g.K, g.ldb, BK);
-  if (!okA || !okB) {
+  CUtensorMap ma, mb, mo, mo2, mi;
+  memset(&mo, 0, sizeof(mo));
+  memset(&mo2, 0, sizeof(mo2));
+  memset(&mi, 0, sizeof(mi));
+  // boxes of one CTA's half: 128 rows of A, BN/2 rows of B
+  bool ok = g.a_kmajor ? tc::make_map_bf16(&ma, g.A, g.K, g.M, g.lda, BM)
+                       : tc::make_map_bf16(&ma, g.A, g.M, g.K, g.lda, BK);
+  ok = ok && (g.b_kmajor ? tc::make_map_bf16(&mb, g.B, g.K, g.N, g.ldb, BN / 2)
+                         : tc::make_map_bf16(&mb, g.B, g.N, g.K, g.ldb, BK));
+  if (TE) {
+    constexpr int eb = int(sizeof(OutT));
+    const void* o = EPI == EPI_RESID ? static_cast<const void*>(g.ep.rout) : g.ep.out;
+    ok = ok && tc::make_map_epi(&mo, o, eb, g.N, g.M, g.ep.ldo);
+    if (EPI == EPI_GELU) ok = ok && tc::make_map_epi(&mo2, g.ep.out2, eb, g.N, g.M, g.ep.ldo);
+    if (EPI == EPI_RESID) ok = ok && tc::make_map_epi(&mi, g.ep.rin, 4, g.N, g.M, g.ep.ldo);
+    if (EPI == EPI_GELU_BWD) ok = ok && tc::make_map_epi(&mi, g.ep.aux, eb, g.N, g.M, g.ep.ldo);
+  }
+  if (!ok) {
     gpt2_internal::set_error("tc gemm: tensor map encoding failed");
     return GPT2_ERR_CUDA;
   }
@@ -566,7 +1046,7 @@ int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
   p.K = g.K;
   p.a_mn = g.a_kmajor ? 0 : 1;
   p.b_mn = g.b_kmajor ? 0 : 1;
-  p.tiles_m = cdiv(g.M, BM);
+  p.tiles_m = cdiv(g.M, BM2);
   p.tiles_n = cdiv(g.N, BN);
   p.num_kb = cdiv(g.K, BK);
   p.kb_per_split = cdiv(p.num_kb, splits);
@@ -575,17 +1055,44 @@ int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
   p.ep = g.ep;
   p.ws = p.splits > 1 ? g.ws : nullptr;
   p.err = device_error_word();
-  const int grid = std::min(p.total_tiles, gpt2_internal::sm_count());
-  gemm_tc_kernel<BN, EPI, OutT><<<grid, kThreads, Cfg::SMEM, st>>>(ma, mb, p);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * std::min(p.total_tiles, pair_slots()));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t le = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, EPI, OutT, TE>, ma, mb, mo, mo2, mi, p);
+  if (le != cudaSuccess) {
+    gpt2_internal::set_error(std::string("tc gemm launch: ") + cudaGetErrorString(le));
+    return GPT2_ERR_CUDA;
+  }
   COUNT_LAUNCH(1);
   if (p.splits > 1) {
-    const int64_t n = int64_t(g.M) * g.N;
-    tc_splitk_reduce_kernel<OutT><<<int(cdiv64(n, 256)), 256, 0, st>>>(g.ws, p.splits, g.M, g.N,
-                                                                       g.ep);
+    const bool vec = (g.N % 4) == 0 && (g.ep.ldo % 4) == 0 && (!g.ep.bias || (reinterpret_cast<uintptr_t>(g.ep.bias) & 15) == 0);
+    if (vec) {
+      const dim3 grid(cdiv(g.N / 4, 128), std::min(g.M, 2048));
+      tc_splitk_reduce4_kernel<OutT><<<grid, 128, 0, st>>>(g.ws, p.splits, g.M, g.N, g.ep);
+    } else {
+      const int64_t n = int64_t(g.M) * g.N;
+      tc_splitk_reduce_kernel<OutT><<<int(cdiv64(n, 256)), 256, 0, st>>>(g.ws, p.splits, g.M, g.N,
+                                                                         g.ep);
+    }
     COUNT_LAUNCH(1);
   }
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;
+}
+
+template <int BN, int EPI, typename OutT>
+int launch_te(const GemmArgs& g, int splits, cudaStream_t st) {
+  return te_eligible(g, splits) ? launch_tc<BN, EPI, OutT, true>(g, splits, st)
+                                : launch_tc<BN, EPI, OutT, false>(g, splits, st);
 }
 
 template <int BN>
@@ -593,14 +1100,14 @@ int dispatch_epi(const GemmArgs& g, int splits, cudaStream_t st) {
   const bool ob = g.ep.out_bf16;
   switch (g.ep.kind) {
     case EPI_STORE:
-      return ob ? launch_tc<BN, EPI_STORE, bf16>(g, splits, st)
-                : launch_tc<BN, EPI_STORE, float>(g, splits, st);
-    case EPI_GELU: return launch_tc<BN, EPI_GELU, bf16>(g, splits, st);
-    case EPI_RESID: return launch_tc<BN, EPI_RESID, float>(g, splits, st);
-    case EPI_ACC: return launch_tc<BN, EPI_ACC, float>(g, splits, st);
-    case EPI_GELU_BWD: return launch_tc<BN, EPI_GELU_BWD, bf16>(g, splits, st);
-    case EPI_CE_GRAD: return launch_tc<BN, EPI_CE_GRAD, bf16>(g, splits, st);
-    case EPI_LSE_PARTIAL: return launch_tc<BN, EPI_LSE_PARTIAL, float>(g, splits, st);
+      return ob ? launch_te<BN, EPI_STORE, bf16>(g, splits, st)
+                : launch_te<BN, EPI_STORE, float>(g, splits, st);
+    case EPI_GELU: return launch_te<BN, EPI_GELU, bf16>(g, splits, st);
+    case EPI_RESID: return launch_te<BN, EPI_RESID, float>(g, splits, st);
+    case EPI_ACC: return launch_te<BN, EPI_ACC, float>(g, splits, st);
+    case EPI_GELU_BWD: return launch_te<BN, EPI_GELU_BWD, bf16>(g, splits, st);
+    case EPI_CE_GRAD: return launch_te<BN, EPI_CE_GRAD, bf16>(g, splits, st);
+    case EPI_LSE_PARTIAL: return launch_tc<BN, EPI_LSE_PARTIAL, float, false>(g, splits, st);
   }
   gpt2_internal::set_error("tc gemm: unknown epilogue");
   return GPT2_ERR_ARG;
@@ -622,6 +1129,20 @@ bool make_map_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t ou
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+bool make_map_epi(CUtensorMap* map, const void* base, int elem_bytes, int64_t inner,
+                  int64_t outer, int64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(outer)};
+  cuuint64_t strides[1] = {cuuint64_t(ld) * cuuint64_t(elem_bytes)};
+  cuuint32_t box[2] = {cuuint32_t(64 / elem_bytes), 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 }  // namespace tc
 
 bool gemm_tc_supported(const GemmArgs& g) {
@@ -640,20 +1161,13 @@ bool gemm_tc_supported(const GemmArgs& g) {
   return true;
 }
 
-int gemm_tc_tile_n() { return 256; }
-
 size_t gemm_tc_workspace_bytes(int M, int N, int K) {
-  const int tiles = cdiv(M, BM) * cdiv(N, 256);
-  const int s = choose_splits_tc(tiles, cdiv(K, BK));
-  return s > 1 ? size_t(s) * M * N * sizeof(float) : 0;
+  const int sp = choose_splits_tc(M, N, K, true, SIZE_MAX);
+  return sp > 1 ? size_t(sp) * M * N * sizeof(float) : 0;
 }
 
 int gemm_tc_launch(const GemmArgs& g, cudaStream_t st) {
-  constexpr int BN = 256;
-  int splits = 1;
-  if (g.ep.kind == EPI_ACC || g.ep.kind == EPI_STORE) {
-    splits = choose_splits_tc(cdiv(g.M, BM) * cdiv(g.N, BN), cdiv(g.K, BK));
-    if (!g.ws || size_t(splits) * g.M * g.N * sizeof(float) > g.ws_bytes) splits = 1;
-  }
-  return dispatch_epi<BN>(g, splits, st);
+  const bool splittable = (g.ep.kind == EPI_ACC || g.ep.kind == EPI_STORE) && g.ws;
+  const int sp = choose_splits_tc(g.M, g.N, g.K, splittable, splittable ? g.ws_bytes : 0);
+  return dispatch_epi<256>(g, sp, st);
 }

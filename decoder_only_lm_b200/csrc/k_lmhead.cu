@@ -9,11 +9,15 @@
 //            the target logit; a merge kernel combines the partials of a row in
 //            order: lse = M + log sum_t s_t exp(m_t - M), loss = lse - z_y.
 //            No logit is ever written to memory.
-//   backward per chunk of <= 2048 rows: the recomputed logits go straight from
-//            TMEM through dz = scale (exp(z - lse) - onehot) to a bf16 chunk
-//            buffer, then dh = dz W and dW (+)= dz^T h.
-// fp32 path (parity mode, CUDA cores): per chunk, logits in an fp32 chunk
-// buffer, a row kernel for lse / loss / dz, then the same two contractions.
+//   backward per chunk of <= 16384 rows: the recomputed logits go straight
+//            from TMEM through dz = scale (exp(z - lse) - onehot) to a bf16
+//            chunk buffer (1.6 GB at Vp = 50304), then dh = dz W and
+//            dW (+)= dz^T h.  Large chunks keep the weight-gradient GEMM long
+//            in K instead of re-accumulating the fp32 [Vp, C] gradient once
+//            per chunk.
+// fp32 path (parity mode, CUDA cores): per chunk of <= 2048 rows, logits in an
+// fp32 chunk buffer, a row kernel for lse / loss / dz, then the same two
+// contractions.
 
 #include <algorithm>
 
@@ -21,8 +25,10 @@
 
 namespace {
 
-constexpr int kChunk = 2048;
-constexpr int kTileN = 256;  // column tile of the tensor-core GEMM
+constexpr int kChunkBf16 = 16384, kChunkF32 = 2048;
+constexpr int kTileN = 256;  // column tile of the LSE-partial tensor-core GEMM
+
+int chunk_rows(int bf16) { return bf16 ? kChunkBf16 : kChunkF32; }
 
 size_t r256(size_t b) { return (b + 255) / 256 * 256; }
 
@@ -31,7 +37,7 @@ struct Layout {
 };
 
 Layout layout(int M, int C, int Vp, int bf16) {
-  const int mc = std::min(kChunk, M);
+  const int mc = std::min(chunk_rows(bf16), M);
   const int nt = cdiv(Vp, kTileN);
   Layout L{};
   L.part = bf16 ? r256(size_t(M) * nt * 4) : 0;  // each of part_max, part_sum
@@ -104,8 +110,8 @@ int lmhead_fwd(const void* h, const void* W, const int32_t* y, int M, int C, int
     GPT2_LAUNCH_CHECK();
     return GPT2_OK;
   }
-  for (int64_t r0 = 0; r0 < M; r0 += kChunk) {
-    const int mc = int(std::min<int64_t>(kChunk, M - r0));
+  for (int64_t r0 = 0; r0 < M; r0 += kChunkF32) {
+    const int mc = int(std::min<int64_t>(kChunkF32, M - r0));
     EpiParams e;
     e.kind = EPI_STORE;
     e.out = z;
@@ -132,8 +138,9 @@ int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse,
   void* dz = w + 2 * L.part + L.tgt + L.z;
   float* gws = reinterpret_cast<float*>(w + 2 * L.part + L.tgt + L.z + L.dz);
   const size_t a = bf16 ? 2 : 4;
-  for (int64_t r0 = 0; r0 < M; r0 += kChunk) {
-    const int mc = int(std::min<int64_t>(kChunk, M - r0));
+  const int chunk = chunk_rows(bf16);
+  for (int64_t r0 = 0; r0 < M; r0 += chunk) {
+    const int mc = int(std::min<int64_t>(chunk, M - r0));
     const void* hr = static_cast<const char*>(h) + r0 * C * int64_t(a);
     int rc;
     if (bf16) {

@@ -246,7 +246,8 @@ int gpt2_profile_read(gpt2_handle* h, int cat, int64_t* launches, double* ms, do
  * y: device int32 [M] in [0, V).  d_loss: device fp32 [1].  d_lse (nullable):
  * device fp32 [M] log-normalisers.  d_dh (nullable, same type as hidden) and
  * d_dw (nullable, fp32 [Vp,C]) request the backward.  The [M,Vp] logits are
- * never stored: at most a bounded row chunk lives in the workspace.
+ * never stored whole: at most a row chunk of dz (16384 rows for GPT2_BF16,
+ * 2048 for GPT2_F32) lives in the workspace.
  * workspace: device memory of at least gpt2_lmhead_ce_workspace() bytes.
  * C must be a multiple of 64 for GPT2_BF16.  Asynchronous on `stream`. */
 int gpt2_lmhead_ce_workspace(int M, int C, int Vp, int dtype, size_t* bytes);

@@ -76,3 +76,6 @@ def test_null_arguments_are_refused(g):
     assert g.lib.gpt2_lmhead_ce_workspace(128, 768, 50304, g.BF16, C.byref(ws)) == g.OK
     assert ws.value >= 128 * 50304 * 2  # holds one bounded chunk of dz (bf16), not all of them
     assert ws.value < 8192 * 50304 * 2  # ... and less than the full [8192, 50304] bf16 logits
+    # the dz chunk is bounded at 16384 rows whatever M is
+    assert g.lib.gpt2_lmhead_ce_workspace(65536, 768, 50304, g.BF16, C.byref(ws)) == g.OK
+    assert 16384 * 50304 * 2 <= ws.value < 32768 * 50304 * 2
