@@ -55,6 +55,49 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// three-input maximum (one instruction on sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// packed pair arithmetic of sm_100: (a0, a1) * (b0, b1) + (c0, c1) and (a0, a1) + (b0, b1)
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  uint64_t ra, rb, rc, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b0), "f"(b1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c0), "f"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(rd));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
+  uint64_t ra, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rd) : "f"(d0), "f"(d1));
+  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(rd) : "l"(ra));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(rd));
+}
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1) {
+  uint64_t ra, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rd) : "f"(d0), "f"(d1));
+  asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(rd) : "l"(ra));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(rd));
+}
+// maximum of 64 values as four independent chains of three-input maxima
+__device__ __forceinline__ float max64(const float (&x)[64]) {
+  float c[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float* y = x + 16 * k;
+    float a = max3f(y[0], y[1], y[2]);
+#pragma unroll
+    for (int i = 3; i < 15; i += 2) a = max3f(a, y[i], y[i + 1]);
+    c[k] = fmaxf(a, y[15]);
+  }
+  return max3f(c[0], c[1], fmaxf(c[2], c[3]));
+}
 __device__ __forceinline__ void wg_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // Row e of a 128 x 64 K-major bf16 operand tile (128-byte swizzle) from 32
@@ -233,32 +276,34 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_arrive(b_sfr(j & 1));
       const int key0 = j * BS;
       const bool need_mask = key0 + BS - 1 > qb * BR || key0 + BS > T;
-      float mx = -INFINITY;
+      float x[64];  // raw scores; keys past the query or past T become -inf
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float v = __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * sl2;
-        const int key = key0 + i;
-        mx = fmaxf(mx, (!need_mask || (key <= q && key < T)) ? v : -INFINITY);
+      for (int i = 0; i < 32; ++i) {
+        x[i] = __uint_as_float(r0[i]);
+        x[32 + i] = __uint_as_float(r1[i]);
       }
-      const float mn = fmaxf(m, mx);
+      if (need_mask) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (key0 + i > q || key0 + i >= T) x[i] = -INFINITY;
+      }
+      // running maximum in log2 units (scale > 0 commutes with max)
+      const float mn = fmaxf(m, max64(x) * sl2);
       const bool resc = mn > m + kRescale;  // always on the first tile (m = -inf)
       const float mu = resc ? mn : m;
       const float corr = resc ? ex2(m - mn) : 1.f;
+      // p = 2^(x sl2 - mu): one packed FMA per pair, ex2 per element, packed sums
       uint32_t pk[32];
-      float rs = 0.f;
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
-        const float v0 = __uint_as_float(i < 32 ? r0[i] : r1[i - 32]) * sl2;
-        const float v1 = __uint_as_float(i + 1 < 32 ? r0[i + 1] : r1[i - 31]) * sl2;
-        float p0 = ex2(v0 - mu), p1 = ex2(v1 - mu);
-        if (need_mask) {
-          const int key = key0 + i;
-          if (key > q || key >= T) p0 = 0.f;
-          if (key + 1 > q || key + 1 >= T) p1 = 0.f;
-        }
-        rs += p0 + p1;
+        float t0, t1;
+        fma2(t0, t1, x[i], x[i + 1], sl2, sl2, -mu, -mu);
+        const float p0 = ex2(t0), p1 = ex2(t1);
+        add2(sa[(i >> 1) & 3], sb[(i >> 1) & 3], p0, p1);
         pk[i >> 1] = pack2(p0, p1);
       }
+      const float rs = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
       l = l * corr + rs;
       m = mu;
       if (j >= 1 && __any_sync(0xffffffffu, resc)) {
@@ -346,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* pPt = smem + 2 * kRowTile + 2 * NSB * kStrTile;
   uint8_t* pDt = pPt + kOpTile;
   const uint32_t sPt = smem_u32(pPt), sDt = smem_u32(pDt);
-  float* sLD = reinterpret_cast<float*>(pDt + kOpTile);  // [64] lse*log2e, [64] delta
+  float* sLD = reinterpret_cast<float*>(pDt + kOpTile);  // [64] -lse*log2e, [64] -delta
   uint64_t* bars = reinterpret_cast<uint64_t*>(sLD + 2 * BS);
   // kv_full | qo_full[NSB] | qo_empty[NSB] | s_full | s_free | p_full | mm_done | slot
   const uint32_t b_kv = smem_u32(bars);
@@ -452,12 +497,23 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float scale = rsqrtf(float(D));
     const float sl2 = scale * kLog2e;
     bool ok = true;
+    // lse and delta of the 64 queries of a tile, fetched one tile ahead so the
+    // global loads overlap the current tile's work (threads e < 64); negated,
+    // so that each pair of queries costs one packed FMA / add
+    const int64_t bh = (int64_t(b) * p.H + h) * T;
+    float nl_next = 0.f, nd_next = 0.f;
+    auto fetch = [&](int i) {
+      const int q = (qt0 + i) * BS + e;
+      nl_next = q < T ? -p.lse[bh + q] * kLog2e : 0.f;
+      nd_next = q < T ? -p.delta[bh + q] : 0.f;
+    };
+    if (e < BS && n > 0) fetch(0);
     for (int i = 0; i < n; ++i) {
       const int q0 = (qt0 + i) * BS;
       if (e < BS) {
-        const int q = q0 + e;
-        sLD[e] = q < T ? p.lse[(int64_t(b) * p.H + h) * T + q] * kLog2e : 0.f;
-        sLD[BS + e] = q < T ? p.delta[(int64_t(b) * p.H + h) * T + q] : 0.f;
+        sLD[e] = nl_next;
+        sLD[BS + e] = nd_next;
+        if (i + 1 < n) fetch(i + 1);
       }
       // an expired wait (error word set) skips later waits but keeps the
       // warpgroup's named barriers in step, so no warp is left at one
@@ -468,37 +524,49 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       tc_fence_after();
       wg_bar();  // sLD of this tile visible
-      uint32_t s0[32], s1[32], d0[32], d1[32];
-      tmem_ld32_async(tS + lo, s0);
-      tmem_ld32_async(tS + lo + 32, s1);
-      tmem_ld32_async(tP + lo, d0);
-      tmem_ld32_async(tP + lo + 32, d1);
-      tmem_wait_ld(s0);
-      reg_after_wait(s1);
-      reg_after_wait(d0);
-      reg_after_wait(d1);
-      tc_fence_before();
-      mbar_arrive(b_sfr);
       const bool need_mask = q0 < kb * BR + BR || q0 + BS > T;
-      uint32_t pp[32], pd[32];
+      // two halves of 32 queries, so that only one half of S^T and dP^T is
+      // held in registers at a time; every 8 queries give one 16-byte chunk
+      // of the P^T and dS^T rows, written at once
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        float pr[2], ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int qc = c + u;
-          const float sv = __uint_as_float(qc < 32 ? s0[qc] : s1[qc - 32]);
-          const float dv = __uint_as_float(qc < 32 ? d0[qc] : d1[qc - 32]);
-          float pv = ex2(sv * sl2 - sLD[qc]);
-          if (need_mask && (q0 + qc < key || q0 + qc >= T)) pv = 0.f;
-          pr[u] = pv;
-          ds[u] = pv * (dv - sLD[BS + qc]);
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sx[32], dx[32];
+        tmem_ld32_async(tS + lo + 32 * hh, sx);
+        tmem_ld32_async(tP + lo + 32 * hh, dx);
+        tmem_wait_ld(sx);
+        reg_after_wait(dx);
+        if (hh == 1) {  // S^T and dP^T read: the MMA may overwrite them
+          tc_fence_before();
+          mbar_arrive(b_sfr);
         }
-        pp[c >> 1] = pack2(pr[0], pr[1]);
-        pd[c >> 1] = pack2(ds[0], ds[1]);
+#pragma unroll
+        for (int c8 = 0; c8 < 32; c8 += 8) {
+          uint32_t pp[4], pd[4];
+#pragma unroll
+          for (int c = c8; c < c8 + 8; c += 2) {
+            const int qc = 32 * hh + c;  // query column within the tile
+            const float2 nl = *reinterpret_cast<const float2*>(sLD + qc);       // -lse log2 e
+            const float2 nd = *reinterpret_cast<const float2*>(sLD + BS + qc);  // -delta
+            float t0, t1;
+            fma2(t0, t1, __uint_as_float(sx[c]), __uint_as_float(sx[c + 1]), sl2, sl2, nl.x,
+                 nl.y);
+            float p0 = ex2(t0), p1 = ex2(t1);
+            if (need_mask) {
+              if (q0 + qc < key || q0 + qc >= T) p0 = 0.f;
+              if (q0 + qc + 1 < key || q0 + qc + 1 >= T) p1 = 0.f;
+            }
+            float g0 = __uint_as_float(dx[c]), g1 = __uint_as_float(dx[c + 1]);
+            add2(g0, g1, nd.x, nd.y);  // dP - delta
+            mul2(g0, g1, p0, p1);      // dS = P (dP - delta)
+            pp[(c - c8) >> 1] = pack2(p0, p1);
+            pd[(c - c8) >> 1] = pack2(g0, g1);
+          }
+          const int ch = (32 * hh + c8) >> 3;  // 16-byte chunk of the 128-byte row
+          const int off = e * 128 + ((ch ^ (e & 7)) << 4);
+          *reinterpret_cast<uint4*>(pPt + off) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
+          *reinterpret_cast<uint4*>(pDt + off) = make_uint4(pd[0], pd[1], pd[2], pd[3]);
+        }
       }
-      put_row64(pPt, e, pp);
-      put_row64(pDt, e, pd);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       mbar_arrive(b_pf);
@@ -509,19 +577,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       bool w = mbar_wait(b_mm, (n - 1) & 1, p.err, 27);
       if (__all_sync(0xffffffffu, w)) {
         tc_fence_after();
-        uint32_t a0[32], a1[32], c0[32], c1[32];
-        tmem_ld32_async(tV + lo, a0);
-        tmem_ld32_async(tV + lo + 32, a1);
-        tmem_ld32_async(tKd + lo, c0);
-        tmem_ld32_async(tKd + lo + 32, c1);
-        tmem_wait_ld(a0);
-        reg_after_wait(a1);
-        reg_after_wait(c0);
-        reg_after_wait(c1);
-        if (key < T) {
-          bf16* drow = p.dqkv + (int64_t(row_base) + key) * 3 * C + h * D;
-          store_row64(drow + 2 * C, a0, a1, 1.f);
-          store_row64(drow + C, c0, c1, scale);
+        bf16* drow = p.dqkv + (int64_t(row_base) + key) * 3 * C + h * D;
+        // dV then dK, one 64-column row each
+#pragma unroll
+        for (int w2 = 0; w2 < 2; ++w2) {
+          uint32_t a0[32], a1[32];
+          tmem_ld32_async((w2 ? tKd : tV) + lo, a0);
+          tmem_ld32_async((w2 ? tKd : tV) + lo + 32, a1);
+          tmem_wait_ld(a0);
+          reg_after_wait(a1);
+          if (key < T) store_row64(drow + (w2 ? C : 2 * C), a0, a1, w2 ? scale : 1.f);
         }
       }
     }
@@ -673,17 +738,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        float ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int kc = c + u;
-          const float sv = __uint_as_float(kc < 32 ? s0[kc] : s1[kc - 32]);
-          const float dv = __uint_as_float(kc < 32 ? d0[kc] : d1[kc - 32]);
-          float pv = ex2(sv * sl2 - L2);
-          if (need_mask && (key0 + kc > q || key0 + kc >= T || q >= T)) pv = 0.f;
-          ds[u] = pv * (dv - Dl);
+        const float sa = __uint_as_float(c < 32 ? s0[c] : s1[c - 32]);
+        const float sb = __uint_as_float(c < 32 ? s0[c + 1] : s1[c - 31]);
+        float g0 = __uint_as_float(c < 32 ? d0[c] : d1[c - 32]);
+        float g1 = __uint_as_float(c < 32 ? d0[c + 1] : d1[c - 31]);
+        float t0, t1;
+        fma2(t0, t1, sa, sb, sl2, sl2, -L2, -L2);
+        float p0 = ex2(t0), p1 = ex2(t1);
+        if (need_mask) {
+          if (key0 + c > q || key0 + c >= T || q >= T) p0 = 0.f;
+          if (key0 + c + 1 > q || key0 + c + 1 >= T || q >= T) p1 = 0.f;
         }
-        pk[c >> 1] = pack2(ds[0], ds[1]);
+        add2(g0, g1, -Dl, -Dl);  // dP - delta
+        mul2(g0, g1, p0, p1);    // dS = P (dP - delta)
+        pk[c >> 1] = pack2(g0, g1);
       }
       put_row64(pDs, e, pk);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -505,7 +505,7 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
     const int tm = tile % p.tiles_m, tn = (tile / p.tiles_m) % p.tiles_n;
     const int acc = wg;
     const int m0 = tm * BM2 + rank * BM;  // first row of this CTA's half
-    if (ok) ok = mbar_wait_cluster(tfull(acc), (t_local >> 1) & 1, p.err, 4);
+    if (ok) ok = mbar_wait(tfull(acc), (t_local >> 1) & 1, p.err, 4);
     tc_fence_after();
     const int m = m0 + e;
     float row_l = 0.f;
@@ -678,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kb0 = sp * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
       const int ma = tm * BM2 + int(rank) * BM, nb = tn * BN + int(rank) * (BN / 2);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait_cluster(empty(stage), phase ^ 1, p.err, 1)) {
+        if (!mbar_wait(empty(stage), phase ^ 1, p.err, 1)) {
           ok = false;
           break;
         }
@@ -709,7 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the MMA has consumed (so the copies have landed in) the last issued stages
     for (int q = 1; q <= min(issued, S); ++q) {
       const int idx = issued - q;
-      mbar_wait_cluster(empty(idx % S), uint32_t((idx / S) & 1), p.err, 5);
+      mbar_wait(empty(idx % S), uint32_t((idx / S) & 1), p.err, 5);
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------ MMA issuer (even CTA)
@@ -723,11 +723,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int sp = rest / p.tiles_n;
       const int kb0 = sp * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
       const int acc = t_local & 1;
+      // arrivals of both CTAs' epilogues (release at cluster scope)
       if (!mbar_wait_cluster(tempty(acc), ((t_local >> 1) & 1) ^ 1, p.err, 2)) break;
       tc_fence_after();
       const uint32_t d = tmem_base + uint32_t(acc * BN);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait_cluster(full(stage), phase, p.err, 3)) {
+        if (!mbar_wait(full(stage), phase, p.err, 3)) {
           ok = false;
           break;
         }
@@ -751,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // all issued MMAs complete before TMEM is released
     if (t_local > 0) {
       const int last = t_local - 1;
-      mbar_wait_cluster(tfull(last & 1), uint32_t((last >> 1) & 1), p.err, 6);
+      mbar_wait(tfull(last & 1), uint32_t((last >> 1) & 1), p.err, 6);
     }
   } else if (warp >= 4 && TE) {
     // ------------------------------------------------ epilogue warpgroup (TMA stores)
@@ -784,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int acc = wg;
       const int m0 = tm * BM2 + int(rank) * BM;
       // an expired wait (error word set) skips later waits, never the barriers
-      if (ok) ok = mbar_wait_cluster(tfull(acc), (t_local >> 1) & 1, p.err, 4);
+      if (ok) ok = mbar_wait(tfull(acc), (t_local >> 1) & 1, p.err, 4);
       tc_fence_after();
       const int m_row = m0 + e;
       int row_tgt = -1;
