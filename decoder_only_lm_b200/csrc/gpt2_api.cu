@@ -474,9 +474,10 @@ int backward_t(gpt2_handle* h, float grad_scale) {
   {
     PROF(GPT2_PROF_LN_BWD, 0, lnb_bytes);
     H_CUDA(h, cudaMemsetAsync(h->dres, 0, M * C * sizeof(float), h->st));
+    // the residual gradient it leaves is the last layer's mlp.proj bias gradient
     H_TRY(h, (launch_layernorm_bwd<A, A>(dhf, h->res[2 * h->L], h->muf, h->rsf, P + h->off_lnfw,
                                           M, C, h->dres, copy, G + h->off_lnfw, G + h->off_lnfb,
-                                          acc, h->ws, h->st)));
+                                          G + h->lo[h->L - 1].fpb, acc, h->ws, h->st)));
   }
   A* du = static_cast<A*>(h->du);
   A* dln = static_cast<A*>(h->dln);
@@ -496,10 +497,6 @@ int backward_t(gpt2_handle* h, float grad_scale) {
       H_TRY(h, gemm(h, dres_a, 0, C, h->g[l], 0, F, C, F, int(M), e));
     }
     {
-      PROF(GPT2_PROF_OTHER, 0, 4.0 * M * C);
-      H_TRY(h, launch_colsum<float>(h->dres, M, C, G + o.fpb, acc, h->ws, h->st));
-    }
-    {
       // mlp.fc: u = ln2 Wfc^T + b
       PROF(GPT2_PROF_GEMM, 2 * gemm_flops(M, C, F), a * (2.0 * M * F + 2.0 * M * C + F * C) + 8.0 * F * C);
       EpiParams e = epi(EPI_STORE, dln, C, ab);
@@ -514,9 +511,10 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     }
     {
       PROF(GPT2_PROF_LN_BWD, 0, lnb_bytes);
+      // ... and attn.proj's bias gradient: column sums of the residual gradient
       H_TRY(h, (launch_layernorm_bwd<A, A>(dln, h->res[2 * l + 1], h->mu2[l], h->rs2[l],
                                             P + o.ln2w, M, C, h->dres, copy, G + o.ln2w,
-                                            G + o.ln2b, acc, h->ws, h->st)));
+                                            G + o.ln2b, G + o.projb, acc, h->ws, h->st)));
     }
     {
       // attn.proj: h' = h + att Wp^T + b
@@ -526,10 +524,6 @@ int backward_t(gpt2_handle* h, float grad_scale) {
       e = epi(EPI_ACC, G + o.projw, C, 0);
       e.accumulate = acc;
       H_TRY(h, gemm(h, dres_a, 0, C, h->att[l], 0, C, C, C, int(M), e));
-    }
-    {
-      PROF(GPT2_PROF_OTHER, 0, 4.0 * M * C);
-      H_TRY(h, launch_colsum<float>(h->dres, M, C, G + o.projb, acc, h->ws, h->st));
     }
     {
       PROF(GPT2_PROF_ATTN_BWD, attn_bwd_flops, a * 9.0 * M * C + 8.0 * M * Hh);
@@ -552,9 +546,11 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     }
     {
       PROF(GPT2_PROF_LN_BWD, 0, lnb_bytes);
+      // ... and the previous layer's mlp.proj bias gradient
       H_TRY(h, (launch_layernorm_bwd<A, A>(dln, h->res[2 * l], h->mu1[l], h->rs1[l], P + o.ln1w,
-                                            M, C, h->dres, copy, G + o.ln1w, G + o.ln1b, acc,
-                                            h->ws, h->st)));
+                                            M, C, h->dres, copy, G + o.ln1w, G + o.ln1b,
+                                            l > 0 ? G + h->lo[l - 1].fpb : nullptr, acc, h->ws,
+                                            h->st)));
     }
   }
   {

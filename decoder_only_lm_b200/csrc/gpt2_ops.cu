@@ -110,10 +110,10 @@ int gpt2_layernorm_bwd(const void* dy, int dy_dtype, const float* x, const float
   float* ws = static_cast<float*>(workspace);
   if (dy_dtype == GPT2_BF16)
     return launch_layernorm_bwd<bf16, bf16>(static_cast<const bf16*>(dy), x, mean, rstd, gamma, M,
-                                            C, dx, nullptr, dgamma, dbeta, 1, ws, st);
+                                            C, dx, nullptr, dgamma, dbeta, nullptr, 1, ws, st);
   if (dy_dtype == GPT2_F32)
     return launch_layernorm_bwd<float, float>(static_cast<const float*>(dy), x, mean, rstd, gamma,
-                                              M, C, dx, nullptr, dgamma, dbeta, 1, ws, st);
+                                              M, C, dx, nullptr, dgamma, dbeta, nullptr, 1, ws, st);
   set_error("layernorm_bwd: bad dtype");
   return GPT2_ERR_ARG;
 }

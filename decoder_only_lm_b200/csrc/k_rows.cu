@@ -409,19 +409,20 @@ template <int NV, typename DyT, typename CopyT>
 __global__ void __launch_bounds__(256) layernorm_bwd_vec_kernel(
     const DyT* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ mean,
     const float* __restrict__ rstd, const float* __restrict__ g, int64_t M,
-    float* __restrict__ dx, CopyT* __restrict__ dx_copy, float* __restrict__ ws) {
+    float* __restrict__ dx, CopyT* __restrict__ dx_copy, float* __restrict__ ws, int want_sum) {
   constexpr int C = NV * 128;
   __shared__ __align__(16) float red[8][C];
   const int warp = threadIdx.x / 32;
   const int64_t w = int64_t(blockIdx.x) * 8 + warp;
   const int lane = threadIdx.x & 31;
   const int64_t r0 = w * kLnVecRows;
-  float gam[NV][4], pg[NV][4], pb[NV][4];
+  // column partials: dgamma, dbeta and (want_sum) the updated dx itself
+  float gam[NV][4], pg[NV][4], pb[NV][4], ps[NV][4];
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     load4<float>(g + 4 * lane + 128 * i, gam[i]);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) pg[i][k] = pb[i][k] = 0.f;
+    for (int k = 0; k < 4; ++k) pg[i][k] = pb[i][k] = ps[i][k] = 0.f;
   }
   for (int r = 0; r < kLnVecRows; ++r) {
     const int64_t row = r0 + r;
@@ -454,33 +455,39 @@ __global__ void __launch_bounds__(256) layernorm_bwd_vec_kernel(
     for (int i = 0; i < NV; ++i) {
       const int c = 4 * lane + 128 * i;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) cur[i][k] += rs * (d[i][k] * gam[i][k] - a - xh[i][k] * bsum);
+      for (int k = 0; k < 4; ++k) {
+        cur[i][k] += rs * (d[i][k] * gam[i][k] - a - xh[i][k] * bsum);
+        ps[i][k] += cur[i][k];
+      }
       store4<float>(dx + row * C + c, cur[i]);
       if (dx_copy) store4<CopyT>(dx_copy + row * C + c, cur[i]);
     }
   }
-  float* out = ws + int64_t(blockIdx.x) * 2 * C;
+  const int parts = want_sum ? 3 : 2;
+  float* out = ws + int64_t(blockIdx.x) * parts * C;
+  for (int part = 0; part < parts; ++part) {
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-#pragma unroll
-    for (int i = 0; i < NV; ++i) store4<float>(&red[warp][4 * lane + 128 * i], half ? pb[i] : pg[i]);
+    for (int i = 0; i < NV; ++i)
+      store4<float>(&red[warp][4 * lane + 128 * i], part == 0 ? pg[i] : part == 1 ? pb[i] : ps[i]);
     __syncthreads();
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
       float t = 0.f;
 #pragma unroll
       for (int k = 0; k < 8; ++k) t += red[k][c];
-      out[half * C + c] = t;
+      out[part * C + c] = t;
     }
     __syncthreads();
   }
 }
 
-// out[c] (+)= sum_p ws[p][c] for c < n (c >= split goes to out1[c - split]),
+// out[c] (+)= sum_p ws[p][c] for c < n (c >= split goes to out1[c - split],
+// c >= 2 split to out2[c - 2 split]),
 // in a fixed order: 8 interleaved row slices per column, then the 8 slices.
 __global__ void __launch_bounds__(256) reduce_rows_kernel(const float* __restrict__ ws, int parts,
                                                           int n, float* __restrict__ out0,
                                                           float* __restrict__ out1, int split,
-                                                          int accumulate) {
+                                                          int accumulate,
+                                                          float* __restrict__ out2 = nullptr) {
   __shared__ float sh[8][33];
   const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + cx;
@@ -493,7 +500,7 @@ __global__ void __launch_bounds__(256) reduce_rows_kernel(const float* __restric
     float t = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) t += sh[k][cx];
-    float* o = c < split ? out0 + c : out1 + (c - split);
+    float* o = c < split ? out0 + c : c < 2 * split ? out1 + (c - split) : out2 + (c - 2 * split);
     *o = accumulate ? *o + t : t;
   }
 }
@@ -776,13 +783,14 @@ template int launch_layernorm_fwd<bf16>(const float*, const float*, const float*
 size_t layernorm_bwd_workspace(int64_t M, int C) {
   const int64_t parts =
       (C % 128 == 0 && C <= 1024) ? cdiv64(M, 8 * kLnVecRows) : cdiv64(M, kLnRowsPerBlock);
-  return size_t(parts) * 2 * C * sizeof(float);
+  // dgamma | dbeta | column sums of dx (generic path: colsum partials after)
+  return std::max(size_t(parts) * 3 * C * sizeof(float), colsum_workspace(M, C));
 }
 
 template <typename DyT, typename CopyT>
 int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const float* rstd,
                          const float* g, int64_t M, int C, float* dx, CopyT* dx_copy, float* dg,
-                         float* db, int accumulate, float* ws, cudaStream_t st) {
+                         float* db, float* dsum, int accumulate, float* ws, cudaStream_t st) {
   if (C > kLnMaxPerLane * 32) {
     gpt2_internal::set_error("layernorm: C above 1024");
     return GPT2_ERR_ARG;
@@ -794,13 +802,14 @@ int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const
 #define LNB(NV)                                                                              \
   case NV:                                                                                   \
     layernorm_bwd_vec_kernel<NV, DyT, CopyT><<<nb, 256, 0, st>>>(dy, x, mean, rstd, g, M, dx, \
-                                                                 dx_copy, ws);               \
+                                                                 dx_copy, ws, dsum != nullptr); \
     break;
       LNB(1) LNB(2) LNB(3) LNB(4) LNB(5) LNB(6) LNB(7) LNB(8)
 #undef LNB
     }
     COUNT_LAUNCH(1);
-    reduce_rows_kernel<<<cdiv(2 * C, 32), 256, 0, st>>>(ws, nb, 2 * C, dg, db, C, accumulate);
+    const int n = (dsum ? 3 : 2) * C;
+    reduce_rows_kernel<<<cdiv(n, 32), 256, 0, st>>>(ws, nb, n, dg, db, C, accumulate, dsum);
     COUNT_LAUNCH(1);
   } else {
     const int nb = int(cdiv64(M, kLnRowsPerBlock));
@@ -810,19 +819,73 @@ int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const
     // ws rows hold [dgamma | dbeta]; both halves are reduced in one pass
     reduce_ln_partials_kernel<<<cdiv(2 * C, 256), 256, 0, st>>>(ws, nb, C, dg, db, accumulate);
     COUNT_LAUNCH(1);
+    if (dsum) {  // column sums of the updated dx (same stream: ws is free again)
+      const int rc = launch_colsum<float>(dx, M, C, dsum, accumulate, ws, st);
+      if (rc) return rc;
+    }
   }
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;
 }
 template int launch_layernorm_bwd<float, float>(const float*, const float*, const float*,
                                                 const float*, const float*, int64_t, int, float*,
-                                                float*, float*, float*, int, float*, cudaStream_t);
+                                                float*, float*, float*, float*, int, float*,
+                                                cudaStream_t);
 template int launch_layernorm_bwd<bf16, bf16>(const bf16*, const float*, const float*, const float*,
                                               const float*, int64_t, int, float*, bf16*, float*,
-                                              float*, int, float*, cudaStream_t);
+                                              float*, float*, int, float*, cudaStream_t);
 template int launch_layernorm_bwd<float, bf16>(const float*, const float*, const float*,
                                                const float*, const float*, int64_t, int, float*,
-                                               bf16*, float*, float*, int, float*, cudaStream_t);
+                                               bf16*, float*, float*, float*, int, float*, cudaStream_t);
+
+// Column sums over a slab of kColRows rows, 16 bytes per lane and row: a block
+// of 32 lanes x 8 row slices covers 32*VEC columns; lanes of a warp read one
+// contiguous 32*16-byte row segment; the 8 slices are combined in shared
+// memory in a fixed order.  Requires N % VEC == 0 and 16-byte aligned rows.
+template <typename InT>
+__global__ void __launch_bounds__(256) colsum_vec_kernel(const InT* __restrict__ in, int64_t M,
+                                                         int N, float* __restrict__ ws) {
+  constexpr int VEC = 16 / int(sizeof(InT));
+  __shared__ float sh[8][32 * VEC];
+  const int lane = threadIdx.x & 31, ry = threadIdx.x >> 5;
+  const int n0 = (blockIdx.x * 32 + lane) * VEC;
+  const int64_t r0 = int64_t(blockIdx.y) * kColRows;
+  const int64_t r1 = min64(M, r0 + kColRows);
+  float acc[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+  if (n0 < N) {
+#pragma unroll 4
+    for (int64_t r = r0 + ry; r < r1; r += 8) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(in + r * N + n0));
+      if constexpr (VEC == 8) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h2[q]);
+          acc[2 * q] += f.x;
+          acc[2 * q + 1] += f.y;
+        }
+      } else {
+        acc[0] += __uint_as_float(u.x);
+        acc[1] += __uint_as_float(u.y);
+        acc[2] += __uint_as_float(u.z);
+        acc[3] += __uint_as_float(u.w);
+      }
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) sh[ry][lane * VEC + v] = acc[v];
+  __syncthreads();
+  for (int c = threadIdx.x; c < 32 * VEC; c += 256) {
+    const int n = blockIdx.x * 32 * VEC + c;
+    if (n >= N) continue;
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += sh[k][c];
+    ws[int64_t(blockIdx.y) * N + n] = t;
+  }
+}
 
 size_t colsum_workspace(int64_t M, int N) { return size_t(cdiv64(M, kColRows)) * N * sizeof(float); }
 
@@ -830,11 +893,20 @@ template <typename InT>
 int launch_colsum(const InT* in, int64_t M, int N, float* out, int accumulate, float* ws,
                   cudaStream_t st) {
   const int parts = int(cdiv64(M, kColRows));
-  dim3 grid(cdiv(N, kThreads), parts);
-  colsum_partial_kernel<InT><<<grid, kThreads, 0, st>>>(in, M, N, ws);
-  COUNT_LAUNCH(1);
-  reduce_partials_kernel<<<cdiv(N, kThreads), kThreads, 0, st>>>(ws, parts, N, out, accumulate);
-  COUNT_LAUNCH(1);
+  constexpr int VEC = 16 / int(sizeof(InT));
+  if (N % VEC == 0 && (reinterpret_cast<uintptr_t>(in) & 15) == 0) {
+    dim3 grid(cdiv(N, 32 * VEC), parts);
+    colsum_vec_kernel<InT><<<grid, 256, 0, st>>>(in, M, N, ws);
+    COUNT_LAUNCH(1);
+    reduce_rows_kernel<<<cdiv(N, 32), 256, 0, st>>>(ws, parts, N, out, nullptr, N, accumulate);
+    COUNT_LAUNCH(1);
+  } else {
+    dim3 grid(cdiv(N, kThreads), parts);
+    colsum_partial_kernel<InT><<<grid, kThreads, 0, st>>>(in, M, N, ws);
+    COUNT_LAUNCH(1);
+    reduce_partials_kernel<<<cdiv(N, kThreads), kThreads, 0, st>>>(ws, parts, N, out, accumulate);
+    COUNT_LAUNCH(1);
+  }
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;
 }

@@ -64,10 +64,13 @@ template <typename OutT>
 int launch_layernorm_fwd(const float* x, const float* g, const float* b, OutT* y, float* mean,
                          float* rstd, int64_t M, int C, float eps, cudaStream_t st);
 size_t layernorm_bwd_workspace(int64_t M, int C);
+// dx (+)= LN backward; dg, db (+)= dgamma, dbeta; dsum (nullable) (+)= column
+// sums of the updated dx.
 template <typename DyT, typename CopyT>
 int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const float* rstd,
                          const float* g, int64_t M, int C, float* dx, CopyT* dx_copy,
-                         float* dg, float* db, int accumulate, float* ws, cudaStream_t st);
+                         float* dg, float* db, float* dsum, int accumulate, float* ws,
+                         cudaStream_t st);
 size_t colsum_workspace(int64_t M, int N);
 template <typename InT>
 int launch_colsum(const InT* in, int64_t M, int N, float* out, int accumulate, float* ws,
