@@ -2,7 +2,7 @@
 // TMEM accumulators, operands loaded by TMA), head size 64, bf16 in / fp32
 // accumulate [ZERO: Attention, OpFlashAttention recomputes the scores in the
 // backward; LECTURE: flash attention, causal mask].  The [T, T] scores and
-// probabilities never leave TMEM, registers and shared memory.
+// probabilities never leave TMEM and registers.
 //
 // Every kernel: one CTA of 192 threads per block of 128 rows (queries, or keys
 // in dK/dV) = the 128 TMEM lanes, streaming 64-row tiles of the other operand:
@@ -10,17 +10,22 @@
 //   warp 1             owns the TMEM allocation (256 columns); one lane issues
 //                      the tcgen05.mma instructions and commits;
 //   warps 2-5          elementwise warpgroup, thread = row (TMEM lane
-//                      32 * (warp % 4) + lane): reads the score tile from TMEM,
-//                      writes probabilities / score gradients as bf16 K-major
-//                      operands (128-byte swizzle) to shared memory.
+//                      32 * (warp % 4) + lane): reads a score tile from TMEM
+//                      and writes the probabilities / score gradients back
+//                      as bf16 over the first 32 columns of that tile, where
+//                      the next MMA takes them as its A operand (kind::f16
+//                      with A in TMEM), so they never pass through shared
+//                      memory.
 // 256 TMEM columns and < 100 KB of shared memory let two CTAs share an SM, so
-// one CTA's elementwise work overlaps the other's MMAs.
+// one CTA's elementwise work overlaps the other's MMAs; the shared memory is
+// a deep ring of streamed K/V (or Q/dO) tiles that hides load latency.
 //
 // Forward (per 128 queries, 64-key tiles j <= diagonal):
 //   S_j = Q K_j^T (TMEM, double buffered); m, l kept in the log2 domain; the
 //   O accumulator (TMEM) is rescaled only when a row maximum grows by more than
 //   2^8 (probabilities are taken relative to the kept maximum, so they stay
-//   <= 256); P_j double buffered in shared memory; O += P_j V_j (V MN-major).
+//   <= 256); P_j (bf16) is written back over its own score buffer in TMEM
+//   and O += P_j V_j reads it from there (A operand in TMEM, V MN-major).
 // Backward, with Delta_i = dO_i . O_i and P = exp(S / sqrt(D) - lse):
 //   dK/dV kernel (per 128 keys, 64-query tiles i >= keys): S^T, dP^T = V dO^T,
 //   dS^T = P^T (dP^T - Delta); dV += P^T dO, dK += dS^T Q / sqrt(D);
@@ -40,7 +45,6 @@ constexpr int BR = 128;                 // rows per CTA = TMEM lanes
 constexpr int BS = 64;                  // rows of a streamed tile
 constexpr int kRowTile = BR * D * 2;    // 16 KB: 128 x 64 bf16
 constexpr int kStrTile = BS * D * 2;    // 8 KB: 64 x 64 bf16
-constexpr int kOpTile = BR * BS * 2;    // 16 KB: 128 x 64 bf16 operand from the warpgroup
 constexpr int kTmemCols = 256;
 constexpr int kThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -100,15 +104,6 @@ __device__ __forceinline__ float max64(const float (&x)[64]) {
 }
 __device__ __forceinline__ void wg_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// Row e of a 128 x 64 K-major bf16 operand tile (128-byte swizzle) from 32
-// packed bf16 pairs.
-__device__ __forceinline__ void put_row64(uint8_t* tile, int e, const uint32_t (&pk)[32]) {
-#pragma unroll
-  for (int ch = 0; ch < 8; ++ch)
-    *reinterpret_cast<uint4*>(tile + e * 128 + ((ch ^ (e & 7)) << 4)) =
-        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-}
-
 // Writes a 64-element fp32 row (two 32-column chunks) as bf16, times scale.
 __device__ __forceinline__ void store_row64(bf16* dst, const uint32_t (&a)[32],
                                             const uint32_t (&b)[32], float scale) {
@@ -136,8 +131,8 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // ====================================================================== forward
-constexpr int NSF = 3;  // K/V stages
-constexpr int kFwdSmem = kRowTile + NSF * 2 * kStrTile + 2 * kOpTile + 256 + 1024;
+constexpr int NSF = 5;  // K/V stages
+constexpr int kFwdSmem = kRowTile + NSF * 2 * kStrTile + 256 + 1024;
 
 struct FwdParams {
   int T, C, H;
@@ -154,9 +149,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sK = sQ + kRowTile;             // NSF x 8 KB
   const uint32_t sV = sK + NSF * kStrTile;       // NSF x 8 KB
-  uint8_t* pP = smem + kRowTile + 2 * NSF * kStrTile;
-  const uint32_t sP = smem_u32(pP);              // 2 x 16 KB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(pP + 2 * kOpTile);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRowTile + 2 * NSF * kStrTile);
   // q_full | kv_full[NSF] | kv_empty[NSF] | s_full[2] | s_free[2] | p_full[2] | o_done[2] | slot
   const uint32_t b_q = smem_u32(bars);
   auto b_kvf = [&](int s) { return smem_u32(bars + 1 + s); };
@@ -242,10 +235,12 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
+        // P_jj sits in the first 32 columns of its score buffer (two bf16 per
+        // column); S_{jj+2} reuses that buffer only after this MMA (issue order)
 #pragma unroll
         for (int k = 0; k < BS / 16; ++k)
-          umma_bf16(tO, desc_kmajor(sP + (jj & 1) * kOpTile, k),
-                    desc_mnmajor(sV + s * kStrTile, k), id_o, (jj > 0 || k > 0) ? 1u : 0u);
+          umma_bf16_ts(tO, tS + (jj & 1) * BS + k * 8, desc_mnmajor(sV + s * kStrTile, k), id_o,
+                       (jj > 0 || k > 0) ? 1u : 0u);
         umma_commit(b_od(jj & 1));
         umma_commit(b_kve(s));
         last_pv = jj;
@@ -328,16 +323,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_st32(tO + lo, f0);
         tmem_st32(tO + lo + 32, f1);
       }
-      // P buffer j%2 was last read by P_{j-2} V_{j-2}
-      if (j >= 2) {
-        w = mbar_wait(b_od(j & 1), ((j - 2) >> 1) & 1, p.err, 18);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-      }
-      put_row64(pP + (j & 1) * kOpTile, e, pk);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // P_j (bf16) over the first 32 columns of S_j's buffer, the A operand of P_j V_j
+      tmem_st32_async(tS + lo + (j & 1) * BS, pk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(b_pf(j & 1));
     }
@@ -365,7 +353,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ====================================================================== backward
-constexpr int NSB = 2;  // streamed-tile stages
 
 struct BwdParams {
   int T, C, H;
@@ -377,8 +364,14 @@ struct BwdParams {
 
 // ---------------------------------------------------------------- dK, dV
 // CTA: 128 keys kb*128 ..; 64-query tiles i from the diagonal to the end.
-// TMEM: S^T +0, dP^T +64, dV +128, dK +192.
-constexpr int kDkdvSmem = 2 * kRowTile + NSB * 2 * kStrTile + 2 * kOpTile + 2 * BS * 4 + 256 + 1024;
+// TMEM: S^T +0, dP^T +64, dV +128, dK +192.  The warpgroup writes P^T (bf16)
+// over the first 32 columns of S^T and dS^T over those of dP^T, where
+// dV += P^T dO and dK += dS^T Q read them (A operands in TMEM).  MMA order per
+// step i: dV(i-1) (after P^T_{i-1} is written); S^T_i; dK(i-1) (after dS^T_{i-1});
+// dP^T_i: each MMA that overwrites a TMEM region is issued after the one
+// that last reads it.
+constexpr int NSK = 4;  // Q/dO stages
+constexpr int kDkdvSmem = 2 * kRowTile + NSK * 2 * kStrTile + 2 * BS * 4 + 256 + 1024;
 
 __global__ void __launch_bounds__(kThreads, 2)
     fa_tc_dkdv_kernel(const __grid_constant__ CUtensorMap q128, const __grid_constant__ CUtensorMap q64,
@@ -386,22 +379,20 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sK = smem_u32(smem), sV = sK + kRowTile;
-  const uint32_t sQ = sV + kRowTile;            // NSB x 8 KB
-  const uint32_t sO = sQ + NSB * kStrTile;      // dO, NSB x 8 KB
-  uint8_t* pPt = smem + 2 * kRowTile + 2 * NSB * kStrTile;
-  uint8_t* pDt = pPt + kOpTile;
-  const uint32_t sPt = smem_u32(pPt), sDt = smem_u32(pDt);
-  float* sLD = reinterpret_cast<float*>(pDt + kOpTile);  // [64] -lse*log2e, [64] -delta
+  const uint32_t sQ = sV + kRowTile;            // NSK x 8 KB
+  const uint32_t sO = sQ + NSK * kStrTile;      // dO, NSK x 8 KB
+  float* sLD = reinterpret_cast<float*>(smem + 2 * kRowTile + 2 * NSK * kStrTile);  // [64] -lse*log2e, [64] -delta
   uint64_t* bars = reinterpret_cast<uint64_t*>(sLD + 2 * BS);
-  // kv_full | qo_full[NSB] | qo_empty[NSB] | s_full | s_free | p_full | mm_done | slot
+  // kv_full | qo_full[NSK] | qo_empty[NSK] | s_full | p_full | dp_full | ds_full | mm_done | slot
   const uint32_t b_kv = smem_u32(bars);
   auto b_qf = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto b_qe = [&](int s) { return smem_u32(bars + 1 + NSB + s); };
-  const uint32_t b_sf = smem_u32(bars + 1 + 2 * NSB);
-  const uint32_t b_sfr = smem_u32(bars + 2 + 2 * NSB);
-  const uint32_t b_pf = smem_u32(bars + 3 + 2 * NSB);
-  const uint32_t b_mm = smem_u32(bars + 4 + 2 * NSB);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5 + 2 * NSB);
+  auto b_qe = [&](int s) { return smem_u32(bars + 1 + NSK + s); };
+  const uint32_t b_sf = smem_u32(bars + 1 + 2 * NSK);
+  const uint32_t b_pf = smem_u32(bars + 2 + 2 * NSK);
+  const uint32_t b_dpf = smem_u32(bars + 3 + 2 * NSK);
+  const uint32_t b_df = smem_u32(bars + 4 + 2 * NSK);
+  const uint32_t b_mm = smem_u32(bars + 5 + 2 * NSK);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * NSK);
 
   const int kb = blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -414,13 +405,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (threadIdx.x == 0) {
     mbar_init(b_kv, 1);
-    for (int s = 0; s < NSB; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(b_qf(s), 1);
       mbar_init(b_qe(s), 1);
     }
     mbar_init(b_sf, 1);
-    mbar_init(b_sfr, 128);
     mbar_init(b_pf, 128);
+    mbar_init(b_dpf, 1);
+    mbar_init(b_df, 128);
     mbar_init(b_mm, 1);
     init_bar_fence();
   }
@@ -437,8 +429,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     tma_load_2d(sV, &q128, b_kv, 2 * C + h * D, row_base + kb * BR);
     int issued = 0;
     for (int i = 0; i < n; ++i) {
-      const int s = i % NSB;
-      if (!mbar_wait(b_qe(s), ((i / NSB) & 1) ^ 1, p.err, 21)) break;
+      const int s = i % NSK;
+      if (!mbar_wait(b_qe(s), ((i / NSK) & 1) ^ 1, p.err, 21)) break;
       mbar_expect_tx(b_qf(s), 2 * kStrTile);
       const int row = row_base + (qt0 + i) * BS;
       tma_load_2d(sQ + s * kStrTile, &q64, b_qf(s), h * D, row);
@@ -446,9 +438,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       ++issued;
     }
     mbar_wait(b_kv, 0, p.err, 25);
-    for (int q = 1; q <= min(issued, NSB); ++q) {
+    for (int q = 1; q <= min(issued, NSK); ++q) {
       const int idx = issued - q;
-      mbar_wait(b_qf(idx % NSB), uint32_t((idx / NSB) & 1), p.err, 25);
+      mbar_wait(b_qf(idx % NSK), uint32_t((idx / NSK) & 1), p.err, 25);
     }
   } else if (warp == 1 && lane == 0) {
     const uint32_t id_s = idesc_bf16(BR, BS, 0, 0);
@@ -456,37 +448,48 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool ok = mbar_wait(b_kv, 0, p.err, 22);
     int mm = 0;
     for (int i = 0; ok && i <= n; ++i) {
-      if (i < n) {
-        const int s = i % NSB;
-        if (!mbar_wait(b_qf(s), (i / NSB) & 1, p.err, 22) ||
-            !mbar_wait(b_sfr, (i & 1) ^ 1, p.err, 22)) {
+      const int s = i % NSK, si = (i + NSK - 1) % NSK;  // stages of tiles i and i-1
+      if (i >= 1) {  // dV += P^T_{i-1} dO_{i-1}
+        if (!mbar_wait(b_pf, (i - 1) & 1, p.err, 23)) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          umma_bf16(tS, desc_kmajor(sK, k), desc_kmajor(sQ + s * kStrTile, k), id_s, k > 0);
-          umma_bf16(tP, desc_kmajor(sV, k), desc_kmajor(sO + s * kStrTile, k), id_s, k > 0);
+        for (int k = 0; k < BS / 16; ++k)
+          umma_bf16_ts(tV, tS + k * 8, desc_mnmajor(sO + si * kStrTile, k), id_o,
+                       (i > 1 || k > 0) ? 1u : 0u);
+      }
+      if (i < n) {  // S^T_i = K Q_i^T
+        if (!mbar_wait(b_qf(s), (i / NSK) & 1, p.err, 22)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          umma_bf16(tS, desc_kmajor(sK, k), desc_kmajor(sQ + s * kStrTile, k), id_s, k > 0);
         umma_commit(b_sf);
       }
-      if (i >= 1) {
-        const int ii = i - 1, s = ii % NSB;
-        if (!mbar_wait(b_pf, ii & 1, p.err, 23)) {
+      if (i >= 1) {  // dK += dS^T_{i-1} Q_{i-1}
+        if (!mbar_wait(b_df, (i - 1) & 1, p.err, 24)) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < BS / 16; ++k) {
-          const uint32_t acc = (ii > 0 || k > 0) ? 1u : 0u;
-          umma_bf16(tV, desc_kmajor(sPt, k), desc_mnmajor(sO + s * kStrTile, k), id_o, acc);
-          umma_bf16(tKd, desc_kmajor(sDt, k), desc_mnmajor(sQ + s * kStrTile, k), id_o, acc);
-        }
+        for (int k = 0; k < BS / 16; ++k)
+          umma_bf16_ts(tKd, tP + k * 8, desc_mnmajor(sQ + si * kStrTile, k), id_o,
+                       (i > 1 || k > 0) ? 1u : 0u);
         umma_commit(b_mm);
-        umma_commit(b_qe(s));
+        umma_commit(b_qe(si));
         ++mm;
+      }
+      if (i < n) {  // dP^T_i = V dO_i^T
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          umma_bf16(tP, desc_kmajor(sV, k), desc_kmajor(sO + s * kStrTile, k), id_s, k > 0);
+        umma_commit(b_dpf);
       }
     }
     if (mm > 0) mbar_wait(b_mm, uint32_t((mm - 1) & 1), p.err, 26);
@@ -517,64 +520,67 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       // an expired wait (error word set) skips later waits but keeps the
       // warpgroup's named barriers in step, so no warp is left at one
-      if (ok) {
-        bool w = mbar_wait(b_sf, i & 1, p.err, 24);
-        if (i >= 1) w = w && mbar_wait(b_mm, (i - 1) & 1, p.err, 24);  // P^T / dS^T free
-        ok = w;
-      }
+      if (ok) ok = mbar_wait(b_sf, i & 1, p.err, 27);
       tc_fence_after();
       wg_bar();  // sLD of this tile visible
       const bool need_mask = q0 < kb * BR + BR || q0 + BS > T;
-      // two halves of 32 queries, so that only one half of S^T and dP^T is
-      // held in registers at a time; every 8 queries give one 16-byte chunk
-      // of the P^T and dS^T rows, written at once
+      // P^T = 2^(S^T sl2 - lse log2 e), masked; kept in fp32 for dS^T
+      float pv[64];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        uint32_t sx[32], dx[32];
+        uint32_t sx[32];
         tmem_ld32_async(tS + lo + 32 * hh, sx);
-        tmem_ld32_async(tP + lo + 32 * hh, dx);
         tmem_wait_ld(sx);
-        reg_after_wait(dx);
-        if (hh == 1) {  // S^T and dP^T read: the MMA may overwrite them
-          tc_fence_before();
-          mbar_arrive(b_sfr);
-        }
 #pragma unroll
-        for (int c8 = 0; c8 < 32; c8 += 8) {
-          uint32_t pp[4], pd[4];
-#pragma unroll
-          for (int c = c8; c < c8 + 8; c += 2) {
-            const int qc = 32 * hh + c;  // query column within the tile
-            const float2 nl = *reinterpret_cast<const float2*>(sLD + qc);       // -lse log2 e
-            const float2 nd = *reinterpret_cast<const float2*>(sLD + BS + qc);  // -delta
-            float t0, t1;
-            fma2(t0, t1, __uint_as_float(sx[c]), __uint_as_float(sx[c + 1]), sl2, sl2, nl.x,
-                 nl.y);
-            float p0 = ex2(t0), p1 = ex2(t1);
-            if (need_mask) {
-              if (q0 + qc < key || q0 + qc >= T) p0 = 0.f;
-              if (q0 + qc + 1 < key || q0 + qc + 1 >= T) p1 = 0.f;
-            }
-            float g0 = __uint_as_float(dx[c]), g1 = __uint_as_float(dx[c + 1]);
-            add2(g0, g1, nd.x, nd.y);  // dP - delta
-            mul2(g0, g1, p0, p1);      // dS = P (dP - delta)
-            pp[(c - c8) >> 1] = pack2(p0, p1);
-            pd[(c - c8) >> 1] = pack2(g0, g1);
+        for (int c = 0; c < 32; c += 2) {
+          const int qc = 32 * hh + c;  // query column within the tile
+          const float2 nl = *reinterpret_cast<const float2*>(sLD + qc);
+          float t0, t1;
+          fma2(t0, t1, __uint_as_float(sx[c]), __uint_as_float(sx[c + 1]), sl2, sl2, nl.x, nl.y);
+          pv[qc] = ex2(t0);
+          pv[qc + 1] = ex2(t1);
+          if (need_mask) {
+            if (q0 + qc < key || q0 + qc >= T) pv[qc] = 0.f;
+            if (q0 + qc + 1 < key || q0 + qc + 1 >= T) pv[qc + 1] = 0.f;
           }
-          const int ch = (32 * hh + c8) >> 3;  // 16-byte chunk of the 128-byte row
-          const int off = e * 128 + ((ch ^ (e & 7)) << 4);
-          *reinterpret_cast<uint4*>(pPt + off) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
-          *reinterpret_cast<uint4*>(pDt + off) = make_uint4(pd[0], pd[1], pd[2], pd[3]);
         }
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) pk[c >> 1] = pack2(pv[c], pv[c + 1]);
+        tmem_st32_async(tS + lo, pk);  // P^T over the first 32 columns of S^T
+        tmem_wait_st();
+      }
       tc_fence_before();
       mbar_arrive(b_pf);
+      if (ok) ok = mbar_wait(b_dpf, i & 1, p.err, 28);
+      tc_fence_after();
+      uint32_t pd[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t dx[32];
+        tmem_ld32_async(tP + lo + 32 * hh, dx);
+        tmem_wait_ld(dx);
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const int qc = 32 * hh + c;
+          const float2 nd = *reinterpret_cast<const float2*>(sLD + BS + qc);  // -delta
+          float g0 = __uint_as_float(dx[c]), g1 = __uint_as_float(dx[c + 1]);
+          add2(g0, g1, nd.x, nd.y);        // dP - delta
+          mul2(g0, g1, pv[qc], pv[qc + 1]);  // dS = P (dP - delta)
+          pd[qc >> 1] = pack2(g0, g1);
+        }
+      }
+      tmem_st32_async(tP + lo, pd);  // dS^T over the first 32 columns of dP^T
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(b_df);
       wg_bar();  // sLD may be rewritten for the next tile
     }
     ok = __all_sync(0xffffffffu, ok);
     if (ok && n > 0) {
-      bool w = mbar_wait(b_mm, (n - 1) & 1, p.err, 27);
+      bool w = mbar_wait(b_mm, (n - 1) & 1, p.err, 29);
       if (__all_sync(0xffffffffu, w)) {
         tc_fence_after();
         bf16* drow = p.dqkv + (int64_t(row_base) + key) * 3 * C + h * D;
@@ -599,8 +605,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 // ---------------------------------------------------------------- dQ
 // CTA: 128 queries qb*128 ..; 64-key tiles j up to the diagonal.
-// TMEM: S +0, dP +64, dQ +128.
-constexpr int kDqSmem = 2 * kRowTile + NSB * 2 * kStrTile + kOpTile + 256 + 1024;
+// TMEM: S +0, dP +64, dQ +128.  The warpgroup writes dS_j (bf16) over the
+// first 32 columns of dP, where dQ += dS_j K_j reads it (A operand in TMEM).
+// MMA order per step j: S_j (after the warpgroup has read S_{j-1});
+// dQ += dS_{j-1} K_{j-1} (after dS_{j-1} is written); dP_j (after that MMA,
+// which still reads the dP columns).  The warpgroup turns S_j into P while
+// those run, then waits for dP_j.
+constexpr int NSQ = 4;  // K/V stages
+constexpr int kDqSmem = 2 * kRowTile + NSQ * 2 * kStrTile + 256 + 1024;
 
 __global__ void __launch_bounds__(kThreads, 2)
     fa_tc_dq_kernel(const __grid_constant__ CUtensorMap q128, const __grid_constant__ CUtensorMap q64,
@@ -608,20 +620,19 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sQ = smem_u32(smem), sO = sQ + kRowTile;
-  const uint32_t sK = sO + kRowTile;            // NSB x 8 KB
-  const uint32_t sV = sK + NSB * kStrTile;      // NSB x 8 KB
-  uint8_t* pDs = smem + 2 * kRowTile + 2 * NSB * kStrTile;
-  const uint32_t sDs = smem_u32(pDs);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(pDs + kOpTile);
+  const uint32_t sK = sO + kRowTile;            // NSQ x 8 KB
+  const uint32_t sV = sK + NSQ * kStrTile;      // NSQ x 8 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kRowTile + 2 * NSQ * kStrTile);
+  // q_full | kv_full[NSQ] | kv_empty[NSQ] | s_full | s_read | dp_full | ds_full | dq_done | slot
   const uint32_t b_q = smem_u32(bars);
   auto b_kf = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto b_ke = [&](int s) { return smem_u32(bars + 1 + NSB + s); };
-  const uint32_t b_sf = smem_u32(bars + 1 + 2 * NSB);
-  const uint32_t b_sfr = smem_u32(bars + 2 + 2 * NSB);
-  const uint32_t b_df = smem_u32(bars + 3 + 2 * NSB);
-  const uint32_t b_mm = smem_u32(bars + 4 + 2 * NSB);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5 + 2 * NSB);
-
+  auto b_ke = [&](int s) { return smem_u32(bars + 1 + NSQ + s); };
+  const uint32_t b_sf = smem_u32(bars + 1 + 2 * NSQ);
+  const uint32_t b_sfr = smem_u32(bars + 2 + 2 * NSQ);
+  const uint32_t b_dpf = smem_u32(bars + 3 + 2 * NSQ);
+  const uint32_t b_df = smem_u32(bars + 4 + 2 * NSQ);
+  const uint32_t b_mm = smem_u32(bars + 5 + 2 * NSQ);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * NSQ);
   const int qb = gridDim.x - 1 - blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
   const int T = p.T, C = p.C;
@@ -629,15 +640,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int nkt = last_key / BS + 1;
   const int row_base = b * T;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-
   if (threadIdx.x == 0) {
     mbar_init(b_q, 1);
-    for (int s = 0; s < NSB; ++s) {
+    for (int s = 0; s < NSQ; ++s) {
       mbar_init(b_kf(s), 1);
       mbar_init(b_ke(s), 1);
     }
     mbar_init(b_sf, 1);
     mbar_init(b_sfr, 128);
+    mbar_init(b_dpf, 1);
     mbar_init(b_df, 128);
     mbar_init(b_mm, 1);
     init_bar_fence();
@@ -648,24 +659,23 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tP = tmem + 64, tQd = tmem + 128;
-
   if (warp == 0 && lane == 0) {
     mbar_expect_tx(b_q, 2 * kRowTile);
     tma_load_2d(sQ, &q128, b_q, h * D, row_base + qb * BR);
     tma_load_2d(sO, &o128, b_q, h * D, row_base + qb * BR);
     int issued = 0;
     for (int j = 0; j < nkt; ++j) {
-      const int s = j % NSB;
-      if (!mbar_wait(b_ke(s), ((j / NSB) & 1) ^ 1, p.err, 31)) break;
+      const int s = j % NSQ;
+      if (!mbar_wait(b_ke(s), ((j / NSQ) & 1) ^ 1, p.err, 31)) break;
       mbar_expect_tx(b_kf(s), 2 * kStrTile);
       tma_load_2d(sK + s * kStrTile, &q64, b_kf(s), C + h * D, row_base + j * BS);
       tma_load_2d(sV + s * kStrTile, &q64, b_kf(s), 2 * C + h * D, row_base + j * BS);
       ++issued;
     }
     mbar_wait(b_q, 0, p.err, 35);
-    for (int q = 1; q <= min(issued, NSB); ++q) {
+    for (int q = 1; q <= min(issued, NSQ); ++q) {
       const int idx = issued - q;
-      mbar_wait(b_kf(idx % NSB), uint32_t((idx / NSB) & 1), p.err, 35);
+      mbar_wait(b_kf(idx % NSQ), uint32_t((idx / NSQ) & 1), p.err, 35);
     }
   } else if (warp == 1 && lane == 0) {
     const uint32_t id_s = idesc_bf16(BR, BS, 0, 0);
@@ -673,23 +683,21 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool ok = mbar_wait(b_q, 0, p.err, 32);
     int mm = 0;
     for (int j = 0; ok && j <= nkt; ++j) {
+      const int s = j % NSQ;
       if (j < nkt) {
-        const int s = j % NSB;
-        if (!mbar_wait(b_kf(s), (j / NSB) & 1, p.err, 32) ||
-            !mbar_wait(b_sfr, (j & 1) ^ 1, p.err, 32)) {
+        if (!mbar_wait(b_kf(s), (j / NSQ) & 1, p.err, 32) ||
+            !mbar_wait(b_sfr, (j & 1) ^ 1, p.err, 32)) {  // S_{j-1} read
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < D / 16; ++k)
           umma_bf16(tS, desc_kmajor(sQ, k), desc_kmajor(sK + s * kStrTile, k), id_s, k > 0);
-          umma_bf16(tP, desc_kmajor(sO, k), desc_kmajor(sV + s * kStrTile, k), id_s, k > 0);
-        }
         umma_commit(b_sf);
       }
       if (j >= 1) {
-        const int jj = j - 1, s = jj % NSB;
+        const int jj = j - 1, sj = jj % NSQ;
         if (!mbar_wait(b_df, jj & 1, p.err, 33)) {
           ok = false;
           break;
@@ -697,11 +705,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < BS / 16; ++k)
-          umma_bf16(tQd, desc_kmajor(sDs, k), desc_mnmajor(sK + s * kStrTile, k), id_o,
-                    (jj > 0 || k > 0) ? 1u : 0u);
+          umma_bf16_ts(tQd, tP + k * 8, desc_mnmajor(sK + sj * kStrTile, k), id_o,
+                       (jj > 0 || k > 0) ? 1u : 0u);
         umma_commit(b_mm);
-        umma_commit(b_ke(s));
+        umma_commit(b_ke(sj));
         ++mm;
+      }
+      if (j < nkt) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          umma_bf16(tP, desc_kmajor(sO, k), desc_kmajor(sV + s * kStrTile, k), id_s, k > 0);
+        umma_commit(b_dpf);
       }
     }
     if (mm > 0) mbar_wait(b_mm, uint32_t((mm - 1) & 1), p.err, 36);
@@ -716,45 +730,57 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool ok = true;
     for (int j = 0; j < nkt; ++j) {
       bool w = mbar_wait(b_sf, j & 1, p.err, 34);
-      if (j >= 1) w = w && mbar_wait(b_mm, (j - 1) & 1, p.err, 34);  // dS buffer free
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t s0[32], s1[32], d0[32], d1[32];
+      uint32_t s0[32], s1[32];
       tmem_ld32_async(tS + lo, s0);
       tmem_ld32_async(tS + lo + 32, s1);
-      tmem_ld32_async(tP + lo, d0);
-      tmem_ld32_async(tP + lo + 32, d1);
       tmem_wait_ld(s0);
       reg_after_wait(s1);
-      reg_after_wait(d0);
-      reg_after_wait(d1);
       tc_fence_before();
       mbar_arrive(b_sfr);
       const int key0 = j * BS;
       const bool need_mask = key0 + BS - 1 > qb * BR || key0 + BS > T || qb * BR + BR > T;
-      uint32_t pk[32];
+      float pv[64];  // P = 2^(S sl2 - lse log2 e), masked
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
         const float sa = __uint_as_float(c < 32 ? s0[c] : s1[c - 32]);
         const float sb = __uint_as_float(c < 32 ? s0[c + 1] : s1[c - 31]);
-        float g0 = __uint_as_float(c < 32 ? d0[c] : d1[c - 32]);
-        float g1 = __uint_as_float(c < 32 ? d0[c + 1] : d1[c - 31]);
         float t0, t1;
         fma2(t0, t1, sa, sb, sl2, sl2, -L2, -L2);
-        float p0 = ex2(t0), p1 = ex2(t1);
+        pv[c] = ex2(t0);
+        pv[c + 1] = ex2(t1);
         if (need_mask) {
-          if (key0 + c > q || key0 + c >= T || q >= T) p0 = 0.f;
-          if (key0 + c + 1 > q || key0 + c + 1 >= T || q >= T) p1 = 0.f;
+          if (key0 + c > q || key0 + c >= T || q >= T) pv[c] = 0.f;
+          if (key0 + c + 1 > q || key0 + c + 1 >= T || q >= T) pv[c + 1] = 0.f;
         }
-        add2(g0, g1, -Dl, -Dl);  // dP - delta
-        mul2(g0, g1, p0, p1);    // dS = P (dP - delta)
-        pk[c >> 1] = pack2(g0, g1);
       }
-      put_row64(pDs, e, pk);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      w = mbar_wait(b_dpf, j & 1, p.err, 38);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t pk[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t d0[32];
+        tmem_ld32_async(tP + lo + 32 * hh, d0);
+        tmem_wait_ld(d0);
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float g0 = __uint_as_float(d0[c]), g1 = __uint_as_float(d0[c + 1]);
+          add2(g0, g1, -Dl, -Dl);                        // dP - delta
+          mul2(g0, g1, pv[32 * hh + c], pv[32 * hh + c + 1]);  // dS = P (dP - delta)
+          pk[16 * hh + (c >> 1)] = pack2(g0, g1);
+        }
+      }
+      // dS_j over the first 32 columns of dP_j (all of this row's dP_j read above)
+      tmem_st32_async(tP + lo, pk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(b_df);
     }
