@@ -84,10 +84,28 @@ struct TcParams {
   int M, N, K;
   int a_mn, b_mn;
   int tiles_m, tiles_n, splits, kb_per_split, num_kb, total_tiles;  // tiles of BM2 x BN
+  int n_fast;  // tile order: 1 = column tiles vary fastest (A panels read once)
   EpiParams ep;
   float* ws;
   int* err;
 };
+
+// Output tile, column tile and K split of linear tile index t.  Consecutive
+// tiles (processed at the same time by neighbouring CTA pairs) share the
+// panel of the larger operand, which is then read from memory once: rows of
+// A when n_fast, columns of B otherwise.
+__device__ __forceinline__ void tile_coords(const TcParams& p, int t, int& tm, int& tn, int& sp) {
+  const int mn = p.tiles_m * p.tiles_n;
+  sp = t / mn;
+  const int r = t - sp * mn;
+  if (p.n_fast) {
+    tn = r % p.tiles_n;
+    tm = r / p.tiles_n;
+  } else {
+    tm = r % p.tiles_m;
+    tn = r / p.tiles_m;
+  }
+}
 
 // Instruction descriptor: kind::f16, bf16 A and B, fp32 D, M = 256 (pair), N = BN.
 template <int BN>
@@ -485,7 +503,8 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
   int next_load = 0;  // next chunk whose input is to be fetched (leader only)
   auto issue_load = [&]() {
     const int tile = pair + (wg + 2 * (next_load / NCH)) * npairs;
-    const int tm = tile % p.tiles_m, tn = (tile / p.tiles_m) % p.tiles_n;
+    int tm, tn, sp;
+    tile_coords(p, tile, tm, tn, sp);
     const int slot = next_load % SL;
     mbar_expect_tx(lbar(slot), 8192);
     tma_load_2d(eb + slot * 8192, mi, lbar(slot), tn * BN + (next_load % NCH) * CW,
@@ -502,7 +521,8 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
   bool ok = true;
   for (int t_local = wg, tile = pair + wg * npairs; tile < p.total_tiles;
        t_local += 2, tile += 2 * npairs) {
-    const int tm = tile % p.tiles_m, tn = (tile / p.tiles_m) % p.tiles_n;
+    int tm, tn, sp;
+    tile_coords(p, tile, tm, tn, sp);
     const int acc = wg;
     const int m0 = tm * BM2 + rank * BM;  // first row of this CTA's half
     if (ok) ok = mbar_wait(tfull(acc), (t_local >> 1) & 1, p.err, 4);
@@ -672,9 +692,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0;
     bool ok = true;
     for (int tile = pair; tile < p.total_tiles && ok; tile += npairs) {
-      const int tm = tile % p.tiles_m;
-      const int rest = tile / p.tiles_m;
-      const int tn = rest % p.tiles_n, sp = rest / p.tiles_n;
+      int tm, tn, sp;
+      tile_coords(p, tile, tm, tn, sp);
       const int kb0 = sp * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
       const int ma = tm * BM2 + int(rank) * BM, nb = tn * BN + int(rank) * (BN / 2);
       for (int kb = kb0; kb < kb1; ++kb) {
@@ -719,8 +738,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int t_local = 0;
     bool ok = true;
     for (int tile = pair; tile < p.total_tiles && ok; tile += npairs, ++t_local) {
-      const int rest = tile / p.tiles_m;
-      const int sp = rest / p.tiles_n;
+      int tm, tn, sp;
+      tile_coords(p, tile, tm, tn, sp);
       const int kb0 = sp * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
       const int acc = t_local & 1;
       // arrivals of both CTAs' epilogues (release at cluster scope)
@@ -779,9 +798,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int t_local = wg, tile = pair + wg * npairs; tile < p.total_tiles;
          t_local += 2, tile += 2 * npairs) {
-      const int tm = tile % p.tiles_m;
-      const int rest = tile / p.tiles_m;
-      const int tn = rest % p.tiles_n, sp = rest / p.tiles_n;
+      int tm, tn, sp;
+      tile_coords(p, tile, tm, tn, sp);
       const int acc = wg;
       const int m0 = tm * BM2 + int(rank) * BM;
       // an expired wait (error word set) skips later waits, never the barriers
@@ -1053,6 +1071,7 @@ int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
   p.kb_per_split = cdiv(p.num_kb, splits);
   p.splits = cdiv(p.num_kb, p.kb_per_split);
   p.total_tiles = p.tiles_m * p.tiles_n * p.splits;
+  p.n_fast = g.M > g.N ? 1 : 0;  // A (M x K) is the larger operand: read its panels once
   p.ep = g.ep;
   p.ws = p.splits > 1 ? g.ws : nullptr;
   p.err = device_error_word();
