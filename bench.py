@@ -21,6 +21,7 @@ workload, each step a bounded sample of it.  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -58,6 +59,28 @@ def n_params(w):
 def flops_per_token(w):
     """Algorithmic: 6N (matmul fwd+bwd) + 6*L*C*T (causal attention)."""
     return 6 * n_params(w) + 6 * w["n_layer"] * w["n_embd"] * w["T"]
+
+
+def stored_traffic(group, workload, launches_per_step):
+    """DRAM bytes per launch of a kernel group from the committed ncu capture
+    (profiles/gemm_dram_traffic_*.json), or None when that capture was taken on
+    another workload or on kernel sources that have changed since."""
+    path = os.path.join(ROOT, "profiles", "gemm_dram_traffic_gpt2_124m_b16_t1024.json")
+    if workload != "gpt2-124m" or not os.path.exists(path):
+        return None, None
+    rec = json.load(open(path))
+    if group not in rec:
+        return None, None
+    h = hashlib.sha256()
+    for f in sorted(rec["kernel_sources"]):
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if h.hexdigest() != rec["kernel_sources_sha256"]:
+        return None, "kernel sources changed since the capture"
+    g = rec[group]
+    per_launch = g["dram_bytes_per_step"] / max(1.0, launches_per_step)
+    return per_launch, ("ncu dram__bytes_read.sum + dram__bytes_write.sum over one step "
+                        f"({g['kernel_launches_per_step']} launches), per launch; "
+                        "profiles/gemm_dram_traffic_gpt2_124m_b16_t1024.md")
 
 
 def load_peaks():
@@ -298,11 +321,12 @@ def main():
     dom = max(groups, key=lambda k: groups[k]["ms"])
     d = groups[dom]
     per_launch_ms = d["ms"] / max(1, d["launches"])
+    traffic, traffic_src = stored_traffic(dom, args.workload, d["launches"] / max(1, args.steps))
     if d["flops"] > 0 and dom in ("gemm", "lmhead", "attn_fwd", "attn_bwd"):
         ach = d["flops"] / (d["ms"] / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": None,
+                "frac": ach / peak, "traffic": traffic, "traffic_source": traffic_src,
                 "kernel": dom, "launches": d["launches"], "ms_per_launch": per_launch_ms,
                 "peak_source": f"{peak_src} bf16 sustained",
                 "measured": "CUDA events around every launch of the group, on the library's stream, "
@@ -311,7 +335,8 @@ def main():
         ach = d["bytes"] / (d["ms"] / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                "traffic": None, "kernel": dom, "launches": d["launches"],
+                "traffic": traffic, "traffic_source": traffic_src, "kernel": dom,
+                "launches": d["launches"],
                 "ms_per_launch": per_launch_ms, "peak_source": f"{peak_src} copy",
                 "measured": "CUDA events around every launch of the group, on the library's stream, "
                             "over a profiled repeat of the timed steps"}
