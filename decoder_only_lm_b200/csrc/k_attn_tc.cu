@@ -279,8 +279,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (need_mask) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (key0 + i > q || key0 + i >= T) x[i] = -INFINITY;
+        for (int i = 0; i < 64; ++i) x[i] = (key0 + i > q || key0 + i >= T) ? -INFINITY : x[i];
       }
       // running maximum in log2 units (scale > 0 commutes with max)
       const float mn = fmaxf(m, max64(x) * sl2);
@@ -290,6 +289,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       // p = 2^(x sl2 - mu): one packed FMA per pair, ex2 per element, packed sums
       uint32_t pk[32];
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+      // branch-free (so the pairs interleave); masked scores are -inf and
+      // ex2.approx(-inf) is exactly 0
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
         float t0, t1;
@@ -532,18 +533,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_ld32_async(tS + lo + 32 * hh, sx);
         tmem_wait_ld(sx);
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < 32; c += 2) {  // branch-free, so the pairs interleave
           const int qc = 32 * hh + c;  // query column within the tile
           const float2 nl = *reinterpret_cast<const float2*>(sLD + qc);
           float t0, t1;
           fma2(t0, t1, __uint_as_float(sx[c]), __uint_as_float(sx[c + 1]), sl2, sl2, nl.x, nl.y);
           pv[qc] = ex2(t0);
           pv[qc + 1] = ex2(t1);
-          if (need_mask) {
-            if (q0 + qc < key || q0 + qc >= T) pv[qc] = 0.f;
-            if (q0 + qc + 1 < key || q0 + qc + 1 >= T) pv[qc + 1] = 0.f;
-          }
         }
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int qc = 0; qc < 64; ++qc)
+          pv[qc] = (q0 + qc < key || q0 + qc >= T) ? 0.f : pv[qc];
       }
       {
         uint32_t pk[32];
@@ -746,17 +748,18 @@ __global__ void __launch_bounds__(kThreads, 2)
       const bool need_mask = key0 + BS - 1 > qb * BR || key0 + BS > T || qb * BR + BR > T;
       float pv[64];  // P = 2^(S sl2 - lse log2 e), masked
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < 64; c += 2) {  // branch-free, so the pairs interleave
         const float sa = __uint_as_float(c < 32 ? s0[c] : s1[c - 32]);
         const float sb = __uint_as_float(c < 32 ? s0[c + 1] : s1[c - 31]);
         float t0, t1;
         fma2(t0, t1, sa, sb, sl2, sl2, -L2, -L2);
         pv[c] = ex2(t0);
         pv[c + 1] = ex2(t1);
-        if (need_mask) {
-          if (key0 + c > q || key0 + c >= T || q >= T) pv[c] = 0.f;
-          if (key0 + c + 1 > q || key0 + c + 1 >= T || q >= T) pv[c + 1] = 0.f;
-        }
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          pv[c] = (key0 + c > q || key0 + c >= T || q >= T) ? 0.f : pv[c];
       }
       w = mbar_wait(b_dpf, j & 1, p.err, 38);
       if (!__all_sync(0xffffffffu, w)) {
