@@ -211,6 +211,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------ MMA
     const uint32_t id_s = idesc_bf16(BR, BS, 0, 0);
     const uint32_t id_o = idesc_bf16(BR, D, 0, 1);
+    // slice-0 descriptors, stage s adds s * kStrTile bytes
+    const uint64_t dQ = desc_kmajor(sQ, 0), dK = desc_kmajor(sK, 0), dVm = desc_mnmajor(sV, 0);
     bool ok = mbar_wait(b_q, 0, p.err, 12);
     int last_pv = -1;
     for (int j = 0; ok && j <= nkt; ++j) {
@@ -224,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tS + (j & 1) * BS, desc_kmajor(sQ, k), desc_kmajor(sK + s * kStrTile, k), id_s,
+          umma_bf16(tS + (j & 1) * BS, desc_at_k_kmajor(dQ, k),
+                    desc_at_k_kmajor(desc_offset(dK, s * kStrTile), k), id_s,
                     k > 0);
         umma_commit(b_sf(j & 1));
       }
@@ -239,7 +242,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         // column); S_{jj+2} reuses that buffer only after this MMA (issue order)
 #pragma unroll
         for (int k = 0; k < BS / 16; ++k)
-          umma_bf16_ts(tO, tS + (jj & 1) * BS + k * 8, desc_mnmajor(sV + s * kStrTile, k), id_o,
+          umma_bf16_ts(tO, tS + (jj & 1) * BS + k * 8,
+                       desc_at_k_mnmajor(desc_offset(dVm, s * kStrTile), k), id_o,
                        (jj > 0 || k > 0) ? 1u : 0u);
         umma_commit(b_od(jj & 1));
         umma_commit(b_kve(s));
@@ -446,6 +450,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp == 1 && lane == 0) {
     const uint32_t id_s = idesc_bf16(BR, BS, 0, 0);
     const uint32_t id_o = idesc_bf16(BR, D, 0, 1);
+    // slice-0 descriptors, stage s adds s * kStrTile bytes
+    const uint64_t dK = desc_kmajor(sK, 0), dV = desc_kmajor(sV, 0);
+    const uint64_t dQ = desc_kmajor(sQ, 0), dO = desc_kmajor(sO, 0);
+    const uint64_t dQm = desc_mnmajor(sQ, 0), dOm = desc_mnmajor(sO, 0);
     bool ok = mbar_wait(b_kv, 0, p.err, 22);
     int mm = 0;
     for (int i = 0; ok && i <= n; ++i) {
@@ -458,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < BS / 16; ++k)
-          umma_bf16_ts(tV, tS + k * 8, desc_mnmajor(sO + si * kStrTile, k), id_o,
+          umma_bf16_ts(tV, tS + k * 8, desc_at_k_mnmajor(desc_offset(dOm, si * kStrTile), k), id_o,
                        (i > 1 || k > 0) ? 1u : 0u);
       }
       if (i < n) {  // S^T_i = K Q_i^T
@@ -469,7 +477,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tS, desc_kmajor(sK, k), desc_kmajor(sQ + s * kStrTile, k), id_s, k > 0);
+          umma_bf16(tS, desc_at_k_kmajor(dK, k), desc_at_k_kmajor(desc_offset(dQ, s * kStrTile), k),
+                    id_s, k > 0);
         umma_commit(b_sf);
       }
       if (i >= 1) {  // dK += dS^T_{i-1} Q_{i-1}
@@ -480,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < BS / 16; ++k)
-          umma_bf16_ts(tKd, tP + k * 8, desc_mnmajor(sQ + si * kStrTile, k), id_o,
+          umma_bf16_ts(tKd, tP + k * 8, desc_at_k_mnmajor(desc_offset(dQm, si * kStrTile), k), id_o,
                        (i > 1 || k > 0) ? 1u : 0u);
         umma_commit(b_mm);
         umma_commit(b_qe(si));
@@ -489,7 +498,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (i < n) {  // dP^T_i = V dO_i^T
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tP, desc_kmajor(sV, k), desc_kmajor(sO + s * kStrTile, k), id_s, k > 0);
+          umma_bf16(tP, desc_at_k_kmajor(dV, k), desc_at_k_kmajor(desc_offset(dO, s * kStrTile), k),
+                    id_s, k > 0);
         umma_commit(b_dpf);
       }
     }
@@ -607,12 +617,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 // ---------------------------------------------------------------- dQ
 // CTA: 128 queries qb*128 ..; 64-key tiles j up to the diagonal.
-// TMEM: S +0, dP +64, dQ +128.  The warpgroup writes dS_j (bf16) over the
-// first 32 columns of dP, where dQ += dS_j K_j reads it (A operand in TMEM).
-// MMA order per step j: S_j (after the warpgroup has read S_{j-1});
-// dQ += dS_{j-1} K_{j-1} (after dS_{j-1} is written); dP_j (after that MMA,
-// which still reads the dP columns).  The warpgroup turns S_j into P while
-// those run, then waits for dP_j.
+// TMEM: S +0, dP +64, dQ +128, dS +192.  The warpgroup writes dS_j (bf16,
+// 32 columns) to its own region, where dQ += dS_j K_j reads it (A operand in
+// TMEM).  MMA order per step j: S_j (once the warpgroup has read S_{j-1});
+// dP_j (once it has read dP_{j-1}); dQ += dS_{j-1} K_{j-1} (once dS_{j-1} is
+// written).  S_j and dP_j are so issued while the warpgroup still works on
+// tile j-1; it waits for dQ(j-1) only before it overwrites dS.
 constexpr int NSQ = 4;  // K/V stages
 constexpr int kDqSmem = 2 * kRowTile + NSQ * 2 * kStrTile + 256 + 1024;
 
@@ -625,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t sK = sO + kRowTile;            // NSQ x 8 KB
   const uint32_t sV = sK + NSQ * kStrTile;      // NSQ x 8 KB
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kRowTile + 2 * NSQ * kStrTile);
-  // q_full | kv_full[NSQ] | kv_empty[NSQ] | s_full | s_read | dp_full | ds_full | dq_done | slot
+  // q_full | kv_full[NSQ] | kv_empty[NSQ] | s_full | s_read | dp_full | ds_full | dq_done | dp_read | slot
   const uint32_t b_q = smem_u32(bars);
   auto b_kf = [&](int s) { return smem_u32(bars + 1 + s); };
   auto b_ke = [&](int s) { return smem_u32(bars + 1 + NSQ + s); };
@@ -634,7 +644,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t b_dpf = smem_u32(bars + 3 + 2 * NSQ);
   const uint32_t b_df = smem_u32(bars + 4 + 2 * NSQ);
   const uint32_t b_mm = smem_u32(bars + 5 + 2 * NSQ);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * NSQ);
+  const uint32_t b_dpr = smem_u32(bars + 6 + 2 * NSQ);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * NSQ);
   const int qb = gridDim.x - 1 - blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
   const int T = p.T, C = p.C;
@@ -653,6 +664,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(b_dpf, 1);
     mbar_init(b_df, 128);
     mbar_init(b_mm, 1);
+    mbar_init(b_dpr, 128);
     init_bar_fence();
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -660,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + 64, tQd = tmem + 128;
+  const uint32_t tS = tmem, tP = tmem + 64, tQd = tmem + 128, tDs = tmem + 192;
   if (warp == 0 && lane == 0) {
     mbar_expect_tx(b_q, 2 * kRowTile);
     tma_load_2d(sQ, &q128, b_q, h * D, row_base + qb * BR);
@@ -682,6 +694,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp == 1 && lane == 0) {
     const uint32_t id_s = idesc_bf16(BR, BS, 0, 0);
     const uint32_t id_o = idesc_bf16(BR, D, 0, 1);
+    // slice-0 descriptors, stage s adds s * kStrTile bytes
+    const uint64_t dQ = desc_kmajor(sQ, 0), dO = desc_kmajor(sO, 0);
+    const uint64_t dK = desc_kmajor(sK, 0), dV = desc_kmajor(sV, 0), dKm = desc_mnmajor(sK, 0);
     bool ok = mbar_wait(b_q, 0, p.err, 32);
     int mm = 0;
     for (int j = 0; ok && j <= nkt; ++j) {
@@ -695,8 +710,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tS, desc_kmajor(sQ, k), desc_kmajor(sK + s * kStrTile, k), id_s, k > 0);
+          umma_bf16(tS, desc_at_k_kmajor(dQ, k), desc_at_k_kmajor(desc_offset(dK, s * kStrTile), k),
+                    id_s, k > 0);
         umma_commit(b_sf);
+        if (!mbar_wait(b_dpr, (j & 1) ^ 1, p.err, 32)) {  // dP_{j-1} read
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          umma_bf16(tP, desc_at_k_kmajor(dO, k), desc_at_k_kmajor(desc_offset(dV, s * kStrTile), k),
+                    id_s, k > 0);
+        umma_commit(b_dpf);
       }
       if (j >= 1) {
         const int jj = j - 1, sj = jj % NSQ;
@@ -707,17 +733,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < BS / 16; ++k)
-          umma_bf16_ts(tQd, tP + k * 8, desc_mnmajor(sK + sj * kStrTile, k), id_o,
+          umma_bf16_ts(tQd, tDs + k * 8, desc_at_k_mnmajor(desc_offset(dKm, sj * kStrTile), k), id_o,
                        (jj > 0 || k > 0) ? 1u : 0u);
         umma_commit(b_mm);
         umma_commit(b_ke(sj));
         ++mm;
-      }
-      if (j < nkt) {
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tP, desc_kmajor(sO, k), desc_kmajor(sV + s * kStrTile, k), id_s, k > 0);
-        umma_commit(b_dpf);
       }
     }
     if (mm > 0) mbar_wait(b_mm, uint32_t((mm - 1) & 1), p.err, 36);
@@ -767,22 +787,32 @@ __global__ void __launch_bounds__(kThreads, 2)
         break;
       }
       tc_fence_after();
+      uint32_t d0[32], d1[32];
+      tmem_ld32_async(tP + lo, d0);
+      tmem_ld32_async(tP + lo + 32, d1);
+      tmem_wait_ld(d0);
+      reg_after_wait(d1);
+      tc_fence_before();
+      mbar_arrive(b_dpr);  // dP_j read: the MMA may write dP_{j+1}
       uint32_t pk[32];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t d0[32];
-        tmem_ld32_async(tP + lo + 32 * hh, d0);
-        tmem_wait_ld(d0);
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float g0 = __uint_as_float(d0[c]), g1 = __uint_as_float(d0[c + 1]);
-          add2(g0, g1, -Dl, -Dl);                        // dP - delta
-          mul2(g0, g1, pv[32 * hh + c], pv[32 * hh + c + 1]);  // dS = P (dP - delta)
-          pk[16 * hh + (c >> 1)] = pack2(g0, g1);
-        }
+      for (int c = 0; c < 64; c += 2) {
+        float g0 = __uint_as_float(c < 32 ? d0[c] : d1[c - 32]);
+        float g1 = __uint_as_float(c < 32 ? d0[c + 1] : d1[c - 31]);
+        add2(g0, g1, -Dl, -Dl);            // dP - delta
+        mul2(g0, g1, pv[c], pv[c + 1]);    // dS = P (dP - delta)
+        pk[c >> 1] = pack2(g0, g1);
       }
-      // dS_j over the first 32 columns of dP_j (all of this row's dP_j read above)
-      tmem_st32_async(tP + lo, pk);
+      // dS_{j-1} consumed by its dQ MMA before dS_j overwrites it
+      if (j >= 1) {
+        w = mbar_wait(b_mm, (j - 1) & 1, p.err, 39);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      tmem_st32_async(tDs + lo, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(b_df);

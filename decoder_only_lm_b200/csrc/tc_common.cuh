@@ -293,6 +293,18 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int k) {
   return smem_desc(tile + k * 16 * 128, BK * 128, 1024);
 }
 
+// Descriptors of further slices from the one of slice 0 (the address field
+// counts 16-byte units and never carries: shared memory is < 256 KB): the
+// k-th 16-element K slice of a K-major tile is 32 B on (+2), of an MN-major
+// tile 16 rows of 128 B on (+128); another tile `bytes` further is +bytes/16.
+__device__ __forceinline__ uint64_t desc_at_k_kmajor(uint64_t d0, int k) { return d0 + uint64_t(2 * k); }
+__device__ __forceinline__ uint64_t desc_at_k_mnmajor(uint64_t d0, int k) {
+  return d0 + uint64_t(128 * k);
+}
+__device__ __forceinline__ uint64_t desc_offset(uint64_t d, uint32_t bytes) {
+  return d + uint64_t(bytes >> 4);
+}
+
 // tcgen05.ld of 32 columns without waiting; the registers are valid only
 // after tmem_wait_ld(r) (which names them, so no use is scheduled earlier) and,
 // for further batches loaded before the same wait, reg_after_wait(r).
