@@ -43,7 +43,14 @@ WORKLOADS = {
                       max_T=1024, B=16, T=1024),
     "gpt2-350m": dict(n_layer=24, n_embd=1024, n_head=16, vocab_size=50257, padded_vocab=50304,
                       max_T=1024, B=16, T=1024),
+    # micro-batch 64 x 8 accumulation (524,288 tokens per optimizer step), warmup + cosine LR,
+    # then a 20-batch evaluation pass on a separate stream (seed 4)
+    "gpt2-124m-accum": dict(n_layer=12, n_embd=768, n_head=12, vocab_size=50257,
+                            padded_vocab=50304, max_T=1024, B=64, T=1024, accum=8, eval_batches=20),
 }
+# schedule of the accumulation workload: max 6e-4, min 6e-5, 100 warmup steps; the decay
+# length is the run's choice (its token budget), 10,000 optimizer steps here
+LR_SCHEDULE = dict(max_lr=6e-4, min_lr=6e-5, warmup_steps=100, total_steps=10000)
 METRIC = "GPT-2 124M training tokens/s (fwd+bwd+AdamW, T=1024, bf16) and MFU"
 DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -171,13 +178,13 @@ def oracle_sample(w, stream, T_sample, with_adamw=True):
 
 def cpu_baseline(w, stream):
     """The oracle on a bounded sample: one 1 x T sequence fwd+bwd and one AdamW
-    pass, scaled to a B x T step."""
-    T = w["T"]
+    pass, scaled to one optimizer step (accum x B x T tokens)."""
+    T, acc = w["T"], w.get("accum", 1)
     t_seq, t_adam, cores = oracle_sample(w, stream, T)
-    step_s = w["B"] * t_seq + t_adam
-    return {"value": w["B"] * T / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    step_s = acc * w["B"] * t_seq + t_adam
+    return {"value": acc * w["B"] * T / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"oracle fp32: fwd+bwd of 1 x {T} tokens ({t_seq:.1f} s) + one clip+AdamW over "
-                      f"all {n_params(w)} params ({t_adam:.2f} s), scaled to one {w['B']}x{T} step"}
+                      f"all {n_params(w)} params ({t_adam:.2f} s), scaled to one {acc}x{w['B']}x{T} step"}
 
 
 def run_reference(args, w, wname):
@@ -191,7 +198,7 @@ def run_reference(args, w, wname):
                      w["max_T"])
     p = m.pack(synth.init_params(0, m.shapes()), np.float32)
     mm, vv = np.zeros_like(p), np.zeros_like(p)
-    share = T_s / (w["B"] * w["T"])  # one AdamW per B*T tokens
+    share = T_s / (w.get("accum", 1) * w["B"] * w["T"])  # one AdamW per optimizer step
     times = []
     for i in range(args.warmup + args.steps):
         x, y = oracle.batch_from_stream(stream, i * T_s, 1, T_s)
@@ -206,7 +213,8 @@ def run_reference(args, w, wname):
     total = sum(times)
     value = args.steps * T_s / total
     sample = (f"oracle fp32 on the host cores: each step = fwd+bwd of 1 x {T_s} tokens of the "
-              f"{wname} workload + AdamW time x {share:.4f} (one update per {w['B']}x{w['T']} tokens)")
+              f"{wname} workload + AdamW time x {share:.4f} "
+              f"(one update per {w.get('accum', 1)}x{w['B']}x{w['T']} tokens)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
@@ -251,8 +259,10 @@ def main():
     import decoder_only_lm_b200 as g
 
     B, T = w["B"], w["T"]
+    acc = w.get("accum", 1)  # micro-batches per optimizer step
     steps_total = args.warmup + args.steps
-    n_tok = (steps_total * world + world + 2) * B * T + 1
+    # timed steps, then the e2e leg's windows at step index steps_total + 1
+    n_tok = ((steps_total + 2) * acc * world + 2) * B * T + 1
     stream_np = synth.token_stream(3, n_tok)
     stream = torch.from_numpy(stream_np.view(np.int16)).cuda()
     model = g.GPT2(w["n_layer"], w["n_embd"], w["n_head"], w["vocab_size"], w["padded_vocab"],
@@ -260,15 +270,24 @@ def main():
     model.set_params(synth.init_params(0, model.shapes()))
     grad_arena = model.arena(g.GRAD) if world > 1 else None
 
+    def hp_at(i):
+        hp = dict(HP)
+        if acc > 1:
+            hp["lr"] = g.cosine_lr(i, **LR_SCHEDULE)
+        return hp
+
     def step(i):
-        off = (i * world + rank) * B * T
-        x, y = model.batch_from_stream(stream, off, B, T)
+        # one optimizer step: acc micro-batches whose gradients add up (loss scaled
+        # by 1/acc), consecutive windows of the stream (rank-offset for data parallel)
         model.zero_grad()
-        model.forward_loss(x, y, loss=False)
-        model.backward(1.0)
+        for a in range(acc):
+            off = ((i * acc + a) * world + rank) * B * T
+            x, y = model.batch_from_stream(stream, off, B, T)
+            model.forward_loss(x, y, loss=False)
+            model.backward(1.0 / acc)
         if world > 1:
             dist.all_reduce(grad_arena, op=dist.ReduceOp.AVG)
-        model.clip_adamw_step(**HP, norm=False)
+        model.clip_adamw_step(**hp_at(i), norm=False)
 
     for i in range(args.warmup):
         step(i)
@@ -310,7 +329,7 @@ def main():
     model.synchronize()
 
     ms_per_step = ms / args.steps
-    tokens = args.steps * B * T * world
+    tokens = args.steps * acc * B * T * world
     value = tokens / (ms / 1e3)
     fpt = flops_per_token(w)
     achieved_tflops = value * fpt / 1e12
@@ -344,26 +363,30 @@ def main():
     # end to end through the public API: host tokens in, loss + norm out, every step
     e2e = None
     if not args.no_e2e:
-        xh = torch.empty((B, T), dtype=torch.int32, pin_memory=True)
-        yh = torch.empty((B, T), dtype=torch.int32, pin_memory=True)
+        # one pinned host buffer pair per micro-batch, filled before the timed step
+        xh = torch.empty((acc, B, T), dtype=torch.int32, pin_memory=True)
+        yh = torch.empty((acc, B, T), dtype=torch.int32, pin_memory=True)
         k_e2e = max(3, args.steps // 2)
         times = []
         for i in range(k_e2e + 1):
-            off = ((steps_total + 1) * world + rank) * B * T
-            win = stream_np[off:off + B * T + 1].astype(np.int32)
-            xh.numpy()[:] = win[:-1].reshape(B, T)
-            yh.numpy()[:] = win[1:].reshape(B, T)
+            for m_ in range(acc):
+                off = (((steps_total + 1) * acc + m_) * world + rank) * B * T
+                win = stream_np[off:off + B * T + 1].astype(np.int32)
+                xh.numpy()[m_] = win[:-1].reshape(B, T)
+                yh.numpy()[m_] = win[1:].reshape(B, T)
             torch.cuda.synchronize()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(st)
-            if world == 1:
-                model.train_step(xh.numpy(), yh.numpy(), **HP, read=True)
+            if world == 1 and acc == 1:
+                model.train_step(xh.numpy()[0], yh.numpy()[0], **HP, read=True)
             else:
                 model.zero_grad()
-                model.forward_loss(xh.numpy(), yh.numpy(), loss=True)
-                model.backward(1.0)
-                dist.all_reduce(grad_arena, op=dist.ReduceOp.AVG)
-                model.clip_adamw_step(**HP, norm=True)
+                for m_ in range(acc):
+                    model.forward_loss(xh.numpy()[m_], yh.numpy()[m_], loss=(m_ == acc - 1))
+                    model.backward(1.0 / acc)
+                if world > 1:
+                    dist.all_reduce(grad_arena, op=dist.ReduceOp.AVG)
+                model.clip_adamw_step(**hp_at(steps_total + i), norm=True)
             b.record(st)
             torch.cuda.synchronize()
             if i > 0:
@@ -373,9 +396,33 @@ def main():
             t = torch.tensor([e_ms], device="cuda")
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = t.item()
-        e2e = {"value": B * T * world / (e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": 2 * B * T * 4, "d2h_bytes_per_step": 8,
-               "ms_per_step": e_ms, "api": "gpt2_train_step (host int32 tokens, loss + norm read back)"}
+        e2e = {"value": acc * B * T * world / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": acc * 2 * B * T * 4, "d2h_bytes_per_step": 8,
+               "ms_per_step": e_ms,
+               "api": ("gpt2_train_step" if acc == 1 and world == 1 else
+                       f"{acc} x (gpt2_forward_loss + gpt2_backward) + gpt2_clip_adamw_step")
+                      + " (host int32 tokens, loss + norm read back)"}
+
+    # evaluation pass (no activations kept, one loss read per batch), separate stream
+    evaluation = None
+    if w.get("eval_batches"):
+        nb = w["eval_batches"]
+        ev_np = synth.token_stream(4, nb * B * T + 1)
+        ev = torch.from_numpy(ev_np.view(np.int16)).cuda()
+        losses = []
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for k in range(nb):
+            x, y = model.batch_from_stream(ev, k * B * T, B, T)
+            losses.append(model.eval_loss(x, y))
+        b.record(st)
+        torch.cuda.synchronize()
+        ev_ms = a.elapsed_time(b)
+        evaluation = {"batches": nb, "tokens": nb * B * T, "ms": ev_ms,
+                      "tokens_per_s": nb * B * T / (ev_ms / 1e3),
+                      "mean_loss": sum(losses) / nb,
+                      "data": "Zipf(1.1)/EOT stream seed 4, consecutive windows"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -387,10 +434,11 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (Zipf(1.1)/EOT token stream seed 3, N(0,0.02) weights seed 0)",
-            "config": {"workload": args.workload, "global_batch": B * world, "seq_len": T,
-                       "micro_batch_per_gpu": B, "parallelism": f"dp{world}",
-                       "l2": "working set (activations ~5 GB, weights+state 2.2 GB) >> 126 MB L2; no flush"},
-            "mfu": {"algorithmic_flops_per_step": fpt * B * T * world,
+            "config": {"workload": args.workload, "global_batch": acc * B * world, "seq_len": T,
+                       "micro_batch_per_gpu": B, "accumulation": acc, "parallelism": f"dp{world}",
+                       "l2": "working set (saved activations and weights + optimizer state, GBs) "
+                             ">> 126 MB L2; no flush"},
+            "mfu": {"algorithmic_flops_per_step": fpt * acc * B * T * world,
                     "achieved_tflops": achieved_tflops,
                     "vs_datasheet_2250": achieved_tflops / DATASHEET_BF16_TFLOPS,
                     "vs_measured_burst": achieved_tflops / peaks["bf16_tflops"],
@@ -404,6 +452,8 @@ def main():
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
+        if evaluation is not None:
+            line["eval"] = evaluation
         print(json.dumps(line), flush=True)
     model.close()
     if world > 1:

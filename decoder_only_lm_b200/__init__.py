@@ -420,6 +420,24 @@ def matmul(A, B, a_kmajor=True, b_kmajor=True, M=None, N=None, K=None, alpha=1.0
     return out
 
 
+def cosine_lr(t, max_lr, min_lr, warmup_steps, total_steps):
+    """Learning rate for schedule step t, counted from 0 [CS336 §2, learning-rate
+    schedule: linear warmup from 0 to max_lr over warmup_steps, then half a
+    cosine period down to min_lr at total_steps, min_lr from there on; LECTURE:
+    max 6e-4 with a minimum of 10% of it].  Host-side: the value is passed to
+    clip_adamw_step as lr.  The optimizer's own step count (bias correction)
+    starts at 1 and is kept by the library."""
+    import math
+    if warmup_steps < 0 or warmup_steps >= total_steps:
+        raise ValueError("cosine_lr needs 0 <= warmup_steps < total_steps")
+    if t >= total_steps:
+        return min_lr
+    if t < warmup_steps:
+        return max_lr * (t / warmup_steps)
+    phase = math.pi * (t - warmup_steps) / (total_steps - warmup_steps)
+    return min_lr + (max_lr - min_lr) * (1.0 + math.cos(phase)) / 2.0
+
+
 def device_error():
     c = C.c_int()
     _check(lib.gpt2_device_error(C.byref(c)))
