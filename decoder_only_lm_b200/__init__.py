@@ -60,6 +60,9 @@ SIGNATURES = {
     "gpt2_train_step": (_i, [_P, _P, _P, _i, _i, _i, _f, _f, _f, _f, _f, _f, C.POINTER(_f),
                              C.POINTER(_f)]),
     "gpt2_eval_loss": (_i, [_P, _P, _P, _i, _i, _i, C.POINTER(_f)]),
+    "gpt2_stream_begin": (_i, [_P, _P, _i64, _i64, _i64, _i, _i, _i, _f, _f, _f, _f, _f]),
+    "gpt2_stream_steps": (_i, [_P, _i, C.POINTER(_f)]),
+    "gpt2_stream_end": (_i, [_P, C.POINTER(_i64)]),
     "gpt2_synchronize": (_i, [_P]),
     "gpt2_arena": (_i, [_P, _i, C.POINTER(C.POINTER(_f)), C.POINTER(_i64)]),
     "gpt2_profile_enable": (_i, [_P, _i]),
@@ -260,6 +263,28 @@ class GPT2:
                                    weight_decay, max_norm, C.byref(loss) if read else None,
                                    C.byref(norm) if read else None), self.h)
         return (loss.value, norm.value) if read else None
+
+    def stream_begin(self, stream_u16, start, stride, B, T, accum=1, beta1=0.9, beta2=0.95,
+                     eps=1e-8, weight_decay=0.1, max_norm=1.0):
+        """gpt2_stream_begin: record one optimizer step over windows of a device
+        token stream (kept referenced until stream_end) as a CUDA graph."""
+        self._stream_ref = stream_u16
+        _check(lib.gpt2_stream_begin(self.h, _ptr(stream_u16), stream_u16.numel(), start, stride,
+                                     B, T, accum, beta1, beta2, eps, weight_decay, max_norm),
+               self.h)
+
+    def stream_steps(self, lrs):
+        """gpt2_stream_steps: one replayed optimizer step per learning rate in lrs."""
+        arr = (C.c_float * len(lrs))(*[float(v) for v in lrs])
+        _check(lib.gpt2_stream_steps(self.h, len(lrs), arr), self.h)
+
+    def stream_end(self):
+        """gpt2_stream_end: returns the cursor (offset of the next window)."""
+        cur = C.c_int64()
+        rc = lib.gpt2_stream_end(self.h, C.byref(cur))
+        self._stream_ref = None
+        _check(rc, self.h)
+        return cur.value
 
     def eval_loss(self, x, y):
         x, y, B, T, dev = self._xy(x, y)

@@ -19,7 +19,8 @@ struct DevStatus {
   int timeout;      // a bounded wait gave up
   int timeout_where;
   int step;         // AdamW step counter t (device copy, authoritative)
-  int pad[3];
+  int window_bad;   // a batch window read at a device cursor ran past its stream
+  int pad[2];
 };
 
 #define GPT2_CUDA_TRY(expr)                                                        \

@@ -98,6 +98,11 @@ struct gpt2_handle {
   void* ws_emb = nullptr;
   double* ws_norm = nullptr;
   DevStatus* status = nullptr;
+  // training from a device token stream, one optimizer step recorded as a CUDA graph
+  int64_t* d_cursor = nullptr;  // offset of the next window in the stream
+  float* d_lr = nullptr;        // learning rate read by the optimizer kernel of the graph
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t graph_exec = nullptr;
   // state
   bool fwd_saved = false;
   int fB = 0, fT = 0;
@@ -314,6 +319,14 @@ int check_status(gpt2_handle* h) {
     c.timeout = 0;
     cudaMemcpy(h->status, &c, sizeof(c), cudaMemcpyHostToDevice);
     return fail(h, GPT2_ERR_TIMEOUT, "a bounded device wait gave up (kernel timeout)");
+  }
+  if (s.window_bad) {
+    DevStatus c = s;
+    c.window_bad = 0;
+    H_CUDA(h, cudaMemcpy(h->status, &c, sizeof(c), cudaMemcpyHostToDevice));
+    h->fwd_saved = false;
+    return fail(h, GPT2_ERR_ARG, "a batch window at the stream cursor ran past the stream "
+                                 "(that step's update was skipped)");
   }
   if (s.token_bad) {
     DevStatus c = s;
@@ -674,6 +687,8 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
   h->ws_emb = A(embed_bwd_workspace(M, int(C)));
   h->ws_norm = static_cast<double*>(A(gradnorm_workspace()));
   h->status = static_cast<DevStatus*>(A(sizeof(DevStatus)));
+  h->d_cursor = static_cast<int64_t*>(A(sizeof(int64_t)));
+  h->d_lr = static_cast<float*>(A(sizeof(float)));
   if (!ok) {
     free_all(h);
     delete h;
@@ -698,6 +713,8 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
 int gpt2_destroy(gpt2_handle* h) {
   if (!h) return GPT2_OK;
   cudaStreamSynchronize(h->st);
+  if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+  if (h->graph) cudaGraphDestroy(h->graph);
   prof_collect(h);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   free_all(h);
@@ -853,7 +870,8 @@ int gpt2_clip_adamw_step(gpt2_handle* h, float lr, float beta1, float beta2, flo
     PROF(GPT2_PROF_OPTIM, 14.0 * h->n_arena, (34.0 + (h->use_bf16 ? 2.0 : 0.0)) * h->n_arena);
     H_TRY(h, launch_gradnorm(h->G, h->n_arena, h->ws_norm, h->d_norm, h->st));
     H_TRY(h, launch_clip_adamw(h->P, h->G, h->Mo, h->Vo, h->Pb, h->n_arena, h->n_decay, h->d_norm,
-                               h->status, lr, beta1, beta2, eps, weight_decay, max_norm, h->st));
+                               h->status, lr, nullptr, beta1, beta2, eps, weight_decay, max_norm,
+                               h->st));
   }
   h->mirror_dirty = false;  // the pass rewrote the bf16 mirror
   if (grad_norm_out) {
@@ -892,6 +910,116 @@ int gpt2_eval_loss(gpt2_handle* h, const int32_t* x, const int32_t* y, int B, in
   else
     H_TRY(h, forward_t<float>(h, B, T, nullptr, false));
   return read_loss(h, loss_out);
+}
+
+// ---------------------------------------------------------------- stream training (graph)
+// One optimizer step on consecutive windows of a device token stream, recorded
+// once as a CUDA graph and replayed: zero the gradients; accum times: cut the
+// window at the device cursor (x = s[o .. o+BT), y = s[o+1 .. o+BT+1]),
+// advance the cursor by `stride`, forward and backward with grad_scale 1/accum;
+// then the gradient norm, clip and AdamW with the learning rate read from the
+// device.  Every launch is stream-ordered with no host synchronisation, which
+// is what lets the step be captured; replaying it costs one graph launch
+// instead of some 400 kernel launches.
+namespace {
+int stream_step_body(gpt2_handle* h, const uint16_t* tok, int64_t len, int64_t stride, int B,
+                     int T, int accum, float beta1, float beta2, float eps, float wd,
+                     float max_norm) {
+  const int64_t n = int64_t(B) * T;
+  h->grads_zero = true;
+  for (int a = 0; a < accum; ++a) {
+    H_TRY(h, launch_slice_batch_cursor(tok, len, h->d_cursor, n, h->xbuf, h->ybuf, h->status,
+                                       h->st));
+    H_TRY(h, launch_advance_cursor(h->d_cursor, stride, h->st));
+    if (h->use_bf16)
+      H_TRY(h, forward_t<bf16>(h, B, T, nullptr, true));
+    else
+      H_TRY(h, forward_t<float>(h, B, T, nullptr, true));
+    if (h->use_bf16)
+      H_TRY(h, backward_t<bf16>(h, 1.f / float(accum)));
+    else
+      H_TRY(h, backward_t<float>(h, 1.f / float(accum)));
+  }
+  H_TRY(h, launch_gradnorm(h->G, h->n_arena, h->ws_norm, h->d_norm, h->st));
+  H_TRY(h, launch_clip_adamw(h->P, h->G, h->Mo, h->Vo, h->Pb, h->n_arena, h->n_decay, h->d_norm,
+                             h->status, 0.f, h->d_lr, beta1, beta2, eps, wd, max_norm, h->st));
+  h->mirror_dirty = false;
+  return GPT2_OK;
+}
+}  // namespace
+
+int gpt2_stream_begin(gpt2_handle* h, const uint16_t* d_stream, int64_t stream_len, int64_t start,
+                      int64_t stride, int B, int T, int accum, float beta1, float beta2, float eps,
+                      float weight_decay, float max_norm) {
+  if (!h || !d_stream) return fail(h, GPT2_ERR_ARG, "NULL argument");
+  H_TRY(h, validate_bt(h, B, T));
+  if (accum < 1 || start < 0 || stride < 0 || stream_len < int64_t(B) * T + 1)
+    return fail(h, GPT2_ERR_ARG, "stream_begin: bad accum, start, stride or stream length");
+  if (!(beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f && eps >= 0.f && max_norm > 0.f))
+    return fail(h, GPT2_ERR_ARG, "bad optimiser hyper-parameters");
+  if (h->prof_on) return fail(h, GPT2_ERR_STATE, "stream_begin: disable profiling first");
+  if (h->graph_exec) {
+    cudaGraphExecDestroy(h->graph_exec);
+    h->graph_exec = nullptr;
+  }
+  if (h->graph) {
+    cudaGraphDestroy(h->graph);
+    h->graph = nullptr;
+  }
+  // the bf16 mirror is brought up to date now, not inside every replay
+  if (h->use_bf16 && h->mirror_dirty) H_TRY(h, launch_to_bf16(h->P, h->Pb, h->n_arena, h->st));
+  h->mirror_dirty = false;
+  H_CUDA(h, cudaMemcpyAsync(h->d_cursor, &start, sizeof(int64_t), cudaMemcpyHostToDevice, h->st));
+  H_CUDA(h, cudaStreamSynchronize(h->st));
+  // Record on a private stream (the handle's stream may be the legacy default
+  // stream, which cannot be captured); everything issued before is complete.
+  cudaStream_t user = h->st, cs = nullptr;
+  H_CUDA(h, cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
+  h->st = cs;
+  int rc = GPT2_OK;
+  cudaGraph_t g = nullptr;
+  cudaError_t ec = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+  if (ec == cudaSuccess) {
+    rc = stream_step_body(h, d_stream, stream_len, stride, B, T, accum, beta1, beta2, eps,
+                          weight_decay, max_norm);
+    ec = cudaStreamEndCapture(cs, &g);
+  }
+  h->st = user;
+  cudaStreamDestroy(cs);
+  if (rc != GPT2_OK) {
+    if (g) cudaGraphDestroy(g);
+    return rc;
+  }
+  if (ec != cudaSuccess)
+    return fail(h, GPT2_ERR_CUDA, std::string("stream_begin: capture failed: ") +
+                                      cudaGetErrorString(ec));
+  h->graph = g;
+  H_CUDA(h, cudaGraphInstantiate(&h->graph_exec, h->graph, 0));
+  return GPT2_OK;
+}
+
+int gpt2_stream_steps(gpt2_handle* h, int n_steps, const float* lr) {
+  if (!h || (n_steps > 0 && !lr)) return fail(h, GPT2_ERR_ARG, "NULL argument");
+  if (!h->graph_exec) return fail(h, GPT2_ERR_STATE, "stream_steps needs stream_begin");
+  for (int i = 0; i < n_steps; ++i) {
+    H_CUDA(h, cudaMemcpyAsync(h->d_lr, lr + i, sizeof(float), cudaMemcpyHostToDevice, h->st));
+    H_CUDA(h, cudaGraphLaunch(h->graph_exec, h->st));
+    h->launches_total += 1;
+  }
+  return GPT2_OK;
+}
+
+int gpt2_stream_end(gpt2_handle* h, int64_t* cursor_out) {
+  if (!h) return GPT2_ERR_ARG;
+  if (cursor_out)
+    H_CUDA(h, cudaMemcpyAsync(cursor_out, h->d_cursor, sizeof(int64_t), cudaMemcpyDeviceToHost,
+                              h->st));
+  H_CUDA(h, cudaStreamSynchronize(h->st));
+  if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+  if (h->graph) cudaGraphDestroy(h->graph);
+  h->graph_exec = nullptr;
+  h->graph = nullptr;
+  return check_status(h);
 }
 
 int gpt2_arena(gpt2_handle* h, int which, float** ptr, int64_t* n_elems) {

@@ -22,6 +22,28 @@ namespace {
 constexpr int kThreads = 256;
 
 // ------------------------------------------------------------ batch slicing
+// The window at the device cursor *cur; a window that would run past the
+// stream (len tokens) is not read: its ids become 0 and window_bad is set,
+// which skips the optimizer update and is reported by the next status read.
+__global__ void slice_batch_cursor_kernel(const uint16_t* __restrict__ s, int64_t len,
+                                          const int64_t* __restrict__ cur, int64_t n,
+                                          int32_t* __restrict__ x, int32_t* __restrict__ y,
+                                          DevStatus* status) {
+  const int64_t off = *cur;
+  const bool ok = off >= 0 && off + n + 1 <= len;
+  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= n) return;
+  if (!ok) {
+    if (i == 0) atomicExch(&status->window_bad, 1);
+    x[i] = 0;
+    y[i] = 0;
+    return;
+  }
+  x[i] = int32_t(s[off + i]);
+  y[i] = int32_t(s[off + i + 1]);
+}
+__global__ void advance_cursor_kernel(int64_t* cur, int64_t stride) { *cur += stride; }
+
 __global__ void slice_batch_kernel(const uint16_t* __restrict__ s, int64_t off, int64_t n,
                                    int32_t* __restrict__ x, int32_t* __restrict__ y) {
   int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
@@ -620,10 +642,11 @@ __global__ void clip_adamw_kernel(float* __restrict__ p, const float* __restrict
                                   float* __restrict__ m, float* __restrict__ v,
                                   bf16* __restrict__ pb, int64_t n, int64_t n_decay,
                                   const float* __restrict__ norm, const DevStatus* __restrict__ st,
-                                  float lr, float b1, float b2, float eps, float wd,
-                                  float max_norm) {
+                                  float lr_arg, const float* __restrict__ lr_dev, float b1,
+                                  float b2, float eps, float wd, float max_norm) {
   const float nrm = *norm;
-  if (st->token_bad || !isfinite(nrm)) return;
+  const float lr = lr_dev ? *lr_dev : lr_arg;  // lr_dev: set on the device between graph replays
+  if (st->token_bad || st->window_bad || !isfinite(nrm)) return;
   const int t = st->step + 1;
   const float s = fminf(1.f, max_norm / (nrm + 1e-6f));
   const float alpha = lr * sqrtf(1.f - powf(b2, float(t))) / (1.f - powf(b1, float(t)));
@@ -661,7 +684,7 @@ __global__ void clip_adamw_kernel(float* __restrict__ p, const float* __restrict
 }
 
 __global__ void step_advance_kernel(const float* __restrict__ norm, DevStatus* st) {
-  if (st->token_bad) return;
+  if (st->token_bad || st->window_bad) return;
   if (!isfinite(*norm)) {
     st->nonfinite = 1;
     return;
@@ -696,6 +719,23 @@ int64_t next_pow2(int64_t n) {
 }  // namespace
 
 // ============================================================ launchers
+
+int launch_slice_batch_cursor(const uint16_t* s, int64_t len, const int64_t* cur, int64_t n,
+                              int32_t* x, int32_t* y, DevStatus* status, cudaStream_t st) {
+  if (n <= 0) return GPT2_OK;
+  slice_batch_cursor_kernel<<<int(cdiv64(n, kThreads)), kThreads, 0, st>>>(s, len, cur, n, x, y,
+                                                                          status);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int launch_advance_cursor(int64_t* cur, int64_t stride, cudaStream_t st) {
+  advance_cursor_kernel<<<1, 1, 0, st>>>(cur, stride);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
+}
 
 int launch_slice_batch(const uint16_t* s, int64_t off, int64_t n, int32_t* x, int32_t* y,
                        cudaStream_t st) {
@@ -925,14 +965,15 @@ int launch_gradnorm(const float* g, int64_t n, double* ws, float* norm, cudaStre
 }
 
 int launch_clip_adamw(float* p, const float* g, float* m, float* v, bf16* pb, int64_t n,
-                      int64_t n_decay, const float* norm, DevStatus* status, float lr, float b1,
-                      float b2, float eps, float wd, float max_norm, cudaStream_t st) {
+                      int64_t n_decay, const float* norm, DevStatus* status, float lr,
+                      const float* lr_dev, float b1, float b2, float eps, float wd, float max_norm,
+                      cudaStream_t st) {
   if ((n & 3) || (n_decay & 3)) {
     gpt2_internal::set_error("clip_adamw: arena sizes must be multiples of 4");
     return GPT2_ERR_ARG;
   }
   clip_adamw_kernel<<<grid_for(n / 4, kThreads), kThreads, 0, st>>>(
-      p, g, m, v, pb, n, n_decay, norm, status, lr, b1, b2, eps, wd, max_norm);
+      p, g, m, v, pb, n, n_decay, norm, status, lr, lr_dev, b1, b2, eps, wd, max_norm);
   COUNT_LAUNCH(1);
   step_advance_kernel<<<1, 1, 0, st>>>(norm, status);
   COUNT_LAUNCH(1);

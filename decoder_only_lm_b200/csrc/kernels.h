@@ -54,6 +54,10 @@ int gemm_launch(const GemmArgs& g, cudaStream_t st);
 // ---------------------------------------------------------------- elementwise / rows
 int launch_slice_batch(const uint16_t* s, int64_t off, int64_t n, int32_t* x, int32_t* y,
                        cudaStream_t st);
+// x, y from the window at the device cursor *cur of a len-token stream (window_bad if outside)
+int launch_slice_batch_cursor(const uint16_t* s, int64_t len, const int64_t* cur, int64_t n,
+                              int32_t* x, int32_t* y, DevStatus* status, cudaStream_t st);
+int launch_advance_cursor(int64_t* cur, int64_t stride, cudaStream_t st);
 int launch_embed_fwd(const int32_t* x, const int32_t* y, const float* wte, const float* wpe,
                      int B, int T, int C, int V, float* out, DevStatus* status, cudaStream_t st);
 // dwte[x_m] += dh[m] (deterministic: sort by id, segmented sums); dwpe[t] (+)= sum_b dh[b,t].
@@ -78,9 +82,11 @@ int launch_colsum(const InT* in, int64_t M, int N, float* out, int accumulate, f
 // gradient norm (deterministic two-stage, double accumulation) into *norm (device)
 size_t gradnorm_workspace();
 int launch_gradnorm(const float* g, int64_t n, double* ws, float* norm, cudaStream_t st);
+// lr_dev (nullable): learning rate read on the device instead of lr
 int launch_clip_adamw(float* p, const float* g, float* m, float* v, bf16* pb, int64_t n,
-                      int64_t n_decay, const float* norm, DevStatus* status, float lr, float b1,
-                      float b2, float eps, float wd, float max_norm, cudaStream_t st);
+                      int64_t n_decay, const float* norm, DevStatus* status, float lr,
+                      const float* lr_dev, float b1, float b2, float eps, float wd, float max_norm,
+                      cudaStream_t st);
 int launch_to_bf16(const float* src, bf16* dst, int64_t n, cudaStream_t st);
 int launch_fill(float* p, float v, int64_t n, cudaStream_t st);
 // cross-entropy over a chunk of logits rows z [rows, Vp] (fp32)

@@ -193,6 +193,39 @@ int gpt2_train_step(gpt2_handle* h, const int32_t* x, const int32_t* y, int B, i
                     int tokens_on_device, float lr, float beta1, float beta2, float eps,
                     float weight_decay, float max_norm, float* loss_out, float* grad_norm_out);
 
+/* Training on consecutive windows of a device-resident token stream, each
+ * optimizer step replayed from a CUDA graph recorded once (no counterpart on
+ * the pages, which launch every operation from Python; the step itself is
+ * theirs: windows x = s[o .. o+BT), y = s[o+1 .. o+BT+1) [CH28 §28.3],
+ * gradient accumulation over `accum` micro-batches with the loss scaled by
+ * 1/accum [LECTURE], then norm, clip and AdamW [CS336 §2]).
+ *
+ * gpt2_stream_begin records one optimizer step: zero the gradients; accum
+ * times { cut the B x T window at the device cursor, advance the cursor by
+ * `stride` tokens, forward, backward with grad_scale 1/accum }; gradient
+ * norm, clip to max_norm, AdamW (lr read on the device at replay).
+ * d_stream: device uint16 ids [stream_len], must stay valid and unchanged in
+ * size until gpt2_stream_end.  The cursor starts at `start` (for data
+ * parallel rank r of R: start = r*B*T, stride = R*B*T).  A window that would
+ * run past the stream is not read: the step's update is skipped and the next
+ * status read (gpt2_stream_end, a loss or norm read) returns GPT2_ERR_ARG.
+ * Profiling must be off.  Synchronises; nothing of the step runs yet.
+ *
+ * gpt2_stream_steps replays n_steps optimizer steps; lr: host [n_steps], the
+ * learning rate of each (a schedule is computed by the caller).
+ * Asynchronous on the handle's stream.
+ *
+ * gpt2_stream_end synchronises, writes the cursor (next window offset) to
+ * *cursor_out (host, nullable), releases the graph and returns the device
+ * status (GPT2_ERR_ARG for a window past the stream, GPT2_ERR_TOKEN,
+ * GPT2_ERR_NONFINITE as in gpt2_clip_adamw_step).  The eager calls remain
+ * usable before, between and after. */
+int gpt2_stream_begin(gpt2_handle* h, const uint16_t* d_stream, int64_t stream_len, int64_t start,
+                      int64_t stride, int B, int T, int accum, float beta1, float beta2, float eps,
+                      float weight_decay, float max_norm);
+int gpt2_stream_steps(gpt2_handle* h, int n_steps, const float* lr);
+int gpt2_stream_end(gpt2_handle* h, int64_t* cursor_out);
+
 /* Forward-only mean loss (no activations saved; the saved state of a
  * previous forward is invalidated) [CH28 §28.4: validation loss].  loss_out
  * (host) is required; the call synchronises. */
