@@ -95,6 +95,11 @@ struct gpt2_handle {
   size_t lm_ws_bytes = 0;
   float* ws = nullptr;
   size_t ws_bytes = 0;
+  // side stream: weight-gradient GEMMs overlap the input-gradient GEMMs they
+  // are independent of (own workspace; joined back before anything else runs)
+  cudaStream_t st2 = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  float* ws2 = nullptr;
   void* ws_emb = nullptr;
   double* ws_norm = nullptr;
   DevStatus* status = nullptr;
@@ -289,12 +294,37 @@ void* aoff(void* base, int64_t elems, size_t esz) {
 }
 
 int gemm(gpt2_handle* h, const void* A, int ak, int64_t lda, const void* B, int bk, int64_t ldb,
-         int M, int N, int K, const EpiParams& ep) {
-  GemmArgs g{A, ak, lda, B, bk, ldb, h->use_bf16, M, N, K, ep, h->ws, h->ws_bytes};
+         int M, int N, int K, const EpiParams& ep, cudaStream_t st = nullptr,
+         float* ws = nullptr) {
+  GemmArgs g{A, ak, lda, B, bk, ldb, h->use_bf16, M, N, K, ep, ws ? ws : h->ws, h->ws_bytes};
   g.ep.out_bf16 = (ep.kind == EPI_ACC || ep.kind == EPI_RESID) ? 0 : ep.out_bf16;
-  H_TRY(h, gemm_launch(g, h->st));
+  H_TRY(h, gemm_launch(g, st ? st : h->st));
   return GPT2_OK;
 }
+
+// Fork / join of the side stream (recorded as parallel branches when the step
+// is captured).  While the profiler is on, side work runs on the main stream
+// so that every kernel group is timed on its own.
+struct Side {
+  gpt2_handle* h;
+  bool on;
+  cudaStream_t st() const { return on ? h->st2 : h->st; }
+  float* ws() const { return on ? h->ws2 : h->ws; }
+  int fork() {
+    if (on) {
+      H_CUDA(h, cudaEventRecord(h->ev_fork, h->st));
+      H_CUDA(h, cudaStreamWaitEvent(h->st2, h->ev_fork, 0));
+    }
+    return GPT2_OK;
+  }
+  int join() {
+    if (on) {
+      H_CUDA(h, cudaEventRecord(h->ev_join, h->st2));
+      H_CUDA(h, cudaStreamWaitEvent(h->st, h->ev_join, 0));
+    }
+    return GPT2_OK;
+  }
+};
 
 EpiParams epi(int kind, void* out, int64_t ldo, int out_bf16) {
   EpiParams e;
@@ -479,8 +509,16 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     // (algorithmic work: the dH and dW contractions; the logits are recomputed)
     PROF(GPT2_PROF_LMHEAD, 2 * gemm_flops(M, Vp, C),
          a * (2.0 * M * C + double(Vp) * C) + 8.0 * double(Vp) * C);
+    LmSide side;  // dW beside dH (not while profiling, so each group is timed alone)
+    if (!h->prof_on) {
+      side.st = h->st2;
+      side.e_fork = h->ev_fork;
+      side.e_join = h->ev_join;
+      side.ws = h->ws2;
+      side.ws_bytes = h->ws_bytes;
+    }
     H_TRY(h, lmhead_bwd(hf, wptr(h, h->off_wte), h->ybuf, h->hlse, int(M), C, Vp, h->use_bf16,
-                        scale, dhf, G + h->off_wte, acc, h->lm_ws, h->lm_ws_bytes, h->st));
+                        scale, dhf, G + h->off_wte, acc, h->lm_ws, h->lm_ws_bytes, h->st, &side));
   }
   A* copy = ab ? dres_a : nullptr;
   const double lnb_bytes = M * C * (4.0 + 8.0 + 2.0 * a) + 8.0 * M;
@@ -497,30 +535,40 @@ int backward_t(gpt2_handle* h, float grad_scale) {
   A* datt = static_cast<A*>(h->datt);
   A* dqkv = static_cast<A*>(h->dqkv);
   const double attn_bwd_flops = 4.0 * B * Hh * double(T) * T * (C / Hh);
+  // Each weight-gradient GEMM (and the bias column sum beside it) is
+  // independent of the input-gradient GEMM of the same layer: they run on the
+  // side stream, launched after it, so that they fill its last partial wave;
+  // joined back before the LayerNorm backward overwrites the bf16 dres copy.
+  Side sd{h, !h->prof_on};
   for (int l = h->L - 1; l >= 0; --l) {
     const LayerOff& o = h->lo[l];
     {
       // mlp.proj: h'' = h' + g Wfp^T + b;  du = (dres Wfp) * gelu'(u)
       PROF(GPT2_PROF_GEMM, 2 * gemm_flops(M, F, C), a * (2.0 * M * C + 3.0 * M * F + F * C) + 8.0 * F * C);
+      H_TRY(h, sd.fork());
       EpiParams e = epi(EPI_GELU_BWD, du, F, ab);
       e.aux = h->u[l];
       H_TRY(h, gemm(h, dres_a, 1, C, wptr(h, o.fpw), 0, F, int(M), F, C, e));
       e = epi(EPI_ACC, G + o.fpw, F, 0);
       e.accumulate = acc;
-      H_TRY(h, gemm(h, dres_a, 0, C, h->g[l], 0, F, C, F, int(M), e));
+      H_TRY(h, gemm(h, dres_a, 0, C, h->g[l], 0, F, C, F, int(M), e, sd.st(), sd.ws()));
+      // no join yet: the side stream runs in order, and the join before the
+      // LayerNorm backward (which rewrites dres_a) also covers this GEMM
     }
     {
       // mlp.fc: u = ln2 Wfc^T + b
       PROF(GPT2_PROF_GEMM, 2 * gemm_flops(M, C, F), a * (2.0 * M * F + 2.0 * M * C + F * C) + 8.0 * F * C);
+      H_TRY(h, sd.fork());
       EpiParams e = epi(EPI_STORE, dln, C, ab);
       H_TRY(h, gemm(h, du, 1, F, wptr(h, o.fcw), 0, C, int(M), C, F, e));
       e = epi(EPI_ACC, G + o.fcw, C, 0);
       e.accumulate = acc;
-      H_TRY(h, gemm(h, du, 0, F, h->ln2[l], 0, C, F, C, int(M), e));
+      H_TRY(h, gemm(h, du, 0, F, h->ln2[l], 0, C, F, C, int(M), e, sd.st(), sd.ws()));
     }
     {
       PROF(GPT2_PROF_OTHER, 0, a * M * F);
-      H_TRY(h, launch_colsum<A>(du, M, F, G + o.fcb, acc, h->ws, h->st));
+      H_TRY(h, launch_colsum<A>(du, M, F, G + o.fcb, acc, sd.ws(), sd.st()));
+      H_TRY(h, sd.join());
     }
     {
       PROF(GPT2_PROF_LN_BWD, 0, lnb_bytes);
@@ -532,30 +580,34 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     {
       // attn.proj: h' = h + att Wp^T + b
       PROF(GPT2_PROF_GEMM, 2 * gemm_flops(M, C, C), a * (4.0 * M * C + C * C) + 8.0 * C * C);
+      H_TRY(h, sd.fork());
       EpiParams e = epi(EPI_STORE, datt, C, ab);
       H_TRY(h, gemm(h, dres_a, 1, C, wptr(h, o.projw), 0, C, int(M), C, C, e));
       e = epi(EPI_ACC, G + o.projw, C, 0);
       e.accumulate = acc;
-      H_TRY(h, gemm(h, dres_a, 0, C, h->att[l], 0, C, C, C, int(M), e));
+      H_TRY(h, gemm(h, dres_a, 0, C, h->att[l], 0, C, C, C, int(M), e, sd.st(), sd.ws()));
     }
     {
       PROF(GPT2_PROF_ATTN_BWD, attn_bwd_flops, a * 9.0 * M * C + 8.0 * M * Hh);
       H_TRY(h, launch_attn_bwd<A>(datt, static_cast<A*>(h->qkv[l]), static_cast<A*>(h->att[l]),
                                   h->alse[l], B, T, C, Hh, dqkv, h->ws, h->st));
+      H_TRY(h, sd.join());  // attn.proj's weight gradient ran beside the attention backward
     }
     {
       // attn.qkv: qkv = ln1 Wqkv^T + b
       PROF(GPT2_PROF_GEMM, 2 * gemm_flops(M, C, 3 * C),
            a * (6.0 * M * C + 2.0 * M * C + 3.0 * C * C) + 12.0 * C * C);
+      H_TRY(h, sd.fork());
       EpiParams e = epi(EPI_STORE, dln, C, ab);
       H_TRY(h, gemm(h, dqkv, 1, 3 * C, wptr(h, o.qkvw), 0, C, int(M), C, 3 * C, e));
       e = epi(EPI_ACC, G + o.qkvw, C, 0);
       e.accumulate = acc;
-      H_TRY(h, gemm(h, dqkv, 0, 3 * C, h->ln1[l], 0, C, 3 * C, C, int(M), e));
+      H_TRY(h, gemm(h, dqkv, 0, 3 * C, h->ln1[l], 0, C, 3 * C, C, int(M), e, sd.st(), sd.ws()));
     }
     {
       PROF(GPT2_PROF_OTHER, 0, a * 3.0 * M * C);
-      H_TRY(h, launch_colsum<A>(dqkv, M, 3 * C, G + o.qkvb, acc, h->ws, h->st));
+      H_TRY(h, launch_colsum<A>(dqkv, M, 3 * C, G + o.qkvb, acc, sd.ws(), sd.st()));
+      H_TRY(h, sd.join());
     }
     {
       PROF(GPT2_PROF_LN_BWD, 0, lnb_bytes);
@@ -684,6 +736,7 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
   for (auto& s : shapes) ws = std::max(ws, gemm_workspace_bytes(s[0], s[1], s[2]));
   h->ws_bytes = ws;
   h->ws = static_cast<float*>(A(ws));
+  h->ws2 = static_cast<float*>(A(ws));
   h->ws_emb = A(embed_bwd_workspace(M, int(C)));
   h->ws_norm = static_cast<double*>(A(gradnorm_workspace()));
   h->status = static_cast<DevStatus*>(A(sizeof(DevStatus)));
@@ -693,6 +746,15 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
     free_all(h);
     delete h;
     return fail(nullptr, GPT2_ERR_OOM, "device allocation failed");
+  }
+  if (cudaStreamCreateWithFlags(&h->st2, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->st2) cudaStreamDestroy(h->st2);
+    free_all(h);
+    delete h;
+    return fail(nullptr, GPT2_ERR_CUDA, "creating the side stream failed");
   }
   cudaStream_t st = h->st;
   bool cz = cudaMemsetAsync(h->P, 0, arena, st) == cudaSuccess &&
@@ -715,6 +777,12 @@ int gpt2_destroy(gpt2_handle* h) {
   cudaStreamSynchronize(h->st);
   if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
   if (h->graph) cudaGraphDestroy(h->graph);
+  if (h->st2) {
+    cudaStreamSynchronize(h->st2);
+    cudaStreamDestroy(h->st2);
+  }
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
   prof_collect(h);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   free_all(h);

@@ -127,7 +127,7 @@ int lmhead_fwd(const void* h, const void* W, const int32_t* y, int M, int C, int
 
 int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse, int M, int C,
                int Vp, int bf16, float scale, void* dh, float* dW, int dw_accumulate, void* ws,
-               size_t ws_bytes, cudaStream_t st) {
+               size_t ws_bytes, cudaStream_t st, const LmSide* side) {
   const Layout L = layout(M, C, Vp, bf16);
   if (!ws || ws_bytes < L.total) {
     gpt2_internal::set_error("lmhead: workspace too small");
@@ -166,6 +166,11 @@ int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse,
                                        st);
     }
     if (rc) return rc;
+    const bool par = side && side->st && dh && dW;
+    if (par) {  // dz of this chunk complete: dW may start beside dH
+      GPT2_CUDA_TRY(cudaEventRecord(side->e_fork, st));
+      GPT2_CUDA_TRY(cudaStreamWaitEvent(side->st, side->e_fork, 0));
+    }
     if (dh) {
       EpiParams e;
       e.kind = EPI_STORE;
@@ -177,14 +182,20 @@ int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse,
       if (rc) return rc;
     }
     if (dW) {
+      // dH and dW only read dz: with a side stream, dW fills dH's last wave
       EpiParams e;
       e.kind = EPI_ACC;
       e.out = dW;
       e.ldo = C;
       e.accumulate = (dw_accumulate || r0 > 0) ? 1 : 0;
-      GemmArgs g{dz, 0, Vp, hr, 0, C, bf16, Vp, C, mc, e, gws, L.gws};
-      rc = gemm_launch(g, st);
+      GemmArgs g{dz, 0, Vp, hr, 0, C, bf16, Vp, C, mc, e, par ? side->ws : gws,
+                 par ? side->ws_bytes : L.gws};
+      rc = gemm_launch(g, par ? side->st : st);
       if (rc) return rc;
+      if (par) {  // dz is rewritten by the next chunk
+        GPT2_CUDA_TRY(cudaEventRecord(side->e_join, side->st));
+        GPT2_CUDA_TRY(cudaStreamWaitEvent(st, side->e_join, 0));
+      }
     }
   }
   return GPT2_OK;

@@ -114,9 +114,18 @@ int launch_attn_bwd(const T* dout, const T* qkv, const T* out, const float* lse,
 size_t lmhead_workspace(int M, int C, int Vp, int bf16);
 int lmhead_fwd(const void* h, const void* W, const int32_t* y, int M, int C, int Vp, int bf16,
                float* lse, float* row_loss, void* ws, size_t ws_bytes, cudaStream_t st);
+// With side != nullptr the dW GEMM of each chunk runs on that stream (its own
+// split-K workspace side_ws of ws-sized need), forked after the chunk's dz and
+// joined before the next chunk rewrites dz (events e_fork, e_join).
+struct LmSide {
+  cudaStream_t st = nullptr;
+  cudaEvent_t e_fork = nullptr, e_join = nullptr;
+  float* ws = nullptr;
+  size_t ws_bytes = 0;
+};
 int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse, int M, int C,
                int Vp, int bf16, float scale, void* dh, float* dW, int dw_accumulate, void* ws,
-               size_t ws_bytes, cudaStream_t st);
+               size_t ws_bytes, cudaStream_t st, const LmSide* side = nullptr);
 bool gemm_tc_supported(const GemmArgs& g);
 
 // device error word of the op-level calls (bounded waits)
