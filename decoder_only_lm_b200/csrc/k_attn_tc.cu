@@ -89,6 +89,29 @@ __device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1) {
   asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(rd) : "l"(ra));
   asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(rd));
 }
+// One 64-deep contraction as four K = 16 MMAs, the accumulate flag an
+// immediate: the first MMA overwrites D unless acc; descriptors advance by
+// a_k / b_k per slice (+2 K-major, +128 MN-major).  A from shared memory (ss)
+// or from TMEM (ts: 8 columns of packed bf16 per slice).
+__device__ __forceinline__ void mma_ss4(uint32_t d, uint64_t a, uint64_t b, uint32_t id,
+                                        uint64_t a_k, uint64_t b_k, bool acc) {
+  if (acc)
+    umma_i<1>(d, a, b, id);
+  else
+    umma_i<0>(d, a, b, id);
+#pragma unroll
+  for (int k = 1; k < 4; ++k) umma_i<1>(d, a + k * a_k, b + k * b_k, id);
+}
+__device__ __forceinline__ void mma_ts4(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id,
+                                        uint64_t b_k, bool acc) {
+  if (acc)
+    umma_ts_i<1>(d, a_tmem, b, id);
+  else
+    umma_ts_i<0>(d, a_tmem, b, id);
+#pragma unroll
+  for (int k = 1; k < 4; ++k) umma_ts_i<1>(d, a_tmem + 8 * k, b + k * b_k, id);
+}
+
 // maximum of 64 values as four independent chains of three-input maxima
 __device__ __forceinline__ float max64(const float (&x)[64]) {
   float c[4];
@@ -224,11 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tS + (j & 1) * BS, desc_at_k_kmajor(dQ, k),
-                    desc_at_k_kmajor(desc_offset(dK, s * kStrTile), k), id_s,
-                    k > 0);
+        mma_ss4(tS + (j & 1) * BS, dQ, desc_offset(dK, s * kStrTile), id_s, 2, 2, false);
         umma_commit(b_sf(j & 1));
       }
       if (j >= 1) {
@@ -240,11 +259,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         // P_jj sits in the first 32 columns of its score buffer (two bf16 per
         // column); S_{jj+2} reuses that buffer only after this MMA (issue order)
-#pragma unroll
-        for (int k = 0; k < BS / 16; ++k)
-          umma_bf16_ts(tO, tS + (jj & 1) * BS + k * 8,
-                       desc_at_k_mnmajor(desc_offset(dVm, s * kStrTile), k), id_o,
-                       (jj > 0 || k > 0) ? 1u : 0u);
+        mma_ts4(tO, tS + (jj & 1) * BS, desc_offset(dVm, s * kStrTile), id_o, 128, jj > 0);
         umma_commit(b_od(jj & 1));
         umma_commit(b_kve(s));
         last_pv = jj;
@@ -464,10 +479,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < BS / 16; ++k)
-          umma_bf16_ts(tV, tS + k * 8, desc_at_k_mnmajor(desc_offset(dOm, si * kStrTile), k), id_o,
-                       (i > 1 || k > 0) ? 1u : 0u);
+        mma_ts4(tV, tS, desc_offset(dOm, si * kStrTile), id_o, 128, i > 1);
       }
       if (i < n) {  // S^T_i = K Q_i^T
         if (!mbar_wait(b_qf(s), (i / NSK) & 1, p.err, 22)) {
@@ -475,10 +487,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tS, desc_at_k_kmajor(dK, k), desc_at_k_kmajor(desc_offset(dQ, s * kStrTile), k),
-                    id_s, k > 0);
+        mma_ss4(tS, dK, desc_offset(dQ, s * kStrTile), id_s, 2, 2, false);
         umma_commit(b_sf);
       }
       if (i >= 1) {  // dK += dS^T_{i-1} Q_{i-1}
@@ -487,19 +496,13 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < BS / 16; ++k)
-          umma_bf16_ts(tKd, tP + k * 8, desc_at_k_mnmajor(desc_offset(dQm, si * kStrTile), k), id_o,
-                       (i > 1 || k > 0) ? 1u : 0u);
+        mma_ts4(tKd, tP, desc_offset(dQm, si * kStrTile), id_o, 128, i > 1);
         umma_commit(b_mm);
         umma_commit(b_qe(si));
         ++mm;
       }
       if (i < n) {  // dP^T_i = V dO_i^T
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tP, desc_at_k_kmajor(dV, k), desc_at_k_kmajor(desc_offset(dO, s * kStrTile), k),
-                    id_s, k > 0);
+        mma_ss4(tP, dV, desc_offset(dO, s * kStrTile), id_s, 2, 2, false);
         umma_commit(b_dpf);
       }
     }
@@ -708,20 +711,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tS, desc_at_k_kmajor(dQ, k), desc_at_k_kmajor(desc_offset(dK, s * kStrTile), k),
-                    id_s, k > 0);
+        mma_ss4(tS, dQ, desc_offset(dK, s * kStrTile), id_s, 2, 2, false);
         umma_commit(b_sf);
         if (!mbar_wait(b_dpr, (j & 1) ^ 1, p.err, 32)) {  // dP_{j-1} read
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          umma_bf16(tP, desc_at_k_kmajor(dO, k), desc_at_k_kmajor(desc_offset(dV, s * kStrTile), k),
-                    id_s, k > 0);
+        mma_ss4(tP, dO, desc_offset(dV, s * kStrTile), id_s, 2, 2, false);
         umma_commit(b_dpf);
       }
       if (j >= 1) {
@@ -731,10 +728,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < BS / 16; ++k)
-          umma_bf16_ts(tQd, tDs + k * 8, desc_at_k_mnmajor(desc_offset(dKm, sj * kStrTile), k), id_o,
-                       (jj > 0 || k > 0) ? 1u : 0u);
+        mma_ts4(tQd, tDs, desc_offset(dKm, sj * kStrTile), id_o, 128, jj > 0);
         umma_commit(b_mm);
         umma_commit(b_ke(sj));
         ++mm;

@@ -733,6 +733,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------ MMA issuer (even CTA)
     const uint32_t idesc = gemm_idesc<BN>(p.a_mn, p.b_mn);
+    // descriptors of stage 0, k-slice 0; a stage is STAGE bytes further, a
+    // 16-element k-slice +2 (K-major) or +128 (MN-major) in the address field
+    const uint64_t a0 = p.a_mn ? desc_mnmajor(sbase, 0) : desc_kmajor(sbase, 0);
+    const uint64_t b0 = p.b_mn ? desc_mnmajor(sbase + Cfg::A_BYTES, 0)
+                               : desc_kmajor(sbase + Cfg::A_BYTES, 0);
+    const uint64_t a_k = p.a_mn ? 128 : 2, b_k = p.b_mn ? 128 : 2;
     int stage = 0;
     uint32_t phase = 0;
     int t_local = 0;
@@ -752,13 +758,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t sa = sbase + stage * Cfg::STAGE, sb = sa + Cfg::A_BYTES;
+        const uint64_t ad = desc_offset(a0, stage * Cfg::STAGE);
+        const uint64_t bd = desc_offset(b0, stage * Cfg::STAGE);
+        if (kb == kb0)  // the tile's first MMA overwrites the accumulator
+          umma_pair_i<0>(d, ad, bd, idesc);
+        else
+          umma_pair_i<1>(d, ad, bd, idesc);
 #pragma unroll
-        for (int k = 0; k < BK / UMMA_K; ++k) {
-          const uint64_t ad = p.a_mn ? desc_mnmajor(sa, k) : desc_kmajor(sa, k);
-          const uint64_t bd = p.b_mn ? desc_mnmajor(sb, k) : desc_kmajor(sb, k);
-          umma_bf16_pair(d, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-        }
+        for (int k = 1; k < BK / UMMA_K; ++k) umma_pair_i<1>(d, ad + k * a_k, bd + k * b_k, idesc);
         umma_commit_pair(empty(stage), 3);  // frees the stage in both CTAs
         if (++stage == S) {
           stage = 0;

@@ -41,9 +41,11 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait on one phase; false (and the error word set) on expiry.
-static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int where) {
-  if (mbar_try(bar, parity)) return true;
+// Bounded wait on one phase; false (and the error word set) on expiry.  The
+// first try is inline (a completed phase costs one try_wait, ~16 cycles);
+// only the polling loop is an out-of-line call (~200 cycles of call overhead).
+static __device__ __noinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity, int* err,
+                                                   int where) {
   const uint64_t t0 = global_ns();
   while (true) {
 #pragma unroll 1
@@ -54,6 +56,9 @@ static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int where) {
+  return mbar_try(bar, parity) || mbar_wait_poll(bar, parity, err, where);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1) {
@@ -158,9 +163,8 @@ __device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) 
 }
 // Bounded wait (acquire at cluster scope) for barriers that the peer CTA or
 // the pair's MMA completes; false (and the error word set) on expiry.
-static __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int* err,
-                                                      int where) {
-  if (mbar_try_cluster(bar, parity)) return true;
+static __device__ __noinline__ bool mbar_wait_cluster_poll(uint32_t bar, uint32_t parity,
+                                                           int* err, int where) {
   const uint64_t t0 = global_ns();
   while (true) {
 #pragma unroll 1
@@ -171,6 +175,10 @@ static __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t par
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int* err,
+                                                  int where) {
+  return mbar_try_cluster(bar, parity) || mbar_wait_cluster_poll(bar, parity, err, where);
 }
 // every thread of both CTAs; the non-.aligned forms allow warps whose lanes
 // arrive at different times (role branches of single lanes)
@@ -247,6 +255,28 @@ __device__ __forceinline__ void bulk_wait_all() {
 // order this thread's generic-proxy shared-memory accesses before later async-proxy ones
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// tcgen05.mma with the accumulate flag as an immediate (ACC = 0: D = A B,
+// 1: D += A B): no predicate set-up per instruction, so a single issuing
+// thread keeps up with the tensor core even for N = 64 / 128 tiles.
+template <int ACC>
+__device__ __forceinline__ void umma_i(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc) {
+  asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, %4;" ::"r"(d), "l"(a),
+               "l"(b), "r"(idesc), "n"(ACC)
+               : "memory");
+}
+template <int ACC>
+__device__ __forceinline__ void umma_ts_i(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc) {
+  asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, %4;" ::"r"(d),
+               "r"(a_tmem), "l"(b), "r"(idesc), "n"(ACC)
+               : "memory");
+}
+template <int ACC>
+__device__ __forceinline__ void umma_pair_i(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc) {
+  asm volatile("tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, %4;" ::"r"(d), "l"(a),
+               "l"(b), "r"(idesc), "n"(ACC)
+               : "memory");
 }
 
 // tcgen05.mma with A read from TMEM (K-major, two bf16 per 32-bit column,
