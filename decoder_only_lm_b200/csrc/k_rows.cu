@@ -16,6 +16,7 @@
 #include <algorithm>
 
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace {
 
@@ -340,8 +341,8 @@ __global__ void reduce_ln_partials_kernel(const float* __restrict__ ws, int part
   *o = accumulate ? *o + acc : acc;
 }
 
-// Vectorised LayerNorm for C = 128 * NV (one warp per row, lane l owns the
-// float4 column groups 4l + 128i): the row lives in registers.
+// Vectorised LayerNorm for C = 128 * NV, one warp per row: lane l owns the
+// float4 column groups 4l + 128i of the row.
 template <typename T>
 __device__ __forceinline__ void load4(const T* p, float (&v)[4]);
 template <>
@@ -378,97 +379,186 @@ __device__ __forceinline__ void store4<bf16>(bf16* p, const float (&v)[4]) {
   *reinterpret_cast<uint2*>(p) = u;
 }
 
-template <int NV, typename OutT>
-__global__ void __launch_bounds__(256) layernorm_fwd_vec_kernel(
-    const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b,
-    OutT* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd, int64_t M,
-    float eps) {
-  constexpr int C = NV * 128;
-  const int64_t row = int64_t(blockIdx.x) * 8 + threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  if (row >= M) return;
-  const float* xr = x + row * C;
-  float v[NV][4];
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    load4<float>(xr + 4 * lane + 128 * i, v[i]);
-    s += (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
-  }
-  const float mu = warp_sum(s) / float(C);
-  float q = 0.f;
-#pragma unroll
-  for (int i = 0; i < NV; ++i)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float d = v[i][k] - mu;
-      q += d * d;
-    }
-  const float rs = rsqrtf(warp_sum(q) / float(C) + eps);
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c = 4 * lane + 128 * i;
-    float gg[4], bb[4], o[4];
-    load4<float>(g + c, gg);
-    load4<float>(b + c, bb);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) o[k] = (v[i][k] - mu) * rs * gg[k] + bb[k];
-    store4<OutT>(y + row * C + c, o);
-  }
+// Rows reach shared memory by bulk copies.  A block is kLnWarps warps and
+// the grid is persistent (a few blocks per SM); warp w of the grid takes rows
+// w, w + W, w + 2W, ... (W warps in the grid) and keeps a ring of S row
+// buffers of its own, each filled by one bulk copy S rows ahead of the row
+// it computes, so every warp has several rows of HBM reads in flight while
+// it reduces and writes the current one.  A wait that expires sets the error
+// word; the warp then computes nothing more but waits (bounded) for the
+// copies it has issued before it leaves.
+constexpr int kLnWarps = 8;
+constexpr int kLnMaxBlocks = 1024;  // grid cap (the backward's partial rows)
+
+// per-warp ring: S mbarriers and S stage buffers of `stage` bytes
+struct LnRing {
+  uint32_t bar0, buf0;
+  uint8_t* buf;
+  int S;
+  uint32_t stage;
+  __device__ uint32_t bar(int64_t k) const { return bar0 + 8u * uint32_t(k % S); }
+  __device__ uint32_t parity(int64_t k) const { return uint32_t((k / S) & 1); }
+  __device__ uint8_t* at(int64_t k) const { return buf + uint32_t(k % S) * stage; }
+  __device__ uint32_t at_s(int64_t k) const { return buf0 + uint32_t(k % S) * stage; }
+};
+// shared memory: kLnWarps * S barriers (padded to 128 bytes), then the
+// stage buffers [warp][stage]
+__host__ __device__ constexpr size_t ln_bar_bytes(int S) {
+  return (size_t(kLnWarps) * S * 8 + 127) / 128 * 128;
+}
+__device__ __forceinline__ LnRing ln_ring(uint8_t* smem, int S, uint32_t stage, int warp,
+                                          int lane) {
+  LnRing r;
+  r.S = S;
+  r.stage = stage;
+  r.bar0 = tc::smem_u32(smem) + uint32_t(warp * S * 8);
+  r.buf = smem + ln_bar_bytes(S) + size_t(warp) * S * stage;
+  r.buf0 = tc::smem_u32(r.buf);
   if (lane == 0) {
-    if (mean) mean[row] = mu;
-    if (rstd) rstd[row] = rs;
+    for (int i = 0; i < S; ++i) tc::mbar_init(r.bar0 + 8u * i, 1);
+    tc::fence_mbar_init();
   }
+  __syncwarp();
+  return r;
+}
+// waits (bounded) for the copies of rows [from, to) of the ring
+__device__ __forceinline__ void ln_drain(const LnRing& r, int64_t from, int64_t to, int* err,
+                                         int where) {
+  for (int64_t k = from; k < to; ++k) tc::mbar_wait(r.bar(k), r.parity(k), err, where);
 }
 
-constexpr int kLnVecRows = 8;  // rows per warp in the vectorised backward
+template <int NV, typename OutT>
+__global__ void __launch_bounds__(kLnWarps * 32) layernorm_fwd_staged_kernel(
+    const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b,
+    OutT* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd, int64_t M,
+    float eps, int S, int* err) {
+  constexpr int C = NV * 128;
+  constexpr uint32_t RB = C * 4;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t W = int64_t(gridDim.x) * kLnWarps;
+  const int64_t w0 = int64_t(blockIdx.x) * kLnWarps + warp;
+  const int64_t nk = w0 < M ? (M - 1 - w0) / W + 1 : 0;  // rows of this warp
+  const LnRing ring = ln_ring(smem, S, RB, warp, lane);
+  auto issue = [&](int64_t k) {
+    tc::mbar_expect_tx(ring.bar(k), RB);
+    tc::bulk_load_1d(ring.at_s(k), x + (w0 + k * W) * C, RB, ring.bar(k));
+  };
+  if (lane == 0)
+    for (int64_t k = 0; k < nk && k < S; ++k) issue(k);
+  float gg[NV][4], bb[NV][4];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    load4<float>(g + 4 * lane + 128 * i, gg[i]);
+    load4<float>(b + 4 * lane + 128 * i, bb[i]);
+  }
+  int64_t k = 0;
+  for (; k < nk; ++k) {
+    if (!__all_sync(0xffffffffu, tc::mbar_wait(ring.bar(k), ring.parity(k), err, 41))) break;
+    const float* xr = reinterpret_cast<const float*>(ring.at(k));
+    float v[NV][4];
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      load4<float>(xr + 4 * lane + 128 * i, v[i]);
+      sum += (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
+    }
+    const float mu = warp_sum(sum) / float(C);  // every lane's reads are done
+    if (lane == 0 && k + S < nk) issue(k + S);
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float dd = v[i][j] - mu;
+        q += dd * dd;
+      }
+    const float rs = rsqrtf(warp_sum(q) / float(C) + eps);
+    const int64_t row = w0 + k * W;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      float o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o[j] = (v[i][j] - mu) * rs * gg[i][j] + bb[i][j];
+      store4<OutT>(y + row * C + 4 * lane + 128 * i, o);
+    }
+    if (lane == 0) {
+      if (mean) mean[row] = mu;
+      if (rstd) rstd[row] = rs;
+    }
+  }
+  if (k < nk) ln_drain(ring, k, k + S < nk ? k + S : nk, err, 42);
+}
 
-// Each warp owns rows [w*8, w*8+8): dx is added into `dx` (and the new value
-// optionally stored rounded to CopyT).  The 8 warps' dgamma/dbeta column
-// partials are summed in warp order in shared memory and the block's partial
-// goes to ws[block][0..C) and ws[block][C..2C).
+// LayerNorm backward, C = 128 * NV: dx is ADDED to `dx` (the residual-stream
+// gradient) and, when dx_copy is given, the new dx is also stored rounded to
+// CopyT.  A stage holds the row's x, dx and dy.  Each warp keeps its column
+// partials of dgamma, dbeta and (want_sum) of the updated dx in registers; at
+// the end the block's warps are summed in warp order and the block's partial
+// goes to ws[block][parts][C] (parts = 2 or 3).
 template <int NV, typename DyT, typename CopyT>
-__global__ void __launch_bounds__(256) layernorm_bwd_vec_kernel(
+__global__ void __launch_bounds__(kLnWarps * 32, 1) layernorm_bwd_staged_kernel(
     const DyT* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ mean,
     const float* __restrict__ rstd, const float* __restrict__ g, int64_t M,
-    float* __restrict__ dx, CopyT* __restrict__ dx_copy, float* __restrict__ ws, int want_sum) {
+    float* __restrict__ dx, CopyT* __restrict__ dx_copy, float* __restrict__ ws, int want_sum,
+    int S, int* err) {
   constexpr int C = NV * 128;
-  __shared__ __align__(16) float red[8][C];
-  const int warp = threadIdx.x / 32;
-  const int64_t w = int64_t(blockIdx.x) * 8 + warp;
-  const int lane = threadIdx.x & 31;
-  const int64_t r0 = w * kLnVecRows;
-  // column partials: dgamma, dbeta and (want_sum) the updated dx itself
+  constexpr uint32_t RB = C * 4, DB = C * sizeof(DyT), ST = 2 * RB + DB;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t W = int64_t(gridDim.x) * kLnWarps;
+  const int64_t w0 = int64_t(blockIdx.x) * kLnWarps + warp;
+  const int64_t nk = w0 < M ? (M - 1 - w0) / W + 1 : 0;
+  const LnRing ring = ln_ring(smem, S, ST, warp, lane);
+  auto issue = [&](int64_t k) {
+    const int64_t row = w0 + k * W;
+    const uint32_t s = ring.at_s(k), bar = ring.bar(k);
+    tc::mbar_expect_tx(bar, ST);
+    tc::bulk_load_1d(s, x + row * C, RB, bar);
+    tc::bulk_load_1d(s + RB, dx + row * C, RB, bar);
+    tc::bulk_load_1d(s + 2 * RB, dy + row * C, DB, bar);
+  };
+  if (lane == 0)
+    for (int64_t k = 0; k < nk && k < S; ++k) issue(k);
   float gam[NV][4], pg[NV][4], pb[NV][4], ps[NV][4];
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     load4<float>(g + 4 * lane + 128 * i, gam[i]);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) pg[i][k] = pb[i][k] = ps[i][k] = 0.f;
+    for (int j = 0; j < 4; ++j) pg[i][j] = pb[i][j] = ps[i][j] = 0.f;
   }
-  for (int r = 0; r < kLnVecRows; ++r) {
-    const int64_t row = r0 + r;
-    if (row >= M) break;  // warp-uniform
-    const float mu = mean[row], rs = rstd[row];
-    float xh[NV][4], d[NV][4], cur[NV][4];
+  float mu = 0.f, rs = 0.f;
+  if (nk > 0) {
+    mu = mean[w0];
+    rs = rstd[w0];
+  }
+  int64_t k = 0;
+  for (; k < nk; ++k) {
+    const int64_t row = w0 + k * W;
+    float mu_n = 0.f, rs_n = 0.f;  // the next row's statistics, loaded early
+    if (k + 1 < nk) {
+      mu_n = mean[row + W];
+      rs_n = rstd[row + W];
+    }
+    if (!__all_sync(0xffffffffu, tc::mbar_wait(ring.bar(k), ring.parity(k), err, 43))) break;
+    const float* xr = reinterpret_cast<const float*>(ring.at(k));
+    const float* dxr = xr + C;
+    const DyT* dyr = reinterpret_cast<const DyT*>(xr + 2 * C);
     float a = 0.f, bsum = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c = 4 * lane + 128 * i;
-      load4<float>(x + row * C + c, xh[i]);
-      load4<DyT>(dy + row * C + c, d[i]);
-      load4<float>(dx + row * C + c, cur[i]);
-    }
+      float xh[4], d[4];
+      load4<float>(xr + c, xh);
+      load4<DyT>(dyr + c, d);
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        xh[i][k] = (xh[i][k] - mu) * rs;
-        const float dxh = d[i][k] * gam[i][k];
+      for (int j = 0; j < 4; ++j) {
+        xh[j] = (xh[j] - mu) * rs;
+        const float dxh = d[j] * gam[i][j];
         a += dxh;
-        bsum += dxh * xh[i][k];
-        pg[i][k] += d[i][k] * xh[i][k];
-        pb[i][k] += d[i][k];
+        bsum += dxh * xh[j];
+        pg[i][j] += d[j] * xh[j];
+        pb[i][j] += d[j];
       }
     }
     a = warp_sum(a) / float(C);
@@ -476,26 +566,41 @@ __global__ void __launch_bounds__(256) layernorm_bwd_vec_kernel(
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c = 4 * lane + 128 * i;
+      float xh[4], d[4], cur[4];
+      load4<float>(xr + c, xh);
+      load4<DyT>(dyr + c, d);
+      load4<float>(dxr + c, cur);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        cur[i][k] += rs * (d[i][k] * gam[i][k] - a - xh[i][k] * bsum);
-        ps[i][k] += cur[i][k];
+      for (int j = 0; j < 4; ++j) {
+        xh[j] = (xh[j] - mu) * rs;
+        cur[j] += rs * (d[j] * gam[i][j] - a - xh[j] * bsum);
+        ps[i][j] += cur[j];
       }
-      store4<float>(dx + row * C + c, cur[i]);
-      if (dx_copy) store4<CopyT>(dx_copy + row * C + c, cur[i]);
+      store4<float>(dx + row * C + c, cur);
+      if (dx_copy) store4<CopyT>(dx_copy + row * C + c, cur);
     }
+    __syncwarp();  // every lane has read the stage
+    if (lane == 0 && k + S < nk) issue(k + S);
+    mu = mu_n;
+    rs = rs_n;
   }
+  if (k < nk) ln_drain(ring, k, k + S < nk ? k + S : nk, err, 44);
+  // the block's column partials, summed over its warps in warp order; the
+  // stage buffers are free now (every copy has landed)
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(smem + ln_bar_bytes(S));  // [kLnWarps][C]
   const int parts = want_sum ? 3 : 2;
   float* out = ws + int64_t(blockIdx.x) * parts * C;
   for (int part = 0; part < parts; ++part) {
 #pragma unroll
     for (int i = 0; i < NV; ++i)
-      store4<float>(&red[warp][4 * lane + 128 * i], part == 0 ? pg[i] : part == 1 ? pb[i] : ps[i]);
+      store4<float>(red + warp * C + 4 * lane + 128 * i,
+                    part == 0 ? pg[i] : part == 1 ? pb[i] : ps[i]);
     __syncthreads();
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
       float t = 0.f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) t += red[k][c];
+      for (int w = 0; w < kLnWarps; ++w) t += red[w * C + c];
       out[part * C + c] = t;
     }
     __syncthreads();
@@ -792,6 +897,38 @@ int launch_embed_bwd(const int32_t* x, const float* dh, int B, int T, int C, int
   return GPT2_OK;
 }
 
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Launch shape of a staged LayerNorm kernel: S stages of `stage` bytes per
+// warp, a grid of as many blocks as fit on the device at once (at most one
+// per kLnWarps rows and kLnMaxBlocks).
+struct LnLaunch {
+  int S = 0, grid = 0;
+  size_t smem = 0;
+};
+template <typename K>
+int ln_launch_shape(K kernel, int64_t M, uint32_t stage, size_t budget, LnLaunch& L) {
+  L.S = int(std::min<size_t>(4, std::max<size_t>(2, budget / (size_t(kLnWarps) * stage))));
+  L.smem = ln_bar_bytes(L.S) + size_t(kLnWarps) * L.S * stage;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L.smem)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    gpt2_internal::set_error("layernorm: shared-memory size not accepted");
+    return GPT2_ERR_CUDA;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kLnWarps * 32, L.smem) !=
+          cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  L.grid = int(std::min<int64_t>({cdiv64(M, kLnWarps),
+                                  int64_t(per_sm) * gpt2_internal::sm_count(),
+                                  int64_t(kLnMaxBlocks)}));
+  return GPT2_OK;
+}
+
 template <typename OutT>
 int launch_layernorm_fwd(const float* x, const float* g, const float* b, OutT* y, float* mean,
                          float* rstd, int64_t M, int C, float eps, cudaStream_t st) {
@@ -799,12 +936,20 @@ int launch_layernorm_fwd(const float* x, const float* g, const float* b, OutT* y
     gpt2_internal::set_error("layernorm: C above 1024");
     return GPT2_ERR_ARG;
   }
-  switch (C) {
-#define LNF(NV)                                                                                  \
-  case NV * 128:                                                                               \
-    layernorm_fwd_vec_kernel<NV, OutT><<<int(cdiv64(M, 8)), 256, 0, st>>>(x, g, b, y, mean, rstd, \
-                                                                          M, eps);             \
-    break;
+  if (M <= 0) return GPT2_OK;
+  // the staged kernels move whole rows by bulk copies and float4 accesses
+  const bool aligned = al16(x) && al16(g) && al16(b) && al16(y);
+  switch (aligned ? C : -1) {
+#define LNF(NV)                                                                              \
+  case NV * 128: {                                                                         \
+    auto k = layernorm_fwd_staged_kernel<NV, OutT>;                                         \
+    LnLaunch L;                                                                            \
+    const int rc = ln_launch_shape(k, M, NV * 128 * 4, 96 * 1024, L);                      \
+    if (rc) return rc;                                                                     \
+    k<<<L.grid, kLnWarps * 32, L.smem, st>>>(x, g, b, y, mean, rstd, M, eps, L.S,           \
+                                            device_error_word());                          \
+    break;                                                                                 \
+  }
     LNF(1) LNF(2) LNF(3) LNF(4) LNF(5) LNF(6) LNF(7) LNF(8)
 #undef LNF
     default:
@@ -821,10 +966,15 @@ template int launch_layernorm_fwd<bf16>(const float*, const float*, const float*
                                         float*, int64_t, int, float, cudaStream_t);
 
 size_t layernorm_bwd_workspace(int64_t M, int C) {
-  const int64_t parts =
-      (C % 128 == 0 && C <= 1024) ? cdiv64(M, 8 * kLnVecRows) : cdiv64(M, kLnRowsPerBlock);
-  // dgamma | dbeta | column sums of dx (generic path: colsum partials after)
-  return std::max(size_t(parts) * 3 * C * sizeof(float), colsum_workspace(M, C));
+  // staged kernel: one [dgamma | dbeta | column sums of dx] row per block;
+  // generic kernel (also taken by unaligned views): [dgamma | dbeta] per 64
+  // rows, then the column-sum partials
+  const int64_t staged = (C % 128 == 0 && C <= 1024)
+                             ? std::min<int64_t>(cdiv64(M, kLnWarps), kLnMaxBlocks) * 3 * C
+                             : 0;
+  const int64_t generic = cdiv64(M, kLnRowsPerBlock) * 2 * C;
+  return std::max({size_t(staged) * sizeof(float), size_t(generic) * sizeof(float),
+                   colsum_workspace(M, C)});
 }
 
 template <typename DyT, typename CopyT>
@@ -835,31 +985,45 @@ int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const
     gpt2_internal::set_error("layernorm: C above 1024");
     return GPT2_ERR_ARG;
   }
-  if (C % 128 == 0 && C <= 1024) {
-    const int64_t warps = cdiv64(M, kLnVecRows);
-    const int nb = int(cdiv64(warps, 8));
-    switch (C / 128) {
+  if (C % 128 == 0 && C <= 1024 && al16(dy) && al16(x) && al16(g) && al16(dx) &&
+      al16(dx_copy) && al16(ws)) {
+    int nb = 0;  // blocks, one partial row of ws each
+    if (M > 0) {
+      switch (C / 128) {
 #define LNB(NV)                                                                              \
-  case NV:                                                                                   \
-    layernorm_bwd_vec_kernel<NV, DyT, CopyT><<<nb, 256, 0, st>>>(dy, x, mean, rstd, g, M, dx, \
-                                                                 dx_copy, ws, dsum != nullptr); \
-    break;
-      LNB(1) LNB(2) LNB(3) LNB(4) LNB(5) LNB(6) LNB(7) LNB(8)
+  case NV: {                                                                               \
+    auto k = layernorm_bwd_staged_kernel<NV, DyT, CopyT>;                                  \
+    LnLaunch L;                                                                            \
+    const int rc =                                                                         \
+        ln_launch_shape(k, M, NV * 128 * (8 + uint32_t(sizeof(DyT))), 200 * 1024, L);      \
+    if (rc) return rc;                                                                     \
+    k<<<L.grid, kLnWarps * 32, L.smem, st>>>(dy, x, mean, rstd, g, M, dx, dx_copy, ws,      \
+                                            dsum != nullptr, L.S, device_error_word());    \
+    nb = L.grid;                                                                           \
+    break;                                                                                 \
+  }
+        LNB(1) LNB(2) LNB(3) LNB(4) LNB(5) LNB(6) LNB(7) LNB(8)
 #undef LNB
+      }
+      COUNT_LAUNCH(1);
     }
-    COUNT_LAUNCH(1);
     const int n = (dsum ? 3 : 2) * C;
     reduce_rows_kernel<<<cdiv(n, 32), 256, 0, st>>>(ws, nb, n, dg, db, C, accumulate, dsum);
     COUNT_LAUNCH(1);
   } else {
     const int nb = int(cdiv64(M, kLnRowsPerBlock));
-    layernorm_bwd_kernel<DyT, CopyT><<<nb, 256, 0, st>>>(dy, x, mean, rstd, g, M, C, dx, dx_copy,
-                                                         ws);
-    COUNT_LAUNCH(1);
+    if (nb > 0) {
+      layernorm_bwd_kernel<DyT, CopyT><<<nb, 256, 0, st>>>(dy, x, mean, rstd, g, M, C, dx,
+                                                           dx_copy, ws);
+      COUNT_LAUNCH(1);
+    }
     // ws rows hold [dgamma | dbeta]; both halves are reduced in one pass
     reduce_ln_partials_kernel<<<cdiv(2 * C, 256), 256, 0, st>>>(ws, nb, C, dg, db, accumulate);
     COUNT_LAUNCH(1);
-    if (dsum) {  // column sums of the updated dx (same stream: ws is free again)
+    if (dsum && M == 0) {  // no rows: the column sums are zero
+      reduce_partials_kernel<<<cdiv(C, 256), 256, 0, st>>>(ws, 0, C, dsum, accumulate);
+      COUNT_LAUNCH(1);
+    } else if (dsum) {  // column sums of the updated dx (same stream: ws is free again)
       const int rc = launch_colsum<float>(dx, M, C, dsum, accumulate, ws, st);
       if (rc) return rc;
     }

@@ -24,7 +24,7 @@ def bf16_round(a):
     return torch.from_numpy(np.asarray(a, np.float32)).bfloat16().float().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("M,C", [(1, 64), (301, 768), (64, 1024)])
+@pytest.mark.parametrize("M,C", [(1, 64), (301, 768), (64, 1024), (20011, 768)])
 @pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
 def test_layernorm(g, M, C, bf16):
     import torch
@@ -49,6 +49,36 @@ def test_layernorm(g, M, C, bf16):
     assert rel_l2(dx.cpu().numpy(), dxo) <= 1e-4
     assert rel_l2(dgam.cpu().numpy(), dgo) <= 1e-4
     assert rel_l2(dbet.cpu().numpy(), dbo) <= 1e-4
+
+
+def test_layernorm_unaligned_view(g):
+    """Rows that do not start on a 16-byte boundary (a view 4 bytes into its
+    buffer) take the element-wise kernels and give the same values."""
+    import torch
+    rng = np.random.default_rng(5)
+    M, C = 97, 768
+    x = (rng.normal(size=(M, C)) * 2).astype(np.float32)
+    gam = rng.normal(size=C).astype(np.float32)
+    bet = rng.normal(size=C).astype(np.float32)
+    dy = rng.normal(size=(M, C)).astype(np.float32)
+    buf = torch.zeros(M * C + 1, device="cuda")
+    xv = buf[1:].view(M, C)
+    xv.copy_(torch.from_numpy(x))
+    assert xv.data_ptr() % 16 != 0
+    gt, bt = torch.from_numpy(gam).cuda(), torch.from_numpy(bet).cuda()
+    y0, m0, r0 = g.layernorm_fwd(torch.from_numpy(x).cuda(), gt, bt)
+    y1, m1, r1 = g.layernorm_fwd(xv, gt, bt)
+    yo, mo, ro = oracle.layernorm(x.astype(np.float64), gam, bet)
+    for y in (y0, y1):
+        assert np.max(np.abs(y.cpu().numpy() - yo)) <= 1e-5 * max(1, np.abs(yo).max())
+    dyt = torch.from_numpy(dy).cuda()
+    dx0, dg0, db0 = g.layernorm_bwd(dyt, torch.from_numpy(x).cuda(), m0, r0, gt)
+    dx1, dg1, db1 = g.layernorm_bwd(dyt, xv, m1, r1, gt)
+    dxo, dgo, dbo = oracle.layernorm_bwd(dy.astype(np.float64), x.astype(np.float64), mo, ro, gam)
+    for dx, dgm, dbt in ((dx0, dg0, db0), (dx1, dg1, db1)):
+        assert rel_l2(dx.cpu().numpy(), dxo) <= 1e-4
+        assert rel_l2(dgm.cpu().numpy(), dgo) <= 1e-4
+        assert rel_l2(dbt.cpu().numpy(), dbo) <= 1e-4
 
 
 @pytest.mark.parametrize("B,T,C,H", [(2, 37, 64, 4), (1, 200, 128, 2), (2, 64, 96, 3)])
