@@ -81,6 +81,7 @@ SIGNATURES = {
     "gpt2_matmul_workspace": (_i, [_i, _i, _i, C.POINTER(_sz)]),
     "gpt2_matmul": (_i, [_P, _i, _i64, _P, _i, _i64, _i, _i, _i, _i, _f, _i, _P, _i, _i64, _P,
                          _sz, _P]),
+    "gpt2_linear": (_i, [_i, _P, _P, _i, _P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "gpt2_device_error": (_i, [C.POINTER(_i)]),
 }
 
@@ -443,6 +444,30 @@ def matmul(A, B, a_kmajor=True, b_kmajor=True, M=None, N=None, K=None, alpha=1.0
                            _dtype_code(out), out.stride(0), _ptr(ws), ws_b.value,
                            _stream_ptr(stream)))
     return out
+
+
+LINEAR_BIAS, LINEAR_BIAS_GELU, LINEAR_RESIDUAL, LINEAR_GELU_BWD = 0, 1, 2, 3
+
+
+def linear(epi, x, w, bias=None, inp=None, w_kn=False, out=None, out2=None, stream=None):
+    """One linear layer with its fused epilogue (gpt2_linear): y = x W^T (W [N,K])
+    or x W (w_kn, W [K,N]), then bias / bias+GELU / residual add / GELU backward.
+    Returns out, or (out, pre-activation) for LINEAR_BIAS_GELU."""
+    import torch
+    M, K = x.shape
+    N = w.shape[1] if w_kn else w.shape[0]
+    if out is None:
+        dt = torch.float32 if epi == LINEAR_RESIDUAL else x.dtype
+        out = torch.empty((M, N), dtype=dt, device=x.device)
+    if epi == LINEAR_BIAS_GELU and out2 is None:
+        out2 = torch.empty((M, N), dtype=x.dtype, device=x.device)
+    ws_b = C.c_size_t()
+    _check(lib.gpt2_matmul_workspace(M, N, K, C.byref(ws_b)))
+    ws = torch.empty(max(ws_b.value, 1), dtype=torch.uint8, device=x.device)
+    _check(lib.gpt2_linear(epi, _ptr(x), _ptr(w), int(w_kn), _ptr(bias), _ptr(inp), _ptr(out),
+                           _ptr(out2), M, N, K, _dtype_code(x), _ptr(ws), ws_b.value,
+                           _stream_ptr(stream)))
+    return (out, out2) if epi == LINEAR_BIAS_GELU else out
 
 
 def cosine_lr(t, max_lr, min_lr, warmup_steps, total_steps):

@@ -189,6 +189,62 @@ int gpt2_matmul(const void* A, int a_kmajor, int64_t lda, const void* B, int b_k
   return gemm_launch(g, static_cast<cudaStream_t>(stream));
 }
 
+int gpt2_linear(int epi, const void* x, const void* w, int w_kn, const float* bias,
+                const void* in, void* out, void* out2, int M, int N, int K, int dtype,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !w || !out || M < 1 || N < 1 || K < 1 || (dtype != GPT2_BF16 && dtype != GPT2_F32)) {
+    set_error("linear: bad arguments");
+    return GPT2_ERR_ARG;
+  }
+  const int bf = dtype == GPT2_BF16;
+  EpiParams e;
+  e.ldo = N;
+  e.out_bf16 = bf;
+  switch (epi) {
+    case GPT2_LINEAR_BIAS:
+      e.kind = EPI_STORE;
+      e.out = out;
+      e.bias = bias;
+      break;
+    case GPT2_LINEAR_BIAS_GELU:
+      if (!bias || !out2) {
+        set_error("linear: bias+GELU needs bias and the pre-activation output");
+        return GPT2_ERR_ARG;
+      }
+      e.kind = EPI_GELU;
+      e.out = out2;  // pre-activation
+      e.out2 = out;  // GELU of it
+      e.bias = bias;
+      break;
+    case GPT2_LINEAR_RESIDUAL:
+      if (!in) {
+        set_error("linear: the residual epilogue needs its input");
+        return GPT2_ERR_ARG;
+      }
+      e.kind = EPI_RESID;
+      e.rin = static_cast<const float*>(in);
+      e.rout = static_cast<float*>(out);
+      e.bias = bias;
+      e.out_bf16 = 0;
+      break;
+    case GPT2_LINEAR_GELU_BWD:
+      if (!in || bias) {
+        set_error("linear: GELU backward needs the pre-activation and no bias");
+        return GPT2_ERR_ARG;
+      }
+      e.kind = EPI_GELU_BWD;
+      e.out = out;
+      e.aux = in;
+      break;
+    default:
+      set_error("linear: unknown epilogue");
+      return GPT2_ERR_ARG;
+  }
+  GemmArgs g{x, 1, K, w, w_kn ? 0 : 1, w_kn ? int64_t(N) : int64_t(K), bf, M, N, K, e,
+             static_cast<float*>(workspace), workspace_bytes};
+  return gemm_launch(g, static_cast<cudaStream_t>(stream));
+}
+
 int gpt2_device_error(int* code) {
   if (!code) return GPT2_ERR_ARG;
   int* w = device_error_word();

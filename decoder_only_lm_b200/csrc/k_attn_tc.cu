@@ -65,30 +65,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// packed pair arithmetic of sm_100: (a0, a1) * (b0, b1) + (c0, c1) and (a0, a1) + (b0, b1)
-__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
-                                     float c0, float c1) {
-  uint64_t ra, rb, rc, rd;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b0), "f"(b1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c0), "f"(c1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(rd));
-}
-__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
-  uint64_t ra, rd;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(rd) : "f"(d0), "f"(d1));
-  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(rd) : "l"(ra));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(rd));
-}
-__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1) {
-  uint64_t ra, rd;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(rd) : "f"(d0), "f"(d1));
-  asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(rd) : "l"(ra));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(rd));
-}
 // One 64-deep contraction as four K = 16 MMAs, the accumulate flag an
 // immediate: the first MMA overwrites D unless acc; descriptors advance by
 // a_k / b_k per slice (+2 K-major, +128 MN-major).  A from shared memory (ss)

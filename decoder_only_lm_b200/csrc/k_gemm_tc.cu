@@ -50,16 +50,26 @@ constexpr int kThreads = 384;  // warps 0-3: TMA, MMA, TMEM, idle; 4-7 and 8-11:
 
 constexpr int kSmemLimit = 232448;  // opt-in dynamic shared memory per block
 
+template <int EPI>
+__host__ __device__ constexpr bool epi_has_input() {
+  return EPI == EPI_RESID || EPI == EPI_GELU_BWD;
+}
+// k-block stages of the operand pipeline: epilogues with an input stream
+// keep more shared memory for their chunk buffers
+template <int EPI>
+__host__ __device__ constexpr int tc_stages(bool te) {
+  return !te ? 5 : epi_has_input<EPI>() ? 4 : 5;
+}
 // Shared memory: [STAGES x (A, B) k-block ring | epilogue area | barriers].
 // With the TMA epilogue (TE) the area is a set of 8 KB chunk buffers; GEMMs
 // whose epilogue reads an input (residual, GELU input) give up one k-block
 // stage for more buffers so that more input bytes are in flight.
-template <int BN, bool TE, bool IN>
+template <int BN, bool TE, int EPI>
 struct TcCfg {
   static constexpr int A_BYTES = BM * BK * 2;        // this CTA's 128 rows of A
   static constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's BN/2 rows of B
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = !TE ? 5 : (IN ? 4 : 5);
+  static constexpr int STAGES = tc_stages<EPI>(TE);
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int BAR_BYTES = 512;
   static constexpr int STAGE_ROW = 36;  // fp32 per staged accumulator row (32 + 4 pad)
@@ -75,10 +85,6 @@ struct TcCfg {
   static_assert(SMEM <= kSmemLimit, "shared memory");
   static_assert(!TE || NBUF_WG >= 4, "epilogue buffers");
 };
-template <int EPI>
-__host__ __device__ constexpr bool epi_has_input() {
-  return EPI == EPI_RESID || EPI == EPI_GELU_BWD;
-}
 
 struct TcParams {
   int M, N, K;
@@ -353,17 +359,54 @@ __device__ __forceinline__ float ex2_hw(float x) {
   return y;
 }
 constexpr float kLog2e = 1.4426950408889634f;
-__device__ __forceinline__ float gelu_hw(float u) {
-  const float k = 0.7978845608028654f, a = 0.044715f;
-  const float t = tanh_hw(u * (k + k * a * u * u));
-  const float h = 0.5f * u;
-  return fmaf(h, t, h);
+// The GELU epilogues two columns per packed instruction (fma/mul/add.f32x2).
+// With z = k (u + a u^3) and t = tanh z:  GELU(u) = u/2 (1 + t),
+// GELU'(u) = (1 + t)/2 + u/2 (1 - t^2) k (1 + 3 a u^2).
+constexpr float kGeluK = 0.7978845608028654f;  // sqrt(2 / pi)
+constexpr float kGeluKA = kGeluK * 0.044715f;
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
 }
-__device__ __forceinline__ float gelu_grad_hw(float u) {
-  const float k = 0.7978845608028654f, a = 0.044715f;
-  const float u2 = u * u;
-  const float t = tanh_hw(u * (k + k * a * u2));
-  return 0.5f * (1.f + t) + 0.5f * u * (1.f - t * t) * k * (1.f + 3.f * a * u2);
+// pre = bf16(v + b) (the stored pre-activation), act = bf16(GELU(pre)): the
+// activation is taken of the rounded value, the one the backward reads.
+__device__ __forceinline__ void gelu_chunk32(const float (&v)[32], const float (&b)[32],
+                                             uint32_t (&pre)[16], uint32_t (&act)[16]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    float x0 = v[j], x1 = v[j + 1];
+    add2(x0, x1, b[j], b[j + 1]);
+    const uint32_t pk = bf16x2_bits(x0, x1);
+    pre[j >> 1] = pk;
+    const float u0 = __uint_as_float(pk << 16), u1 = __uint_as_float(pk & 0xffff0000u);
+    float s0 = u0, s1 = u1, z0, z1;
+    mul2(s0, s1, u0, u1);
+    fma2(z0, z1, s0, s1, kGeluKA, kGeluKA, kGeluK, kGeluK);
+    mul2(z0, z1, u0, u1);
+    const float t0 = tanh_hw(z0), t1 = tanh_hw(z1);
+    float h0 = u0, h1 = u1, g0, g1;
+    mul2(h0, h1, 0.5f, 0.5f);
+    fma2(g0, g1, h0, h1, t0, t1, h0, h1);
+    act[j >> 1] = bf16x2_bits(g0, g1);
+  }
+}
+// (d0, d1) *= GELU'(u0, u1)
+__device__ __forceinline__ void gelu_bwd_pair(float& d0, float& d1, float u0, float u1) {
+  float s0 = u0, s1 = u1, z0, z1, q0, q1, m0, m1, g0, g1;
+  mul2(s0, s1, u0, u1);
+  fma2(z0, z1, s0, s1, kGeluKA, kGeluKA, kGeluK, kGeluK);
+  mul2(z0, z1, u0, u1);
+  const float t0 = tanh_hw(z0), t1 = tanh_hw(z1);
+  fma2(q0, q1, s0, s1, 3.f * kGeluKA, 3.f * kGeluKA, kGeluK, kGeluK);  // k (1 + 3 a u^2)
+  fma2(m0, m1, t0, t1, t0, t1, -1.f, -1.f);                            // t^2 - 1
+  float r0 = u0, r1 = u1;
+  mul2(r0, r1, -0.5f, -0.5f);
+  mul2(r0, r1, m0, m1);  // u/2 (1 - t^2)
+  mul2(r0, r1, q0, q1);
+  add2(r0, r1, 0.5f, 0.5f);
+  fma2(g0, g1, t0, t1, 0.5f, 0.5f, r0, r1);
+  mul2(d0, d1, g0, g1);
 }
 
 // Chunks of the TMA epilogue: 128 rows x 64 bytes (32 bf16 or 16 fp32
@@ -428,6 +471,13 @@ __device__ __forceinline__ void row_put<float>(uint8_t* buf, int r, const float 
   for (int u = 0; u < 4; ++u)
     *reinterpret_cast<float4*>(buf + swz64(r, u)) =
         make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+}
+// a row of 32 bf16 already packed in pairs
+__device__ __forceinline__ void row_put_bits(uint8_t* buf, int r, const uint32_t (&x)[16]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    *reinterpret_cast<uint4*>(buf + swz64(r, u)) =
+        make_uint4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
 }
 template <typename T>
 __device__ __forceinline__ void row_get(const uint8_t* buf, int r, float (&v)[64 / sizeof(T)]);
@@ -569,19 +619,17 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
           for (int j = 0; j < CW; ++j) v[j] += r[j];
         } else {
 #pragma unroll
-          for (int j = 0; j < CW; ++j) v[j] *= gelu_grad_hw(r[j]);
+          for (int j = 0; j < CW; j += 2) gelu_bwd_pair(v[j], v[j + 1], r[j], r[j + 1]);
         }
         row_put<OutT>(b0, e, v);
       } else if constexpr (EPI == EPI_GELU) {
-        float bb[CW], w[CW];
+        static_assert(CW == 32, "bf16 GELU chunks");
+        float bb[CW];
         bias_chunk<CW>(ep.bias, n0, p.N, bb);
-#pragma unroll
-        for (int j = 0; j < CW; ++j) {
-          v[j] = round_through<OutT>(v[j] + bb[j]);
-          w[j] = gelu_hw(v[j]);
-        }
-        row_put<OutT>(b0, e, v);
-        row_put<OutT>(b0 + 8192, e, w);
+        uint32_t pre[CW / 2], act[CW / 2];
+        gelu_chunk32(v, bb, pre, act);
+        row_put_bits(b0, e, pre);
+        row_put_bits(b0 + 8192, e, act);
       } else if constexpr (EPI == EPI_STORE) {
         if (ep.bias) {
           float bb[CW];
@@ -644,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tma_o,
                    const __grid_constant__ CUtensorMap tma_o2,
                    const __grid_constant__ CUtensorMap tma_i, const TcParams p) {
-  using Cfg = TcCfg<BN, TE, epi_has_input<EPI>()>;
+  using Cfg = TcCfg<BN, TE, EPI>;
   constexpr int S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -993,7 +1041,7 @@ int pair_slots() {
   static int slots = 0;
   static std::once_flag once;
   std::call_once(once, [] {
-    using Cfg = TcCfg<256, true, false>;
+    using Cfg = TcCfg<256, true, EPI_STORE>;
     auto kern = gemm_tc_kernel<256, EPI_STORE, bf16, true>;
     int n = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) ==
@@ -1034,7 +1082,7 @@ bool te_eligible(const GemmArgs& g, int splits) {
 
 template <int BN, int EPI, typename OutT, bool TE>
 int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
-  using Cfg = TcCfg<BN, TE, epi_has_input<EPI>()>;
+  using Cfg = TcCfg<BN, TE, EPI>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, OutT, TE>,

@@ -4,6 +4,7 @@
     python -m decoder_only_lm_b200.opbench lmhead --M 8192 --C 768 --Vp 50304 [--fwd-only]
     python -m decoder_only_lm_b200.opbench attention --B 16 --T 1024 --C 768 --H 12 [--bwd]
     python -m decoder_only_lm_b200.opbench layernorm --M 16384 --C 768 [--bwd]
+    python -m decoder_only_lm_b200.opbench linear --M 16384 --N 3072 --K 768 --epi gelu [--graph]
 
 Each call is timed with CUDA events on the current stream after warm-up and
 reported as one JSON line (ms per call, and TFLOP/s or GB/s of algorithmic
@@ -33,9 +34,36 @@ def timed(fn, iters, warmup):
     return a.elapsed_time(b) / iters
 
 
+def timed_graph(fn, iters, warmup):
+    """As timed(), but the iters calls are captured once as a CUDA graph and
+    the replay is timed: no host (binding) time between the launches."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for _ in range(iters):
+            fn()
+    gr.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    gr.replay()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+EPIS = {"bias": g.LINEAR_BIAS, "gelu": g.LINEAR_BIAS_GELU, "resid": g.LINEAR_RESIDUAL,
+        "gelu_bwd": g.LINEAR_GELU_BWD}
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["matmul", "lmhead", "attention", "layernorm"])
+    ap.add_argument("op", choices=["matmul", "lmhead", "attention", "layernorm", "linear"])
+    ap.add_argument("--epi", choices=sorted(EPIS), default="bias")
+    ap.add_argument("--graph", action="store_true",
+                    help="time a CUDA-graph replay of the calls (no host time in between)")
     ap.add_argument("--M", type=int, default=16384)
     ap.add_argument("--N", type=int, default=3072)
     ap.add_argument("--K", type=int, default=768)
@@ -53,6 +81,9 @@ def main():
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     a = ap.parse_args()
+    if a.graph:
+        global timed
+        timed = timed_graph
     torch.manual_seed(0)
     dev = "cuda"
     out = {"op": a.op}
@@ -65,6 +96,25 @@ def main():
         ms = timed(fn, a.iters, a.warmup)
         fl = 2.0 * a.M * a.N * a.K
         out.update(M=a.M, N=a.N, K=a.K, a_mn=a.a_mn, b_mn=a.b_mn, ms=ms, tflops=fl / ms / 1e9)
+    elif a.op == "linear":
+        # one linear layer of the block with its fused epilogue: x [M,K], W [N,K]
+        # (GELU backward: W [K,N]), bf16
+        x = torch.randn((a.M, a.K), device=dev).bfloat16()
+        w_kn = a.epi == "gelu_bwd"
+        w = (torch.randn((a.K, a.N) if w_kn else (a.N, a.K), device=dev) / a.K ** 0.5).bfloat16()
+        bias = None if w_kn else torch.randn(a.N, device=dev)
+        odt = torch.float32 if a.epi == "resid" else torch.bfloat16
+        o = torch.empty((a.M, a.N), device=dev, dtype=odt)
+        o2 = torch.empty((a.M, a.N), device=dev, dtype=torch.bfloat16) if a.epi == "gelu" else None
+        inp = None
+        if a.epi == "resid":
+            inp = torch.randn((a.M, a.N), device=dev)
+        elif a.epi == "gelu_bwd":
+            inp = torch.randn((a.M, a.N), device=dev).bfloat16()
+        fn = lambda: g.linear(EPIS[a.epi], x, w, bias=bias, inp=inp, w_kn=w_kn, out=o, out2=o2)
+        ms = timed(fn, a.iters, a.warmup)
+        fl = 2.0 * a.M * a.N * a.K
+        out.update(M=a.M, N=a.N, K=a.K, epi=a.epi, ms=ms, tflops=fl / ms / 1e9)
     elif a.op == "lmhead":
         h = torch.randn((a.M, a.C), device=dev).bfloat16()
         W = (0.02 * torch.randn((a.Vp, a.C), device=dev)).bfloat16()

@@ -351,6 +351,32 @@ int gpt2_matmul(const void* A, int a_kmajor, int64_t lda, const void* B, int b_k
                 int dtype, int M, int N, int K, float alpha, int accumulate, void* D, int d_dtype,
                 int64_t ldd, void* workspace, size_t workspace_bytes, void* stream);
 
+/* One linear layer of the block with its fused epilogue [ZERO: Transformer
+ * Block; LECTURE: GELU (tanh form)], as the training step runs it:
+ *   y = x W^T  with x [M,K] row-major and W [N,K] row-major (w_kn = 0: a
+ *   layer's weight as it is stored), or y = x W with W [K,N] (w_kn = 1: the
+ *   input-gradient contraction of the backward);
+ * then, by `epi`:
+ *   GPT2_LINEAR_BIAS       out = y + bias (bias may be NULL)
+ *   GPT2_LINEAR_BIAS_GELU  out2 = y + bias rounded to `dtype` (the
+ *                          pre-activation), out = GELU(out2); bias required
+ *   GPT2_LINEAR_RESIDUAL   out = in + y + bias, in and out fp32 (the residual
+ *                          stream; bias may be NULL; out must not overlap in)
+ *   GPT2_LINEAR_GELU_BWD   out = y * GELU'(in), in = the pre-activation
+ *                          (`dtype`); bias must be NULL
+ * GELU(u) = u/2 (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))).  x, W and the
+ * non-residual outputs are of type `dtype` (GPT2_BF16: tensor cores, fp32
+ * accumulation; GPT2_F32: SIMT).  Rows are contiguous (strides K, N).
+ * workspace >= gpt2_matmul_workspace(M, N, K).  GPT2_ERR_ARG on a null
+ * required pointer, a size below 1 or an unknown epi. */
+#define GPT2_LINEAR_BIAS 0
+#define GPT2_LINEAR_BIAS_GELU 1
+#define GPT2_LINEAR_RESIDUAL 2
+#define GPT2_LINEAR_GELU_BWD 3
+int gpt2_linear(int epi, const void* x, const void* w, int w_kn, const float* bias,
+                const void* in, void* out, void* out2, int M, int N, int K, int dtype,
+                void* workspace, size_t workspace_bytes, void* stream);
+
 /* Reads and clears the device error word shared by the op-level calls
  * (bounded-wait timeouts).  *code = GPT2_OK when nothing was recorded.
  * Synchronises the device. */

@@ -79,3 +79,17 @@ def test_null_arguments_are_refused(g):
     # the dz chunk is bounded at 16384 rows whatever M is
     assert g.lib.gpt2_lmhead_ce_workspace(65536, 768, 50304, g.BF16, C.byref(ws)) == g.OK
     assert 16384 * 50304 * 2 <= ws.value < 32768 * 50304 * 2
+    # fused linear layer: missing inputs and unknown epilogues are refused on the host
+    buf = C.c_void_p(16)  # never dereferenced: the arguments are rejected first
+    L = g.lib.gpt2_linear
+    assert L(g.LINEAR_BIAS, None, buf, 0, None, None, buf, None, 8, 8, 8, g.BF16, None, 0,
+             None) == g.ERR_ARG
+    assert L(g.LINEAR_BIAS_GELU, buf, buf, 0, None, None, buf, buf, 8, 8, 8, g.BF16, None, 0,
+             None) == g.ERR_ARG  # no bias
+    assert L(g.LINEAR_RESIDUAL, buf, buf, 0, None, None, buf, None, 8, 8, 8, g.BF16, None, 0,
+             None) == g.ERR_ARG  # no residual input
+    assert L(g.LINEAR_GELU_BWD, buf, buf, 1, buf, buf, buf, None, 8, 8, 8, g.BF16, None, 0,
+             None) == g.ERR_ARG  # a bias given
+    assert L(7, buf, buf, 0, None, None, buf, None, 8, 8, 8, g.BF16, None, 0, None) == g.ERR_ARG
+    assert L(g.LINEAR_BIAS, buf, buf, 0, None, None, buf, None, 0, 8, 8, g.BF16, None, 0,
+             None) == g.ERR_ARG

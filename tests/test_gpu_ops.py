@@ -168,3 +168,43 @@ def test_matmul_layouts(g, ak, bk, M, N, K, bf16):
     out2 = g.matmul(At, Bt, a_kmajor=bool(ak), b_kmajor=bool(bk), M=M, N=N, K=K, alpha=0.5,
                     out=out.clone(), accumulate=True)
     assert rel_l2(out2.cpu().numpy(), 1.5 * ref) <= 1e-5
+
+
+@pytest.mark.parametrize("epi", ["bias", "bias_gelu", "residual", "gelu_bwd"])
+@pytest.mark.parametrize("M,N,K", [(300, 520, 136), (1, 64, 64), (2050, 768, 3072)])
+@pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
+def test_linear_epilogues(g, epi, M, N, K, bf16):
+    """The fused linear layer against the oracle: the contraction in fp64 from
+    the same (rounded) operands, then the epilogue of the block it fuses."""
+    import torch
+    rng = np.random.default_rng(M + 7 * N + K)
+    dt = torch.bfloat16 if bf16 else torch.float32
+    w_kn = epi == "gelu_bwd"  # the backward contraction reads W as [K, N]
+    x = torch.from_numpy(rng.normal(size=(M, K)).astype(np.float32)).cuda().to(dt)
+    w = torch.from_numpy((rng.normal(size=(K, N) if w_kn else (N, K)) / np.sqrt(K))
+                         .astype(np.float32)).cuda().to(dt)
+    bias = torch.from_numpy(rng.normal(size=N).astype(np.float32)).cuda()
+    xr = x.float().cpu().numpy().astype(np.float64)
+    wr = w.float().cpu().numpy().astype(np.float64)
+    y = xr @ (wr if w_kn else wr.T)
+    tol = 1e-2 if bf16 else 1e-5
+    if epi == "bias":
+        out = g.linear(g.LINEAR_BIAS, x, w, bias=bias)
+        ref = y + bias.cpu().numpy()
+    elif epi == "bias_gelu":
+        out, pre = g.linear(g.LINEAR_BIAS_GELU, x, w, bias=bias)
+        pre_ref = y + bias.cpu().numpy()
+        assert rel_l2(pre.float().cpu().numpy(), pre_ref) <= tol
+        # the activation is taken of the stored (rounded) pre-activation
+        ref = oracle.gelu(pre.float().cpu().numpy().astype(np.float64))
+    elif epi == "residual":
+        res = torch.from_numpy(rng.normal(size=(M, N)).astype(np.float32)).cuda()
+        out = g.linear(g.LINEAR_RESIDUAL, x, w, bias=bias, inp=res)
+        assert out.dtype == torch.float32
+        ref = res.cpu().numpy() + y + bias.cpu().numpy()
+    else:
+        u = torch.from_numpy(rng.normal(size=(M, N)).astype(np.float32)).cuda().to(dt)
+        out = g.linear(g.LINEAR_GELU_BWD, x, w, inp=u, w_kn=True)
+        ref = oracle.gelu_bwd(y, u.float().cpu().numpy().astype(np.float64))
+    assert rel_l2(out.float().cpu().numpy(), ref) <= tol
+    assert g.device_error() == 0
