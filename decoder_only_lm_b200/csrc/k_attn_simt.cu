@@ -93,30 +93,33 @@ __global__ void attn_delta_kernel(const T* __restrict__ dout, const T* __restric
   if (lane == 0) delta[idx] = s;
 }
 
-// Delta for head size 64, bf16: one thread per (b, t, h) with h fastest, so a
-// warp reads consecutive 128-byte head slices of dO and O (16-byte loads).
+// Delta for head size 64, bf16: eight lanes per (b, t, h) row, h fastest, so
+// a warp's 16-byte loads cover four consecutive 128-byte head slices of dO
+// and of O (512 contiguous bytes each); the eight partial dot products are
+// summed with three shuffles.
 __global__ void attn_delta64_kernel(const bf16* __restrict__ dout, const bf16* __restrict__ out,
                                     int B, int Tn, int C, int H, float* __restrict__ delta) {
-  const int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-  if (idx >= int64_t(B) * Tn * H) return;
+  const int64_t idx = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 3;  // row
+  const int part = threadIdx.x & 7;
+  if (idx >= int64_t(B) * Tn * H) return;  // whole 8-lane groups leave together
   const int h = int(idx % H);
   const int64_t bt = idx / H;  // b * T + t
   const int b = int(bt / Tn), t = int(bt % Tn);
-  const uint4* pa = reinterpret_cast<const uint4*>(dout + bt * C + h * 64);
-  const uint4* pb = reinterpret_cast<const uint4*>(out + bt * C + h * 64);
+  const uint4 ua = *reinterpret_cast<const uint4*>(dout + bt * C + h * 64 + part * 8);
+  const uint4 ub = *reinterpret_cast<const uint4*>(out + bt * C + h * 64 + part * 8);
+  const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&ua);
+  const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&ub);
   float s = 0.f;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint4 ua = pa[k], ub = pb[k];
-    const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&ua);
-    const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&ub);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 fa = __bfloat1622float2(ha[j]), fb = __bfloat1622float2(hb[j]);
-      s += fa.x * fb.x + fa.y * fb.y;
-    }
+  for (int j = 0; j < 4; ++j) {
+    const float2 fa = __bfloat1622float2(ha[j]), fb = __bfloat1622float2(hb[j]);
+    s += fa.x * fb.x + fa.y * fb.y;
   }
-  delta[(int64_t(b) * H + h) * Tn + t] = s;
+  const unsigned grp = 0xffu << (threadIdx.x & 24);  // this row's eight lanes
+  s += __shfl_xor_sync(grp, s, 4);
+  s += __shfl_xor_sync(grp, s, 2);
+  s += __shfl_xor_sync(grp, s, 1);
+  if (part == 0) delta[(int64_t(b) * H + h) * Tn + t] = s;
 }
 
 // One thread per key j: dv_j = sum_{i>=j} p_ij do_i, dk_j = sum_{i>=j} ds_ij q_i / sqrt(D)
@@ -347,7 +350,7 @@ int launch_attn_bwd<bf16>(const bf16* dout, const bf16* qkv, const bf16* out, co
   if (!attn_tc_supported(B, Tn, C, H))
     return launch_attn_simt_bwd<bf16>(dout, qkv, out, lse, B, Tn, C, H, dqkv, ws, st);
   const int64_t rows = int64_t(B) * H * Tn;
-  attn_delta64_kernel<<<int(cdiv64(rows, 256)), 256, 0, st>>>(dout, out, B, Tn, C, H, ws);
+  attn_delta64_kernel<<<int(cdiv64(rows * 8, 256)), 256, 0, st>>>(dout, out, B, Tn, C, H, ws);
   COUNT_LAUNCH(1);
   return launch_attn_tc_bwd(dout, qkv, lse, ws, B, Tn, C, H, dqkv, st);
 }
