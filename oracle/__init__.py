@@ -233,3 +233,51 @@ def lmhead_ce(h, W, y, vocab_size=None, grad_scale=1.0, grads=True):
                                                         M, Cc, Vp, vocab_size or Vp, grad_scale,
                                                         C.byref(loss), _ptr(rl), _ptr(dh), _ptr(dW)))
     return loss.value, rl, dh, dW
+
+
+def sample(logits, vocab, temperature, top_k, top_p, u):
+    """Next-token choice for each row of ``logits`` [B, >= vocab] (fp32), following
+    the text-generation section of the CS336 pre-training page (§5: temperature,
+    top-p) and the lecture's top-k, step by step:
+
+    - temperature == 0 (or top_k == 1): the highest logit, the first such id on
+      ties (greedy decoding);
+    - else p_i = exp((z_i - max z) / temperature) in fp32 over the first
+      ``vocab`` columns (the real vocabulary; padding columns are never drawn);
+    - order the ids by probability, highest first, the smaller id first among
+      equal probabilities;
+    - top_k > 0: keep the first top_k of that order;
+    - top_p < 1: keep, in that order, each id whose cumulative probability
+      before it (fp64, relative to the kept mass) is below top_p, i.e. the
+      shortest prefix whose mass reaches top_p;
+    - draw with u[b] in [0, 1): walk the kept ids in increasing id order,
+      accumulating p in fp64, and return the first id at which the sum exceeds
+      u[b] times the kept mass (the last kept id if rounding leaves none).
+
+    Returns int32 [B].
+    """
+    z_all = np.asarray(logits, dtype=np.float32)
+    B = z_all.shape[0]
+    u = np.asarray(u, dtype=np.float32).reshape(-1) if u is not None else None
+    out = np.empty(B, dtype=np.int32)
+    for b in range(B):
+        z = z_all[b, :vocab]
+        if temperature == 0 or top_k == 1:
+            out[b] = int(np.argmax(z))
+            continue
+        p = np.exp((z - z.max()) / np.float32(temperature)).astype(np.float32)
+        ids = np.arange(vocab)
+        order = np.lexsort((ids, -p))  # probability descending, then id ascending
+        if 0 < top_k < vocab:
+            order = order[:top_k]
+        if top_p < 1:
+            cum = np.cumsum(p[order].astype(np.float64))
+            cut = int(np.argmax(cum >= np.float64(np.float32(top_p)) * cum[-1])) + 1
+            order = order[:cut]
+        kept = np.sort(order)
+        pk = p[kept].astype(np.float64)
+        target = np.float64(u[b]) * pk.sum()
+        cum = np.cumsum(pk)
+        hit = np.nonzero(cum > target)[0]
+        out[b] = kept[hit[0]] if hit.size else kept[-1]
+    return out
