@@ -235,6 +235,10 @@ def lmhead_ce(h, W, y, vocab_size=None, grad_scale=1.0, grads=True):
     return loss.value, rl, dh, dW
 
 
+# weights of the draw: probabilities as integers in units of 2^-36 (exact sums)
+SAMPLE_WEIGHT_SCALE = 2.0 ** 36
+
+
 def sample(logits, vocab, temperature, top_k, top_p, u):
     """Next-token choice for each row of ``logits`` [B, >= vocab] (fp32), following
     the text-generation section of the CS336 pre-training page (§5: temperature,
@@ -243,16 +247,17 @@ def sample(logits, vocab, temperature, top_k, top_p, u):
     - temperature == 0 (or top_k == 1): the highest logit, the first such id on
       ties (greedy decoding);
     - else p_i = exp((z_i - max z) / temperature) in fp32 over the first
-      ``vocab`` columns (the real vocabulary; padding columns are never drawn);
+      ``vocab`` columns (the real vocabulary; padding columns are never drawn),
+      and the weight of id i is w_i = rint(p_i * 2^36) (an integer: every
+      cumulative probability below is an exact integer sum);
     - order the ids by probability, highest first, the smaller id first among
       equal probabilities;
     - top_k > 0: keep the first top_k of that order;
-    - top_p < 1: keep, in that order, each id whose cumulative probability
-      before it (fp64, relative to the kept mass) is below top_p, i.e. the
-      shortest prefix whose mass reaches top_p;
+    - top_p < 1: keep, in that order, the shortest prefix whose weight reaches
+      top_p times the kept weight (the crossing id included);
     - draw with u[b] in [0, 1): walk the kept ids in increasing id order,
-      accumulating p in fp64, and return the first id at which the sum exceeds
-      u[b] times the kept mass (the last kept id if rounding leaves none).
+      accumulating w, and return the first id at which the sum exceeds
+      u[b] times the kept weight (the last kept id if none does).
 
     Returns int32 [B].
     """
@@ -266,18 +271,20 @@ def sample(logits, vocab, temperature, top_k, top_p, u):
             out[b] = int(np.argmax(z))
             continue
         p = np.exp((z - z.max()) / np.float32(temperature)).astype(np.float32)
+        w = np.rint(p.astype(np.float64) * SAMPLE_WEIGHT_SCALE).astype(np.int64)
         ids = np.arange(vocab)
         order = np.lexsort((ids, -p))  # probability descending, then id ascending
         if 0 < top_k < vocab:
             order = order[:top_k]
         if top_p < 1:
-            cum = np.cumsum(p[order].astype(np.float64))
-            cut = int(np.argmax(cum >= np.float64(np.float32(top_p)) * cum[-1])) + 1
+            cum = np.cumsum(w[order])
+            need = np.float64(np.float32(top_p)) * np.float64(cum[-1])
+            cut = int(np.argmax(cum.astype(np.float64) >= need)) + 1
             order = order[:cut]
         kept = np.sort(order)
-        pk = p[kept].astype(np.float64)
-        target = np.float64(u[b]) * pk.sum()
-        cum = np.cumsum(pk)
+        wk = w[kept]
+        target = np.float64(u[b]) * np.float64(wk.sum())
+        cum = np.cumsum(wk).astype(np.float64)
         hit = np.nonzero(cum > target)[0]
         out[b] = kept[hit[0]] if hit.size else kept[-1]
     return out
