@@ -60,6 +60,9 @@ SIGNATURES = {
     "gpt2_train_step": (_i, [_P, _P, _P, _i, _i, _i, _f, _f, _f, _f, _f, _f, C.POINTER(_f),
                              C.POINTER(_f)]),
     "gpt2_eval_loss": (_i, [_P, _P, _P, _i, _i, _i, C.POINTER(_f)]),
+    "gpt2_logits_last": (_i, [_P, _P, _i, _i, _i, _P, _i64]),
+    "gpt2_sample": (_i, [_P, _i64, _i, _i, _f, _i, _f, _P, _P, _i64, _P]),
+    "gpt2_generate": (_i, [_P, _P, _i, _i, _i, _f, _i, _f, _P, _P]),
     "gpt2_stream_begin": (_i, [_P, _P, _i64, _i64, _i64, _i, _i, _i, _f, _f, _f, _f, _f]),
     "gpt2_stream_steps": (_i, [_P, _i, C.POINTER(_f)]),
     "gpt2_stream_end": (_i, [_P, C.POINTER(_i64)]),
@@ -293,6 +296,26 @@ class GPT2:
         _check(lib.gpt2_eval_loss(self.h, _ptr(x), _ptr(y), B, T, dev, C.byref(out)), self.h)
         return out.value
 
+    def logits_last(self, x):
+        """fp32 logits [B, padded_vocab] of the last position of each row of x [B, T]."""
+        torch = self.torch
+        x, _, B, T, dev = self._xy(x, x)
+        out = torch.empty((B, self.cfg.padded_vocab), dtype=torch.float32, device="cuda")
+        _check(lib.gpt2_logits_last(self.h, _ptr(x), B, T, dev, _ptr(out), out.stride(0)), self.h)
+        return out
+
+    def generate(self, prompt, n_new, temperature=0.8, top_k=0, top_p=0.9, uniform=None):
+        """prompt: int32 cuda [B, T0]; uniform: fp32 cuda [n_new, B] in [0, 1) (None
+        for greedy settings).  Returns int32 cuda [B, T0 + n_new]."""
+        torch = self.torch
+        prompt = prompt.to(device="cuda", dtype=torch.int32).contiguous()
+        B, T0 = prompt.shape
+        out = torch.empty((B, T0 + n_new), dtype=torch.int32, device="cuda")
+        u = None if uniform is None else uniform.to(device="cuda", dtype=torch.float32).contiguous()
+        _check(lib.gpt2_generate(self.h, _ptr(prompt), B, T0, n_new, temperature, top_k, top_p,
+                                 _ptr(u), _ptr(out)), self.h)
+        return out
+
     def synchronize(self):
         _check(lib.gpt2_synchronize(self.h), self.h)
 
@@ -468,6 +491,21 @@ def linear(epi, x, w, bias=None, inp=None, w_kn=False, out=None, out2=None, stre
                            _ptr(out2), M, N, K, _dtype_code(x), _ptr(ws), ws_b.value,
                            _stream_ptr(stream)))
     return (out, out2) if epi == LINEAR_BIAS_GELU else out
+
+
+def sample(logits, vocab, temperature=0.8, top_k=0, top_p=0.9, uniform=None, out=None,
+           stream=None):
+    """Next token of each row of fp32 cuda logits [B, >= vocab] (gpt2_sample);
+    uniform: fp32 cuda [B] in [0, 1) (None for greedy settings)."""
+    import torch
+    B = logits.shape[0]
+    if out is None:
+        out = torch.empty(B, dtype=torch.int32, device=logits.device)
+    u = None if uniform is None else uniform.to(device=logits.device, dtype=torch.float32).contiguous()
+    _check(lib.gpt2_sample(_ptr(logits), logits.stride(0), B, vocab, temperature, top_k, top_p,
+                           _ptr(u), _ptr(out), out.stride(0) if out.dim() > 1 else 1,
+                           _stream_ptr(stream)))
+    return out
 
 
 def cosine_lr(t, max_lr, min_lr, warmup_steps, total_steps):

@@ -81,6 +81,7 @@ struct gpt2_handle {
   bf16* Pb = nullptr;
   // activations
   int32_t *xbuf = nullptr, *ybuf = nullptr;
+  float* gen_logits = nullptr;  // [max_B, Vp] fp32, allocated by the first generation call
   std::vector<float*> res;
   std::vector<void*> ln1, qkv, att, ln2, u, g;
   std::vector<float*> mu1, rs1, mu2, rs2, alse;
@@ -395,8 +396,11 @@ int stage_tokens(gpt2_handle* h, const int32_t* x, const int32_t* y, int64_t M, 
 
 double gemm_flops(int64_t M, int64_t N, int64_t K) { return 2.0 * double(M) * double(N) * double(K); }
 
+// With d_logits the step ends after the final LayerNorm with the tied head
+// applied to the last position of each sequence only (fp32 [B, ld_logits]).
 template <typename A>
-int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save) {
+int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save,
+              float* d_logits = nullptr, int64_t ld_logits = 0) {
   const int64_t M = int64_t(B) * T;
   const int C = h->C, F = h->F, Vp = h->Vp, Hh = h->H;
   const int ab = h->use_bf16;
@@ -468,6 +472,17 @@ int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save) {
     PROF(GPT2_PROF_LN_FWD, 0, ln_bytes);
     H_TRY(h, launch_layernorm_fwd<A>(h->res[2 * h->L], P + h->off_lnfw, P + h->off_lnfb, hf,
                                      h->muf, h->rsf, M, C, h->cfg.ln_eps, h->st));
+  }
+  if (d_logits) {
+    // rows T-1, 2T-1, ...: the last position of each sequence (row stride T*C)
+    PROF(GPT2_PROF_LMHEAD, gemm_flops(B, Vp, C), a * (double(B) * C + double(Vp) * C) + 4.0 * B * Vp);
+    EpiParams e = epi(EPI_STORE, d_logits, ld_logits, 0);
+    H_TRY(h, gemm(h, hf + int64_t(T - 1) * C, 1, int64_t(T) * C, wptr(h, h->off_wte), 1, C, B, Vp,
+                  C, e));
+    h->fwd_saved = false;
+    h->fB = B;
+    h->fT = T;
+    return GPT2_OK;
   }
   {
     // tied head + cross-entropy: no logits are stored (see lmhead_fwd)
@@ -978,6 +993,60 @@ int gpt2_eval_loss(gpt2_handle* h, const int32_t* x, const int32_t* y, int B, in
   else
     H_TRY(h, forward_t<float>(h, B, T, nullptr, false));
   return read_loss(h, loss_out);
+}
+
+int gpt2_logits_last(gpt2_handle* h, const int32_t* x, int B, int T, int tokens_on_device,
+                     float* logits, int64_t ld) {
+  if (!h || !x || !logits) return fail(h, GPT2_ERR_ARG, "NULL argument");
+  H_TRY(h, validate_bt(h, B, T));
+  if (ld < h->Vp) return fail(h, GPT2_ERR_ARG, "logits_last: ld below padded_vocab");
+  h->fwd_saved = false;
+  // the targets buffer only feeds the embedding's id range check: give it x
+  H_TRY(h, stage_tokens(h, x, x, int64_t(B) * T, tokens_on_device));
+  if (h->use_bf16)
+    H_TRY(h, forward_t<bf16>(h, B, T, nullptr, false, logits, ld));
+  else
+    H_TRY(h, forward_t<float>(h, B, T, nullptr, false, logits, ld));
+  return check_status(h);
+}
+
+int gpt2_generate(gpt2_handle* h, const int32_t* prompt, int B, int T0, int n_new,
+                  float temperature, int top_k, float top_p, const float* uniform,
+                  int32_t* out) {
+  if (!h || !prompt || !out) return fail(h, GPT2_ERR_ARG, "NULL argument");
+  if (B < 1 || B > h->cfg.max_B || T0 < 1 || n_new < 0)
+    return fail(h, GPT2_ERR_ARG, "generate: B outside 1..max_B, T0 < 1 or n_new < 0");
+  const bool greedy = temperature == 0.f || top_k == 1;
+  if (!(temperature >= 0.f) || top_k < 0 || !(top_p > 0.f && top_p <= 1.f) ||
+      (!greedy && !uniform))
+    return fail(h, GPT2_ERR_ARG, "generate: bad sampling settings or no uniform numbers");
+  if (h->V > kSampleMaxVocab) return fail(h, GPT2_ERR_ARG, "generate: vocab_size above 53248");
+  const int Wmax = std::min(h->Tmax, h->cfg.max_Tseq);
+  const int64_t Ttot = int64_t(T0) + n_new;
+  h->fwd_saved = false;
+  if (!h->gen_logits) {
+    h->gen_logits = static_cast<float*>(dev_alloc(h, size_t(h->cfg.max_B) * h->Vp * sizeof(float)));
+    if (!h->gen_logits) return fail(h, GPT2_ERR_OOM, "generate: logits buffer");
+  }
+  H_CUDA(h, cudaMemcpy2DAsync(out, Ttot * sizeof(int32_t), prompt, T0 * sizeof(int32_t),
+                              T0 * sizeof(int32_t), B, cudaMemcpyDeviceToDevice, h->st));
+  for (int s = 0; s < n_new; ++s) {
+    const int64_t Tc = int64_t(T0) + s;
+    const int W = int(std::min<int64_t>(Tc, Wmax));
+    // the window out[:, Tc-W .. Tc) as a contiguous [B, W] batch
+    H_CUDA(h, cudaMemcpy2DAsync(h->xbuf, W * sizeof(int32_t), out + (Tc - W),
+                                Ttot * sizeof(int32_t), W * sizeof(int32_t), B,
+                                cudaMemcpyDeviceToDevice, h->st));
+    H_CUDA(h, cudaMemcpyAsync(h->ybuf, h->xbuf, size_t(B) * W * sizeof(int32_t),
+                              cudaMemcpyDeviceToDevice, h->st));
+    if (h->use_bf16)
+      H_TRY(h, forward_t<bf16>(h, B, W, nullptr, false, h->gen_logits, h->Vp));
+    else
+      H_TRY(h, forward_t<float>(h, B, W, nullptr, false, h->gen_logits, h->Vp));
+    H_TRY(h, launch_sample(h->gen_logits, h->Vp, B, h->V, temperature, top_k, top_p,
+                           greedy ? nullptr : uniform + int64_t(s) * B, out + Tc, Ttot, h->st));
+  }
+  return check_status(h);
 }
 
 // ---------------------------------------------------------------- stream training (graph)

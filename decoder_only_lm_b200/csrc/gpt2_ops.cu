@@ -245,6 +245,20 @@ int gpt2_linear(int epi, const void* x, const void* w, int w_kn, const float* bi
   return gemm_launch(g, static_cast<cudaStream_t>(stream));
 }
 
+int gpt2_sample(const float* logits, int64_t ld, int B, int V, float temperature, int top_k,
+                float top_p, const float* uniform, int32_t* out, int64_t out_stride,
+                void* stream) {
+  const bool greedy = temperature == 0.f || top_k == 1;
+  if (!logits || !out || B < 1 || V < 1 || V > kSampleMaxVocab || ld < V || out_stride < 1 ||
+      !(temperature >= 0.f) || top_k < 0 || !(top_p > 0.f && top_p <= 1.f) ||
+      (!greedy && !uniform)) {
+    set_error("sample: bad arguments");
+    return GPT2_ERR_ARG;
+  }
+  return launch_sample(logits, ld, B, V, temperature, top_k, top_p, uniform, out, out_stride,
+                       static_cast<cudaStream_t>(stream));
+}
+
 int gpt2_device_error(int* code) {
   if (!code) return GPT2_ERR_ARG;
   int* w = device_error_word();

@@ -97,6 +97,17 @@ int launch_ce_rows_bwd(const float* z, const float* lse, const int32_t* y, int r
                        float scale, OutT* dz, cudaStream_t st);
 int launch_mean(const float* v, int64_t n, float* out, cudaStream_t st);
 
+// ---------------------------------------------------------------- sampling
+// next token of each of B rows of fp32 logits (row stride ld, first V columns):
+// temperature (0 = greedy), top_k (0 = off), top_p (1 = off), uniform[b] in
+// [0, 1); out[b * out_stride] (int32).  V <= kSampleMaxVocab (one row in
+// shared memory, ids in 16 bits).
+constexpr int kSampleMaxVocab = 53248;
+size_t sample_max_vocab();
+int launch_sample(const float* logits, int64_t ld, int B, int V, float temperature, int top_k,
+                  float top_p, const float* uniform, int32_t* out, int64_t out_stride,
+                  cudaStream_t st);
+
 // ---------------------------------------------------------------- attention
 template <typename T>
 int launch_attn_fwd(const T* qkv, int B, int Tn, int C, int H, T* out, float* lse,

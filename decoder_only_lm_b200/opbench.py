@@ -5,6 +5,8 @@
     python -m decoder_only_lm_b200.opbench attention --B 16 --T 1024 --C 768 --H 12 [--bwd]
     python -m decoder_only_lm_b200.opbench layernorm --M 16384 --C 768 [--bwd]
     python -m decoder_only_lm_b200.opbench linear --M 16384 --N 3072 --K 768 --epi gelu [--graph]
+    python -m decoder_only_lm_b200.opbench sample --B 16 --V 50257 [--temperature 0.8 --top-k 0 --top-p 0.9]
+    python -m decoder_only_lm_b200.opbench generate --B 16 --T0 64 --new 64 (GPT-2 124M, bf16)
 
 Each call is timed with CUDA events on the current stream after warm-up and
 reported as one JSON line (ms per call, and TFLOP/s or GB/s of algorithmic
@@ -60,7 +62,13 @@ EPIS = {"bias": g.LINEAR_BIAS, "gelu": g.LINEAR_BIAS_GELU, "resid": g.LINEAR_RES
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["matmul", "lmhead", "attention", "layernorm", "linear"])
+    ap.add_argument("op", choices=["matmul", "lmhead", "attention", "layernorm", "linear",
+                                   "sample", "generate"])
+    ap.add_argument("--temperature", type=float, default=0.8)
+    ap.add_argument("--top-k", type=int, default=0)
+    ap.add_argument("--top-p", type=float, default=0.9)
+    ap.add_argument("--T0", type=int, default=64)
+    ap.add_argument("--new", type=int, default=64)
     ap.add_argument("--epi", choices=sorted(EPIS), default="bias")
     ap.add_argument("--graph", action="store_true",
                     help="time a CUDA-graph replay of the calls (no host time in between)")
@@ -115,6 +123,36 @@ def main():
         ms = timed(fn, a.iters, a.warmup)
         fl = 2.0 * a.M * a.N * a.K
         out.update(M=a.M, N=a.N, K=a.K, epi=a.epi, ms=ms, tflops=fl / ms / 1e9)
+    elif a.op == "sample":
+        # next-token choice over B rows of fp32 logits (the padded width, V drawn)
+        z = 3.0 * torch.randn((a.B, a.Vp), device=dev)
+        u = torch.rand(a.B, device=dev)
+        o = torch.empty(a.B, dtype=torch.int32, device=dev)
+        fn = lambda: g.sample(z, a.V, a.temperature, a.top_k, a.top_p, u, out=o)
+        ms = timed(fn, a.iters, a.warmup)
+        out.update(B=a.B, V=a.V, temperature=a.temperature, top_k=a.top_k, top_p=a.top_p, ms=ms,
+                   gbs=a.B * a.V * 4 / ms / 1e6)
+    elif a.op == "generate":
+        # GPT-2 124M (bf16, N(0, 0.02) weights): a prompt of T0 ids, then `new`
+        # tokens, each recomputing the whole window (no KV cache)
+        import synth
+        m = g.GPT2(12, 768, 12, 50257, 50304, 1024, bf16=True, max_B=a.B, max_Tseq=1024)
+        m.set_params(synth.init_params(0, m.shapes()))
+        prompt = torch.randint(0, 50257, (a.B, a.T0), dtype=torch.int32, device=dev)
+        u = torch.rand((a.new, a.B), device=dev)
+        for _ in range(a.warmup):
+            m.generate(prompt, 2, a.temperature, a.top_k, a.top_p, u[:2])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        m.generate(prompt, a.new, a.temperature, a.top_k, a.top_p, u)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        out.update(B=a.B, T0=a.T0, new=a.new, temperature=a.temperature, top_k=a.top_k,
+                   top_p=a.top_p, ms=ms, ms_per_token_step=ms / a.new,
+                   tokens_per_s=a.B * a.new / ms * 1e3)
+        m.close()
     elif a.op == "lmhead":
         h = torch.randn((a.M, a.C), device=dev).bfloat16()
         W = (0.02 * torch.randn((a.Vp, a.C), device=dev)).bfloat16()

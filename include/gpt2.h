@@ -232,6 +232,53 @@ int gpt2_stream_end(gpt2_handle* h, int64_t* cursor_out);
 int gpt2_eval_loss(gpt2_handle* h, const int32_t* x, const int32_t* y, int B, int T,
                    int tokens_on_device, float* loss_out);
 
+/* ---------------------------------------------------------------- generation */
+
+/* Logits of the last position of every sequence [CS336: text generation,
+ * "the last position's logits"; LECTURE: sampling loop]: the forward pass over
+ * x (int32 [B*T], host or device as in gpt2_forward_loss; no activations
+ * saved, a saved forward is invalidated), the final LayerNorm, and the tied
+ * head for row T-1 of each sequence only:
+ *   logits[b*ld + v] = hf[b, T-1] . wte[v]   for v < padded_vocab (fp32, device)
+ * ld >= padded_vocab.  Synchronises (an id out of range gives GPT2_ERR_TOKEN).
+ * Needs 1 <= B <= max_B, 1 <= T <= max_Tseq. */
+int gpt2_logits_last(gpt2_handle* h, const int32_t* x, int B, int T, int tokens_on_device,
+                     float* logits, int64_t ld);
+
+/* Next token of each of B rows of fp32 logits [CS336: text generation —
+ * temperature and top-p; LECTURE: top-k]:
+ *   temperature == 0 or top_k == 1: the highest logit (the smaller id on ties);
+ *   otherwise p_i = exp((z_i - max z) / temperature) in fp32 over the first V
+ *   columns (the real vocabulary: padding columns are never drawn); ids are
+ *   ordered by p, the smaller id first among equal p; top_k > 0 keeps the
+ *   first top_k of that order; top_p < 1 keeps its shortest prefix whose mass
+ *   reaches top_p times the kept mass (the crossing id included); the draw
+ *   walks the kept ids in increasing id order, summing p in fp64, and returns
+ *   the first id at which the sum exceeds uniform[b] * (kept mass) (the last
+ *   kept id if rounding leaves the target unreached).
+ * logits: device fp32, row b at logits + b*ld (ld >= V).  uniform: device fp32
+ * [B] in [0, 1) (values outside are clamped; may be NULL for greedy choices).
+ * out: device int32, out[b*out_stride].  Deterministic.  GPT2_ERR_ARG unless
+ * 1 <= V <= 53248, B >= 1, temperature >= 0, top_k >= 0, 0 < top_p <= 1. */
+int gpt2_sample(const float* logits, int64_t ld, int B, int V, float temperature, int top_k,
+                float top_p, const float* uniform, int32_t* out, int64_t out_stride,
+                void* stream);
+
+/* Autoregressive generation without a KV cache [CS336: text generation —
+ * every step recomputes the whole window, keeping only the most recent
+ * context-length tokens]: out (device int32 [B, T0 + n_new]) receives the
+ * prompt (device int32 [B, T0]) followed by n_new tokens; token T0 + s of row b
+ * is gpt2_sample over the logits of gpt2_logits_last on the window
+ * out[b, max(0, T0+s-W) .. T0+s) with W = min(max_T, max_Tseq), drawn with
+ * uniform[s*B + b] (device fp32 [n_new, B]; NULL allowed for greedy choices).
+ * Every step runs on the handle's stream without host synchronisation; the call
+ * synchronises once at the end (GPT2_ERR_TOKEN for an id out of range in the
+ * prompt).  No early stop at an end-of-text id: the caller cuts the rows.
+ * Needs 1 <= B <= max_B, T0 >= 1, n_new >= 0, vocab_size <= 53248. */
+int gpt2_generate(gpt2_handle* h, const int32_t* prompt, int B, int T0, int n_new,
+                  float temperature, int top_k, float top_p, const float* uniform,
+                  int32_t* out);
+
 /* Waits for the stream and reports a device-side error recorded since the
  * last check (token range, non-finite norm, bounded-wait timeout). */
 int gpt2_synchronize(gpt2_handle* h);

@@ -93,3 +93,15 @@ def test_null_arguments_are_refused(g):
     assert L(7, buf, buf, 0, None, None, buf, None, 8, 8, 8, g.BF16, None, 0, None) == g.ERR_ARG
     assert L(g.LINEAR_BIAS, buf, buf, 0, None, None, buf, None, 0, 8, 8, g.BF16, None, 0,
              None) == g.ERR_ARG
+    # sampling: sizes and settings are checked on the host before any launch
+    S = g.lib.gpt2_sample
+    assert S(buf, 16, 1, 0, 1.0, 0, 0.9, buf, buf, 1, None) == g.ERR_ARG  # V = 0
+    assert S(buf, 16, 1, 53249, 1.0, 0, 0.9, buf, buf, 1, None) == g.ERR_ARG  # V too large
+    assert S(buf, 8, 1, 16, 1.0, 0, 0.9, buf, buf, 1, None) == g.ERR_ARG  # ld < V
+    assert S(buf, 16, 1, 16, -0.5, 0, 0.9, buf, buf, 1, None) == g.ERR_ARG  # temperature < 0
+    assert S(buf, 16, 1, 16, 1.0, -1, 0.9, buf, buf, 1, None) == g.ERR_ARG  # top_k < 0
+    assert S(buf, 16, 1, 16, 1.0, 0, 0.0, buf, buf, 1, None) == g.ERR_ARG  # top_p = 0
+    assert S(buf, 16, 1, 16, 1.0, 0, 1.5, buf, buf, 1, None) == g.ERR_ARG  # top_p > 1
+    assert S(buf, 16, 1, 16, 1.0, 0, 0.9, None, buf, 1, None) == g.ERR_ARG  # no uniforms
+    assert g.lib.gpt2_generate(None, buf, 1, 4, 4, 0.0, 0, 1.0, None, buf) == g.ERR_ARG
+    assert g.lib.gpt2_logits_last(None, buf, 1, 4, 1, buf, 64) == g.ERR_ARG
