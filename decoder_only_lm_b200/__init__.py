@@ -63,6 +63,7 @@ SIGNATURES = {
     "gpt2_logits_last": (_i, [_P, _P, _i, _i, _i, _P, _i64]),
     "gpt2_sample": (_i, [_P, _i64, _i, _i, _f, _i, _f, _P, _P, _i64, _P]),
     "gpt2_generate": (_i, [_P, _P, _i, _i, _i, _f, _i, _f, _P, _P]),
+    "gpt2_generate_cached": (_i, [_P, _P, _i, _i, _i, _f, _i, _f, _P, _P]),
     "gpt2_stream_begin": (_i, [_P, _P, _i64, _i64, _i64, _i, _i, _i, _f, _f, _f, _f, _f]),
     "gpt2_stream_steps": (_i, [_P, _i, C.POINTER(_f)]),
     "gpt2_stream_end": (_i, [_P, C.POINTER(_i64)]),
@@ -304,16 +305,20 @@ class GPT2:
         _check(lib.gpt2_logits_last(self.h, _ptr(x), B, T, dev, _ptr(out), out.stride(0)), self.h)
         return out
 
-    def generate(self, prompt, n_new, temperature=0.8, top_k=0, top_p=0.9, uniform=None):
+    def generate(self, prompt, n_new, temperature=0.8, top_k=0, top_p=0.9, uniform=None,
+                 cached=False):
         """prompt: int32 cuda [B, T0]; uniform: fp32 cuda [n_new, B] in [0, 1) (None
-        for greedy settings).  Returns int32 cuda [B, T0 + n_new]."""
+        for greedy settings).  cached: keep a key/value cache (gpt2_generate_cached)
+        instead of recomputing the window every step.  Returns int32 cuda
+        [B, T0 + n_new]."""
         torch = self.torch
         prompt = prompt.to(device="cuda", dtype=torch.int32).contiguous()
         B, T0 = prompt.shape
         out = torch.empty((B, T0 + n_new), dtype=torch.int32, device="cuda")
         u = None if uniform is None else uniform.to(device="cuda", dtype=torch.float32).contiguous()
-        _check(lib.gpt2_generate(self.h, _ptr(prompt), B, T0, n_new, temperature, top_k, top_p,
-                                 _ptr(u), _ptr(out)), self.h)
+        fn = lib.gpt2_generate_cached if cached else lib.gpt2_generate
+        _check(fn(self.h, _ptr(prompt), B, T0, n_new, temperature, top_k, top_p, _ptr(u), _ptr(out)),
+               self.h)
         return out
 
     def synchronize(self):

@@ -82,6 +82,11 @@ struct gpt2_handle {
   // activations
   int32_t *xbuf = nullptr, *ybuf = nullptr;
   float* gen_logits = nullptr;  // [max_B, Vp] fp32, allocated by the first generation call
+  // key/value cache of incremental decoding: per layer [max_B, H, kv_T, D] (activation type),
+  // allocated by the first cached generation
+  void* kcache = nullptr;
+  void* vcache = nullptr;
+  int kv_T = 0;
   std::vector<float*> res;
   std::vector<void*> ln1, qkv, att, ln2, u, g;
   std::vector<float*> mu1, rs1, mu2, rs2, alse;
@@ -398,9 +403,16 @@ double gemm_flops(int64_t M, int64_t N, int64_t K) { return 2.0 * double(M) * do
 
 // With d_logits the step ends after the final LayerNorm with the tied head
 // applied to the last position of each sequence only (fp32 [B, ld_logits]).
+// With kv the tokens sit at positions kv->pos0 .. pos0 + T - 1, each layer's
+// keys and values are stored into the cache there, and (kv->decode, T = 1)
+// attention reads the cache positions 0 .. pos0 instead of the batch.
+struct KvStep {
+  int pos0;
+  bool decode;
+};
 template <typename A>
 int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save,
-              float* d_logits = nullptr, int64_t ld_logits = 0) {
+              float* d_logits = nullptr, int64_t ld_logits = 0, const KvStep* kv = nullptr) {
   const int64_t M = int64_t(B) * T;
   const int C = h->C, F = h->F, Vp = h->Vp, Hh = h->H;
   const int ab = h->use_bf16;
@@ -413,7 +425,7 @@ int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save,
   {
     PROF(GPT2_PROF_EMBED, 0, 12.0 * M * C);
     H_TRY(h, launch_embed_fwd(h->xbuf, h->ybuf, P + h->off_wte, P + h->off_wpe, B, T, C, h->V,
-                              h->res[0], h->status, h->st));
+                              h->res[0], h->status, h->st, kv ? kv->pos0 : 0));
   }
   const double ln_bytes = M * C * (4.0 + a) + 8.0 * M;
   const double attn_flops = 2.0 * B * Hh * double(T) * T * (C / Hh);
@@ -434,7 +446,16 @@ int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save,
       e.bias = P + o.qkvb;
       H_TRY(h, gemm(h, ln1, 1, C, wptr(h, o.qkvw), 1, C, int(M), 3 * C, C, e));
     }
-    {
+    if (kv) {
+      const size_t per_layer = size_t(h->cfg.max_B) * Hh * h->kv_T * (C / Hh);
+      A* kc = static_cast<A*>(h->kcache) + l * per_layer;
+      A* vc = static_cast<A*>(h->vcache) + l * per_layer;
+      PROF(GPT2_PROF_ATTN_FWD, 0, a * 4.0 * M * C);
+      H_TRY(h, launch_kv_store<A>(qkv, B, T, C, Hh, kv->pos0, h->kv_T, kc, vc, h->st));
+      if (kv->decode)
+        H_TRY(h, launch_attn_decode<A>(qkv, kc, vc, B, C, Hh, h->kv_T, kv->pos0 + 1, att, h->st));
+    }
+    if (!kv || !kv->decode) {
       PROF(GPT2_PROF_ATTN_FWD, attn_flops, a * 4.0 * M * C + 4.0 * M * Hh);
       H_TRY(h, launch_attn_fwd<A>(qkv, B, T, C, Hh, att, h->alse[l], h->st));
     }
@@ -1045,6 +1066,58 @@ int gpt2_generate(gpt2_handle* h, const int32_t* prompt, int B, int T0, int n_ne
       H_TRY(h, forward_t<float>(h, B, W, nullptr, false, h->gen_logits, h->Vp));
     H_TRY(h, launch_sample(h->gen_logits, h->Vp, B, h->V, temperature, top_k, top_p,
                            greedy ? nullptr : uniform + int64_t(s) * B, out + Tc, Ttot, h->st));
+  }
+  return check_status(h);
+}
+
+int gpt2_generate_cached(gpt2_handle* h, const int32_t* prompt, int B, int T0, int n_new,
+                         float temperature, int top_k, float top_p, const float* uniform,
+                         int32_t* out) {
+  if (!h || !prompt || !out) return fail(h, GPT2_ERR_ARG, "NULL argument");
+  const int Tc = std::min(h->Tmax, h->cfg.max_Tseq);
+  if (B < 1 || B > h->cfg.max_B || T0 < 1 || n_new < 0 || int64_t(T0) + n_new > Tc)
+    return fail(h, GPT2_ERR_ARG,
+                "generate_cached: B outside 1..max_B, T0 < 1, n_new < 0 or T0 + n_new above "
+                "min(max_T, max_Tseq)");
+  const bool greedy = temperature == 0.f || top_k == 1;
+  if (!(temperature >= 0.f) || top_k < 0 || !(top_p > 0.f && top_p <= 1.f) ||
+      (!greedy && !uniform))
+    return fail(h, GPT2_ERR_ARG, "generate_cached: bad sampling settings or no uniform numbers");
+  if (h->V > kSampleMaxVocab)
+    return fail(h, GPT2_ERR_ARG, "generate_cached: vocab_size above 53248");
+  if (Tc > 4096 || (h->C / h->H) > 128 || 128 % (h->C / h->H) != 0)
+    return fail(h, GPT2_ERR_ARG, "generate_cached: context above 4096 or head size unsupported");
+  const int64_t Ttot = int64_t(T0) + n_new;
+  h->fwd_saved = false;
+  if (!h->gen_logits) {
+    h->gen_logits = static_cast<float*>(dev_alloc(h, size_t(h->cfg.max_B) * h->Vp * sizeof(float)));
+    if (!h->gen_logits) return fail(h, GPT2_ERR_OOM, "generate: logits buffer");
+  }
+  if (!h->kcache) {
+    const size_t bytes = size_t(h->L) * h->cfg.max_B * h->C * size_t(Tc) * h->act_size();
+    h->kcache = dev_alloc(h, bytes);
+    h->vcache = dev_alloc(h, bytes);
+    if (!h->kcache || !h->vcache) return fail(h, GPT2_ERR_OOM, "generate_cached: KV cache");
+    h->kv_T = Tc;
+  }
+  H_CUDA(h, cudaMemcpy2DAsync(out, Ttot * sizeof(int32_t), prompt, T0 * sizeof(int32_t),
+                              T0 * sizeof(int32_t), B, cudaMemcpyDeviceToDevice, h->st));
+  for (int s = 0; s < n_new; ++s) {
+    // step 0: the prompt at positions 0 .. T0-1 fills the cache; step s > 0:
+    // the token generated last, at position T0 + s - 1, attends to the cache
+    const int Tn = s == 0 ? T0 : 1;
+    const KvStep kv{s == 0 ? 0 : T0 + s - 1, s > 0};
+    const int32_t* src = s == 0 ? out : out + (T0 + s - 1);
+    H_CUDA(h, cudaMemcpy2DAsync(h->xbuf, Tn * sizeof(int32_t), src, Ttot * sizeof(int32_t),
+                                Tn * sizeof(int32_t), B, cudaMemcpyDeviceToDevice, h->st));
+    H_CUDA(h, cudaMemcpyAsync(h->ybuf, h->xbuf, size_t(B) * Tn * sizeof(int32_t),
+                              cudaMemcpyDeviceToDevice, h->st));
+    if (h->use_bf16)
+      H_TRY(h, forward_t<bf16>(h, B, Tn, nullptr, false, h->gen_logits, h->Vp, &kv));
+    else
+      H_TRY(h, forward_t<float>(h, B, Tn, nullptr, false, h->gen_logits, h->Vp, &kv));
+    H_TRY(h, launch_sample(h->gen_logits, h->Vp, B, h->V, temperature, top_k, top_p,
+                           greedy ? nullptr : uniform + int64_t(s) * B, out + T0 + s, Ttot, h->st));
   }
   return check_status(h);
 }

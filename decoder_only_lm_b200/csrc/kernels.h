@@ -58,8 +58,10 @@ int launch_slice_batch(const uint16_t* s, int64_t off, int64_t n, int32_t* x, in
 int launch_slice_batch_cursor(const uint16_t* s, int64_t len, const int64_t* cur, int64_t n,
                               int32_t* x, int32_t* y, DevStatus* status, cudaStream_t st);
 int launch_advance_cursor(int64_t* cur, int64_t stride, cudaStream_t st);
+// positions pos0 .. pos0 + T - 1 (pos0 > 0: one step of incremental decoding)
 int launch_embed_fwd(const int32_t* x, const int32_t* y, const float* wte, const float* wpe,
-                     int B, int T, int C, int V, float* out, DevStatus* status, cudaStream_t st);
+                     int B, int T, int C, int V, float* out, DevStatus* status, cudaStream_t st,
+                     int pos0 = 0);
 // dwte[x_m] += dh[m] (deterministic: sort by id, segmented sums); dwpe[t] (+)= sum_b dh[b,t].
 size_t embed_bwd_workspace(int64_t M, int C);
 int launch_embed_bwd(const int32_t* x, const float* dh, int B, int T, int C, int V, float* dwte,
@@ -96,6 +98,17 @@ template <typename OutT>
 int launch_ce_rows_bwd(const float* z, const float* lse, const int32_t* y, int rows, int Vp,
                        float scale, OutT* dz, cudaStream_t st);
 int launch_mean(const float* v, int64_t n, float* out, cudaStream_t st);
+
+// ---------------------------------------------------------------- KV-cache decoding
+// K, V caches per layer: [B, H, Tc, D] of the activation type.
+template <typename T>
+int launch_kv_store(const T* qkv, int B, int Tn, int C, int H, int pos0, int Tc, T* kc, T* vc,
+                    cudaStream_t st);
+// out[b, h*D .. ] = attention of the single query row b of qkv [B, 3C] over
+// cache positions 0 .. L-1 (L <= Tc, L <= 4096, D <= 128 dividing 128)
+template <typename T>
+int launch_attn_decode(const T* qkv, const T* kc, const T* vc, int B, int C, int H, int Tc, int L,
+                       T* out, cudaStream_t st);
 
 // ---------------------------------------------------------------- sampling
 // next token of each of B rows of fp32 logits (row stride ld, first V columns):

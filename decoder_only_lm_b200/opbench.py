@@ -6,7 +6,7 @@
     python -m decoder_only_lm_b200.opbench layernorm --M 16384 --C 768 [--bwd]
     python -m decoder_only_lm_b200.opbench linear --M 16384 --N 3072 --K 768 --epi gelu [--graph]
     python -m decoder_only_lm_b200.opbench sample --B 16 --V 50257 [--temperature 0.8 --top-k 0 --top-p 0.9]
-    python -m decoder_only_lm_b200.opbench generate --B 16 --T0 64 --new 64 (GPT-2 124M, bf16)
+    python -m decoder_only_lm_b200.opbench generate --B 16 --T0 64 --new 64 [--cached] (GPT-2 124M, bf16)
 
 Each call is timed with CUDA events on the current stream after warm-up and
 reported as one JSON line (ms per call, and TFLOP/s or GB/s of algorithmic
@@ -69,6 +69,7 @@ def main():
     ap.add_argument("--top-p", type=float, default=0.9)
     ap.add_argument("--T0", type=int, default=64)
     ap.add_argument("--new", type=int, default=64)
+    ap.add_argument("--cached", action="store_true", help="generate with the key/value cache")
     ap.add_argument("--epi", choices=sorted(EPIS), default="bias")
     ap.add_argument("--graph", action="store_true",
                     help="time a CUDA-graph replay of the calls (no host time in between)")
@@ -141,15 +142,15 @@ def main():
         prompt = torch.randint(0, 50257, (a.B, a.T0), dtype=torch.int32, device=dev)
         u = torch.rand((a.new, a.B), device=dev)
         for _ in range(a.warmup):
-            m.generate(prompt, 2, a.temperature, a.top_k, a.top_p, u[:2])
+            m.generate(prompt, 2, a.temperature, a.top_k, a.top_p, u[:2], cached=a.cached)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        m.generate(prompt, a.new, a.temperature, a.top_k, a.top_p, u)
+        m.generate(prompt, a.new, a.temperature, a.top_k, a.top_p, u, cached=a.cached)
         e1.record()
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1)
-        out.update(B=a.B, T0=a.T0, new=a.new, temperature=a.temperature, top_k=a.top_k,
+        out.update(B=a.B, T0=a.T0, new=a.new, cached=a.cached, temperature=a.temperature, top_k=a.top_k,
                    top_p=a.top_p, ms=ms, ms_per_token_step=ms / a.new,
                    tokens_per_s=a.B * a.new / ms * 1e3)
         m.close()

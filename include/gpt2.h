@@ -279,6 +279,20 @@ int gpt2_generate(gpt2_handle* h, const int32_t* prompt, int B, int T0, int n_ne
                   float temperature, int top_k, float top_p, const float* uniform,
                   int32_t* out);
 
+/* gpt2_generate with a key/value cache [CS336: text generation — the cache
+ * reuses the history instead of recomputing the window]: the prompt runs once
+ * through the model at positions 0 .. T0-1 and every layer's keys and values
+ * are kept; each later step runs only the last generated token (position
+ * T0+s-1) through the block, its attention reading the cached positions
+ * 0 .. T0+s-1.  Same arguments, output and sampling as gpt2_generate, the same
+ * tokens up to floating-point order (the same computation regrouped).  Needs
+ * T0 + n_new <= min(max_T, max_Tseq) <= 4096 (no window slides) and a head
+ * size dividing 128.  The first call allocates the cache: 2 * n_layer *
+ * max_B * n_embd * min(max_T, max_Tseq) activation elements. */
+int gpt2_generate_cached(gpt2_handle* h, const int32_t* prompt, int B, int T0, int n_new,
+                         float temperature, int top_k, float top_p, const float* uniform,
+                         int32_t* out);
+
 /* Waits for the stream and reports a device-side error recorded since the
  * last check (token range, non-finite norm, bounded-wait timeout). */
 int gpt2_synchronize(gpt2_handle* h);

@@ -104,4 +104,5 @@ def test_null_arguments_are_refused(g):
     assert S(buf, 16, 1, 16, 1.0, 0, 1.5, buf, buf, 1, None) == g.ERR_ARG  # top_p > 1
     assert S(buf, 16, 1, 16, 1.0, 0, 0.9, None, buf, 1, None) == g.ERR_ARG  # no uniforms
     assert g.lib.gpt2_generate(None, buf, 1, 4, 4, 0.0, 0, 1.0, None, buf) == g.ERR_ARG
+    assert g.lib.gpt2_generate_cached(None, buf, 1, 4, 4, 0.0, 0, 1.0, None, buf) == g.ERR_ARG
     assert g.lib.gpt2_logits_last(None, buf, 1, 4, 1, buf, 64) == g.ERR_ARG

@@ -132,3 +132,57 @@ def test_generate_fp32_matches_oracle_loop(g):
         seq = np.concatenate([seq, nxt[:, None]], axis=1)
     np.testing.assert_array_equal(out, seq)
     gm.close()
+
+
+@pytest.mark.parametrize("setting", [(0.0, 0, 1.0), (0.8, 0, 0.9), (1.0, 20, 1.0)])
+def test_cached_generation_fp32_equals_recompute_and_oracle(g, setting):
+    """fp32 mode: the KV-cache path gives the tokens of the recompute path and
+    of the oracle's own loop (prompt + new tokens within the context)."""
+    import torch
+    T, k, p = setting
+    om, params, gm = tiny(g, False)
+    rng = np.random.default_rng(21)
+    B, T0, n = 3, 17, 30
+    prompt = rng.integers(0, 512, size=(B, T0)).astype(np.int32)
+    u = rng.random((n, B)).astype(np.float32)
+    ut = None if T == 0 else torch.from_numpy(u).cuda()
+    pt = torch.from_numpy(prompt).cuda()
+    cached = gm.generate(pt, n, T, k, p, ut, cached=True).cpu().numpy()
+    full = gm.generate(pt, n, T, k, p, ut).cpu().numpy()
+    np.testing.assert_array_equal(cached, full)
+    seq = prompt.copy()
+    for s in range(n):
+        lg = oracle_last_logits(om, params, seq).astype(np.float32)
+        seq = np.concatenate([seq, oracle.sample(lg, 512, T, k, p, u[s])[:, None]], axis=1)
+    np.testing.assert_array_equal(cached, seq)
+    gm.close()
+
+
+def test_cached_generation_bf16_tracks_recompute(g):
+    """bf16 mode: greedy tokens of the cached and the recompute path agree (the
+    two paths group the same bf16 computation differently, so a near-tie may
+    flip a late token), and the cached path is deterministic."""
+    import torch
+    om, params, gm = tiny(g, True)
+    rng = np.random.default_rng(22)
+    B, T0, n = 4, 9, 40
+    pt = torch.from_numpy(rng.integers(0, 512, size=(B, T0)).astype(np.int32)).cuda()
+    a = gm.generate(pt, n, 0.0, 0, 1.0, None, cached=True).cpu().numpy()
+    b = gm.generate(pt, n, 0.0, 0, 1.0, None, cached=True).cpu().numpy()
+    np.testing.assert_array_equal(a, b)
+    full = gm.generate(pt, n, 0.0, 0, 1.0, None).cpu().numpy()
+    # the first generated token comes from the same prefill forward
+    np.testing.assert_array_equal(a[:, T0], full[:, T0])
+    first_diff = [next((t for t in range(T0, T0 + n) if a[r, t] != full[r, t]), T0 + n)
+                  for r in range(B)]
+    assert np.mean(first_diff) >= T0 + n / 2, first_diff
+    gm.close()
+
+
+def test_cached_generation_refuses_a_sliding_window(g):
+    import torch
+    _, _, gm = tiny(g, False)
+    pt = torch.zeros((1, 60), dtype=torch.int32, device="cuda")
+    with pytest.raises(g.GPT2Error):
+        gm.generate(pt, 10, 0.0, 0, 1.0, None, cached=True)  # 70 > context 64
+    gm.close()
