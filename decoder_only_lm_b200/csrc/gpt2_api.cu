@@ -87,6 +87,7 @@ struct gpt2_handle {
   void* kcache = nullptr;
   void* vcache = nullptr;
   int kv_T = 0;
+  int* gen_step = nullptr;  // device step counter of a replayed decoding step
   std::vector<float*> res;
   std::vector<void*> ln1, qkv, att, ln2, u, g;
   std::vector<float*> mu1, rs1, mu2, rs2, alse;
@@ -409,6 +410,7 @@ double gemm_flops(int64_t M, int64_t N, int64_t K) { return 2.0 * double(M) * do
 struct KvStep {
   int pos0;
   bool decode;
+  const int* d_step = nullptr;  // device offset added to pos0 (a replayed decoding step)
 };
 template <typename A>
 int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save,
@@ -425,7 +427,8 @@ int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save,
   {
     PROF(GPT2_PROF_EMBED, 0, 12.0 * M * C);
     H_TRY(h, launch_embed_fwd(h->xbuf, h->ybuf, P + h->off_wte, P + h->off_wpe, B, T, C, h->V,
-                              h->res[0], h->status, h->st, kv ? kv->pos0 : 0));
+                              h->res[0], h->status, h->st, kv ? kv->pos0 : 0,
+                              kv ? kv->d_step : nullptr));
   }
   const double ln_bytes = M * C * (4.0 + a) + 8.0 * M;
   const double attn_flops = 2.0 * B * Hh * double(T) * T * (C / Hh);
@@ -451,9 +454,10 @@ int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save,
       A* kc = static_cast<A*>(h->kcache) + l * per_layer;
       A* vc = static_cast<A*>(h->vcache) + l * per_layer;
       PROF(GPT2_PROF_ATTN_FWD, 0, a * 4.0 * M * C);
-      H_TRY(h, launch_kv_store<A>(qkv, B, T, C, Hh, kv->pos0, h->kv_T, kc, vc, h->st));
+      H_TRY(h, launch_kv_store<A>(qkv, B, T, C, Hh, kv->pos0, h->kv_T, kc, vc, h->st, kv->d_step));
       if (kv->decode)
-        H_TRY(h, launch_attn_decode<A>(qkv, kc, vc, B, C, Hh, h->kv_T, kv->pos0 + 1, att, h->st));
+        H_TRY(h, launch_attn_decode<A>(qkv, kc, vc, B, C, Hh, h->kv_T, kv->pos0 + 1, att, h->st,
+                                       kv->d_step));
     }
     if (!kv || !kv->decode) {
       PROF(GPT2_PROF_ATTN_FWD, attn_flops, a * 4.0 * M * C + 4.0 * M * Hh);
@@ -1102,23 +1106,84 @@ int gpt2_generate_cached(gpt2_handle* h, const int32_t* prompt, int B, int T0, i
   }
   H_CUDA(h, cudaMemcpy2DAsync(out, Ttot * sizeof(int32_t), prompt, T0 * sizeof(int32_t),
                               T0 * sizeof(int32_t), B, cudaMemcpyDeviceToDevice, h->st));
-  for (int s = 0; s < n_new; ++s) {
-    // step 0: the prompt at positions 0 .. T0-1 fills the cache; step s > 0:
-    // the token generated last, at position T0 + s - 1, attends to the cache
-    const int Tn = s == 0 ? T0 : 1;
-    const KvStep kv{s == 0 ? 0 : T0 + s - 1, s > 0};
-    const int32_t* src = s == 0 ? out : out + (T0 + s - 1);
-    H_CUDA(h, cudaMemcpy2DAsync(h->xbuf, Tn * sizeof(int32_t), src, Ttot * sizeof(int32_t),
-                                Tn * sizeof(int32_t), B, cudaMemcpyDeviceToDevice, h->st));
-    H_CUDA(h, cudaMemcpyAsync(h->ybuf, h->xbuf, size_t(B) * Tn * sizeof(int32_t),
+  if (n_new == 0) return check_status(h);
+  if (h->use_bf16 && h->mirror_dirty) H_TRY(h, launch_to_bf16(h->P, h->Pb, h->n_arena, h->st));
+  h->mirror_dirty = false;
+  // step 0: the prompt at positions 0 .. T0-1 fills the cache and gives token T0
+  {
+    const KvStep kv{0, false};
+    H_CUDA(h, cudaMemcpy2DAsync(h->xbuf, T0 * sizeof(int32_t), out, Ttot * sizeof(int32_t),
+                                T0 * sizeof(int32_t), B, cudaMemcpyDeviceToDevice, h->st));
+    H_CUDA(h, cudaMemcpyAsync(h->ybuf, h->xbuf, size_t(B) * T0 * sizeof(int32_t),
                               cudaMemcpyDeviceToDevice, h->st));
     if (h->use_bf16)
-      H_TRY(h, forward_t<bf16>(h, B, Tn, nullptr, false, h->gen_logits, h->Vp, &kv));
+      H_TRY(h, forward_t<bf16>(h, B, T0, nullptr, false, h->gen_logits, h->Vp, &kv));
     else
-      H_TRY(h, forward_t<float>(h, B, Tn, nullptr, false, h->gen_logits, h->Vp, &kv));
+      H_TRY(h, forward_t<float>(h, B, T0, nullptr, false, h->gen_logits, h->Vp, &kv));
     H_TRY(h, launch_sample(h->gen_logits, h->Vp, B, h->V, temperature, top_k, top_p,
-                           greedy ? nullptr : uniform + int64_t(s) * B, out + T0 + s, Ttot, h->st));
+                           greedy ? nullptr : uniform, out + T0, Ttot, h->st));
   }
+  if (n_new == 1) return check_status(h);
+  // Steps s = 1 .. n_new-1: the token at position T0+s-1 through the block,
+  // attending to the cache; s lives on the device (*gen_step) so that one
+  // recorded step serves every position.
+  if (!h->gen_step) {
+    h->gen_step = static_cast<int*>(dev_alloc(h, sizeof(int)));
+    if (!h->gen_step) return fail(h, GPT2_ERR_OOM, "generate_cached: step counter");
+  }
+  const int one = 1;
+  H_CUDA(h, cudaMemcpyAsync(h->gen_step, &one, sizeof(int), cudaMemcpyHostToDevice, h->st));
+  const KvStep kv{T0 - 1, true, h->gen_step};
+  auto step = [&]() -> int {
+    H_TRY(h, launch_gen_tokens(out, Ttot, B, T0 - 1, h->gen_step, h->xbuf, h->ybuf, h->st));
+    if (h->use_bf16)
+      H_TRY(h, forward_t<bf16>(h, B, 1, nullptr, false, h->gen_logits, h->Vp, &kv));
+    else
+      H_TRY(h, forward_t<float>(h, B, 1, nullptr, false, h->gen_logits, h->Vp, &kv));
+    H_TRY(h, launch_sample(h->gen_logits, h->Vp, B, h->V, temperature, top_k, top_p,
+                           greedy ? nullptr : uniform, out + T0, Ttot, h->st, h->gen_step,
+                           int64_t(B), 1));
+    H_TRY(h, launch_step_add(h->gen_step, h->st));
+    return GPT2_OK;
+  };
+  if (h->prof_on) {  // every kernel group timed on its own: no graph
+    for (int s = 1; s < n_new; ++s) H_TRY(h, step());
+    return check_status(h);
+  }
+  // record one step on a private stream (the handle's stream may be the legacy
+  // default stream, which cannot be captured), then replay it n_new-1 times
+  H_CUDA(h, cudaStreamSynchronize(h->st));
+  cudaStream_t user = h->st, cs = nullptr;
+  H_CUDA(h, cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
+  h->st = cs;
+  int rc = GPT2_OK;
+  cudaGraph_t g = nullptr;
+  cudaError_t ec = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+  if (ec == cudaSuccess) {
+    rc = step();
+    ec = cudaStreamEndCapture(cs, &g);
+  }
+  h->st = user;
+  cudaStreamDestroy(cs);
+  if (rc != GPT2_OK || ec != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    if (rc != GPT2_OK) return rc;
+    return fail(h, GPT2_ERR_CUDA, std::string("generate_cached: capture failed: ") +
+                                      cudaGetErrorString(ec));
+  }
+  cudaGraphExec_t ge = nullptr;
+  cudaError_t ei = cudaGraphInstantiate(&ge, g, 0);
+  cudaGraphDestroy(g);
+  if (ei != cudaSuccess)
+    return fail(h, GPT2_ERR_CUDA, std::string("generate_cached: graph instantiation failed: ") +
+                                      cudaGetErrorString(ei));
+  cudaError_t el = cudaSuccess;
+  for (int s = 1; s < n_new && el == cudaSuccess; ++s) el = cudaGraphLaunch(ge, h->st);
+  cudaError_t es = cudaStreamSynchronize(h->st);
+  cudaGraphExecDestroy(ge);
+  if (el != cudaSuccess || es != cudaSuccess)
+    return fail(h, GPT2_ERR_CUDA, std::string("generate_cached: replay failed: ") +
+                                      cudaGetErrorString(el != cudaSuccess ? el : es));
   return check_status(h);
 }
 

@@ -936,7 +936,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
 }
 
-// Split-K reduction, splits added in order:
+// Split-K reduction, splits added in order, then the GEMM's epilogue on the
+// sum (this kernel: every kind; the vectorised one below: EPI_STORE and
+// EPI_ACC):
 //   EPI_ACC:   out = (accumulate ? out : 0) + alpha * sum_z ws[z]      (fp32)
 //   EPI_STORE: out = alpha * sum_z ws[z] + bias[n]                    (OutT)
 template <typename OutT>
@@ -947,13 +949,7 @@ __global__ void tc_splitk_reduce_kernel(const float* __restrict__ ws, int splits
   const int m = int(i / N), n = int(i % N);
   float acc = 0.f;
   for (int z = 0; z < splits; ++z) acc += ws[int64_t(z) * M * N + i];
-  const int64_t o = int64_t(m) * e.ldo + n;
-  if (e.kind == EPI_ACC) {
-    float* out = reinterpret_cast<float*>(e.out);
-    out[o] = (e.accumulate ? out[o] : 0.f) + e.alpha * acc;
-  } else {
-    reinterpret_cast<OutT*>(e.out)[o] = from_f32<OutT>(e.alpha * acc + (e.bias ? e.bias[n] : 0.f));
-  }
+  epi_apply<OutT>(e, e.kind, m, n, acc);  // the GEMM's own epilogue on the summed value
 }
 
 // Same reduction, four columns per thread (N and ldo multiples of 4), rows
@@ -1149,7 +1145,9 @@ int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
   }
   COUNT_LAUNCH(1);
   if (p.splits > 1) {
-    const bool vec = (g.N % 4) == 0 && (g.ep.ldo % 4) == 0 && (!g.ep.bias || (reinterpret_cast<uintptr_t>(g.ep.bias) & 15) == 0);
+    const bool vec = (g.ep.kind == EPI_STORE || g.ep.kind == EPI_ACC) && (g.N % 4) == 0 &&
+                     (g.ep.ldo % 4) == 0 &&
+                     (!g.ep.bias || (reinterpret_cast<uintptr_t>(g.ep.bias) & 15) == 0);
     if (vec) {
       const dim3 grid(cdiv(g.N / 4, 128), std::min(g.M, 2048));
       tc_splitk_reduce4_kernel<OutT><<<grid, 128, 0, st>>>(g.ws, p.splits, g.M, g.N, g.ep);
@@ -1242,7 +1240,10 @@ size_t gemm_tc_workspace_bytes(int M, int N, int K) {
 }
 
 int gemm_tc_launch(const GemmArgs& g, cudaStream_t st) {
-  const bool splittable = (g.ep.kind == EPI_ACC || g.ep.kind == EPI_STORE) && g.ws;
+  // split-K needs the workspace; its reduction applies any epilogue but the
+  // LM-head ones (the cost model splits only when the output tiles leave most
+  // CTA pairs idle, e.g. the one-row GEMMs of incremental decoding)
+  const bool splittable = g.ep.kind != EPI_LSE_PARTIAL && g.ep.kind != EPI_CE_GRAD && g.ws;
   const int sp = choose_splits_tc(g.M, g.N, g.K, splittable, splittable ? g.ws_bytes : 0);
   return dispatch_epi<256>(g, sp, st);
 }

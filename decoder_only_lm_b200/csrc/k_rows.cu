@@ -60,7 +60,7 @@ __global__ void slice_batch_kernel(const uint16_t* __restrict__ s, int64_t off, 
 __global__ void embed_fwd_kernel(const int32_t* __restrict__ x, const int32_t* __restrict__ y,
                                  const float* __restrict__ wte, const float* __restrict__ wpe,
                                  int T, int C, int V, int64_t M, float* __restrict__ out,
-                                 DevStatus* status, int pos0) {
+                                 DevStatus* status, int pos0, const int* __restrict__ d_step) {
   int64_t m = blockIdx.x;
   if (m >= M) return;
   int id = x[m];
@@ -69,7 +69,7 @@ __global__ void embed_fwd_kernel(const int32_t* __restrict__ x, const int32_t* _
     if (id < 0 || id >= V || yy < 0 || yy >= V) atomicExch(&status->token_bad, 1);
   }
   if (id < 0 || id >= V) id = 0;
-  const int t = pos0 + int(m % T);
+  const int t = pos0 + (d_step ? *d_step : 0) + int(m % T);
   const float* a = wte + int64_t(id) * C;
   const float* b = wpe + int64_t(t) * C;
   float* o = out + m * C;
@@ -853,9 +853,9 @@ int launch_slice_batch(const uint16_t* s, int64_t off, int64_t n, int32_t* x, in
 
 int launch_embed_fwd(const int32_t* x, const int32_t* y, const float* wte, const float* wpe, int B,
                      int T, int C, int V, float* out, DevStatus* status, cudaStream_t st,
-                     int pos0) {
+                     int pos0, const int* d_step) {
   const int64_t M = int64_t(B) * T;
-  embed_fwd_kernel<<<int(M), 192, 0, st>>>(x, y, wte, wpe, T, C, V, M, out, status, pos0);
+  embed_fwd_kernel<<<int(M), 192, 0, st>>>(x, y, wte, wpe, T, C, V, M, out, status, pos0, d_step);
   COUNT_LAUNCH(1);
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;

@@ -72,8 +72,12 @@ __device__ __forceinline__ uint64_t weight(float p) {
 __global__ void __launch_bounds__(kSampleThreads) sample_kernel(
     const float* __restrict__ logits, int64_t ld, int V, float temperature, int top_k,
     float top_p, const float* __restrict__ uniform, int32_t* __restrict__ out,
-    int64_t out_stride) {
+    int64_t out_stride, const int* __restrict__ d_step, int64_t u_step, int64_t out_step) {
   extern __shared__ float ps[];  // V values of this row
+  if (d_step) {
+    if (uniform) uniform += int64_t(*d_step) * u_step;
+    out += int64_t(*d_step) * out_step;
+  }
   __shared__ uint64_t sh_u[kSampleWarps + 1];
   __shared__ int sh_i[kSampleWarps + 1];
   __shared__ uint64_t warp_base[kSampleWarps];
@@ -212,7 +216,7 @@ size_t sample_max_vocab() { return kSampleMaxVocab; }
 
 int launch_sample(const float* logits, int64_t ld, int B, int V, float temperature, int top_k,
                   float top_p, const float* uniform, int32_t* out, int64_t out_stride,
-                  cudaStream_t st) {
+                  cudaStream_t st, const int* d_step, int64_t u_step, int64_t out_step) {
   if (B < 1 || V < 1 || V > kSampleMaxVocab) {
     gpt2_internal::set_error("sample: V outside 1..53248");
     return GPT2_ERR_ARG;
@@ -228,7 +232,8 @@ int launch_sample(const float* logits, int64_t ld, int B, int V, float temperatu
     attr_set = true;
   }
   sample_kernel<<<B, kSampleThreads, size_t(V) * sizeof(float), st>>>(
-      logits, ld, V, temperature, top_k, top_p, uniform, out, out_stride);
+      logits, ld, V, temperature, top_k, top_p, uniform, out, out_stride, d_step, u_step,
+      out_step);
   COUNT_LAUNCH(1);
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;

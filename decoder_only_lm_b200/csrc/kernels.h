@@ -58,10 +58,11 @@ int launch_slice_batch(const uint16_t* s, int64_t off, int64_t n, int32_t* x, in
 int launch_slice_batch_cursor(const uint16_t* s, int64_t len, const int64_t* cur, int64_t n,
                               int32_t* x, int32_t* y, DevStatus* status, cudaStream_t st);
 int launch_advance_cursor(int64_t* cur, int64_t stride, cudaStream_t st);
-// positions pos0 .. pos0 + T - 1 (pos0 > 0: one step of incremental decoding)
+// positions p0 .. p0 + T - 1 with p0 = pos0 + (*d_step when d_step is given:
+// a step of incremental decoding replayed from a graph)
 int launch_embed_fwd(const int32_t* x, const int32_t* y, const float* wte, const float* wpe,
                      int B, int T, int C, int V, float* out, DevStatus* status, cudaStream_t st,
-                     int pos0 = 0);
+                     int pos0 = 0, const int* d_step = nullptr);
 // dwte[x_m] += dh[m] (deterministic: sort by id, segmented sums); dwpe[t] (+)= sum_b dh[b,t].
 size_t embed_bwd_workspace(int64_t M, int C);
 int launch_embed_bwd(const int32_t* x, const float* dh, int B, int T, int C, int V, float* dwte,
@@ -100,15 +101,22 @@ int launch_ce_rows_bwd(const float* z, const float* lse, const int32_t* y, int r
 int launch_mean(const float* v, int64_t n, float* out, cudaStream_t st);
 
 // ---------------------------------------------------------------- KV-cache decoding
-// K, V caches per layer: [B, H, Tc, D] of the activation type.
+// K, V caches per layer: [B, H, Tc, D] of the activation type.  With d_step
+// the position (and the attention length) is offset by *d_step on the device,
+// so one recorded decoding step can be replayed for every position.
 template <typename T>
 int launch_kv_store(const T* qkv, int B, int Tn, int C, int H, int pos0, int Tc, T* kc, T* vc,
-                    cudaStream_t st);
+                    cudaStream_t st, const int* d_step = nullptr);
 // out[b, h*D .. ] = attention of the single query row b of qkv [B, 3C] over
-// cache positions 0 .. L-1 (L <= Tc, L <= 4096, D <= 128 dividing 128)
+// cache positions 0 .. L-1 (L <= Tc, L <= 4096; a head row of D elements is
+// G = D * sizeof(T) / 16 sixteen-byte vectors, G dividing 32)
 template <typename T>
 int launch_attn_decode(const T* qkv, const T* kc, const T* vc, int B, int C, int H, int Tc, int L,
-                       T* out, cudaStream_t st);
+                       T* out, cudaStream_t st, const int* d_step = nullptr);
+// x[b] = y[b] = tokens[b * ld + col0 + *d_step] (the token a replayed decoding step reads)
+int launch_gen_tokens(const int32_t* tokens, int64_t ld, int B, int64_t col0, const int* d_step,
+                      int32_t* x, int32_t* y, cudaStream_t st);
+int launch_step_add(int* d_step, cudaStream_t st);  // *d_step += 1
 
 // ---------------------------------------------------------------- sampling
 // next token of each of B rows of fp32 logits (row stride ld, first V columns):
@@ -117,9 +125,11 @@ int launch_attn_decode(const T* qkv, const T* kc, const T* vc, int B, int C, int
 // shared memory, ids in 16 bits).
 constexpr int kSampleMaxVocab = 53248;
 size_t sample_max_vocab();
+// With d_step: uniform + *d_step * u_step and out + *d_step * out_step.
 int launch_sample(const float* logits, int64_t ld, int B, int V, float temperature, int top_k,
                   float top_p, const float* uniform, int32_t* out, int64_t out_stride,
-                  cudaStream_t st);
+                  cudaStream_t st, const int* d_step = nullptr, int64_t u_step = 0,
+                  int64_t out_step = 0);
 
 // ---------------------------------------------------------------- attention
 template <typename T>
