@@ -149,7 +149,8 @@ def test_lmhead_ce_full_size_sampled_rows(g):
 
 
 @pytest.mark.parametrize("ak,bk", [(1, 1), (1, 0), (0, 1), (0, 0)])
-@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 200, 136), (1024, 768, 768)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 200, 136), (1024, 768, 768), (16, 520, 256),
+                                   (3, 50304, 768)])
 @pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
 def test_matmul_layouts(g, ak, bk, M, N, K, bf16):
     import torch
@@ -171,7 +172,8 @@ def test_matmul_layouts(g, ak, bk, M, N, K, bf16):
 
 
 @pytest.mark.parametrize("epi", ["bias", "bias_gelu", "residual", "gelu_bwd"])
-@pytest.mark.parametrize("M,N,K", [(300, 520, 136), (1, 64, 64), (2050, 768, 3072)])
+@pytest.mark.parametrize("M,N,K", [(300, 520, 136), (1, 64, 64), (2050, 768, 3072), (4, 2304, 768),
+                                   (3, 384, 3072), (16, 384, 3072)])
 @pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
 def test_linear_epilogues(g, epi, M, N, K, bf16):
     """The fused linear layer against the oracle: the contraction in fp64 from
