@@ -63,13 +63,45 @@ __device__ __forceinline__ T block_reduce(T v, T* sh, Op op) {
   return r;
 }
 
+// Two sums in one pass (same fixed order as block_reduce).
+__device__ __forceinline__ void block_sum2(uint64_t& a, uint64_t& c, uint64_t* sh_a,
+                                           uint64_t* sh_c) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+  }
+  if (lane == 0) {
+    sh_a[warp] = a;
+    sh_c[warp] = c;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint64_t x = sh_a[lane], y = sh_c[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      x += __shfl_xor_sync(0xffffffffu, x, o);
+      y += __shfl_xor_sync(0xffffffffu, y, o);
+    }
+    if (lane == 0) {
+      sh_a[kSampleWarps] = x;
+      sh_c[kSampleWarps] = y;
+    }
+  }
+  __syncthreads();
+  a = sh_a[kSampleWarps];
+  c = sh_c[kSampleWarps];
+  __syncthreads();
+}
+
 constexpr double kWeightScale = 68719476736.0;  // 2^36
 
 __device__ __forceinline__ uint64_t weight(float p) {
   return uint64_t(__double2ll_rn(double(p) * kWeightScale));
 }
 
-__global__ void __launch_bounds__(kSampleThreads) sample_kernel(
+__global__ void __launch_bounds__(kSampleThreads, 1) sample_kernel(
     const float* __restrict__ logits, int64_t ld, int V, float temperature, int top_k,
     float top_p, const float* __restrict__ uniform, int32_t* __restrict__ out,
     int64_t out_stride, const int* __restrict__ d_step, int64_t u_step, int64_t out_step) {
@@ -79,6 +111,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(
     out += int64_t(*d_step) * out_step;
   }
   __shared__ uint64_t sh_u[kSampleWarps + 1];
+  __shared__ uint64_t sh_c[kSampleWarps + 1];
   __shared__ int sh_i[kSampleWarps + 1];
   __shared__ uint64_t warp_base[kSampleWarps];
   const int b = blockIdx.x, tid = threadIdx.x;
@@ -131,9 +164,15 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(
           part += by_weight ? weight(p) : 1;
         }
       }
-      if (double(block_reduce(part, sh_u, uadd)) >= goal) {
+      // ids in play at or above mid (high half) and below it (low half)
+      const int n_ge = __popcll(static_cast<long long>(ge));
+      uint64_t counts = (uint64_t(n_ge) << 32) | uint64_t(__popcll(static_cast<long long>(play)) - n_ge);
+      block_sum2(part, counts, sh_u, sh_c);
+      uint64_t left;  // ids still in play after this step
+      if (double(part) >= goal) {
         lo = mid;
         play = ge;  // keys below mid leave
+        left = counts >> 32;
       } else {
         hi = mid;  // keys at or above mid are always counted from now on
         for (uint64_t m = ge; m; m &= m - 1) {
@@ -141,6 +180,18 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(
           above += by_weight ? weight(ps[tid + j * kSampleThreads]) : 1;
         }
         play &= ~ge;
+        left = counts & 0xFFFFFFFFu;
+      }
+      if (left == 1) {
+        // f(lo) >= goal > f(hi) and f changes only at the one key left in
+        // [lo, hi): that key is the answer
+        uint64_t k = 0;
+        if (play) {
+          const int j = __ffsll(static_cast<long long>(play)) - 1;
+          k = prob_key(ps[tid + j * kSampleThreads], tid + j * kSampleThreads);
+        }
+        lo = block_reduce(k, sh_u, umax);
+        break;
       }
     }
     return lo;
