@@ -96,3 +96,43 @@ def test_padding_columns_are_never_drawn():
     z[0, 12:] = 50.0  # huge logits in the padding columns 12..15
     ids = draws(z[0], 12, 1.0, 0, 1.0, 300)
     assert ids.max() < 12
+
+
+def test_edge_cases():
+    """One-token vocabulary; all logits equal (the tie order decides the
+    nucleus); a tiny top-p keeps only the most probable token; u at the ends."""
+    z1 = np.array([[3.0]], np.float32)
+    for T, k, p in ((0.0, 0, 1.0), (1.0, 0, 0.5), (0.7, 5, 1.0)):
+        assert oracle.sample(z1, 1, T, k, p, [0.99])[0] == 0
+    V = 10
+    flat = np.zeros((1, V), np.float32)
+    # equal probabilities: ids enter the order smallest first, so top-p = 0.25
+    # keeps ids 0, 1, 2 (3 x 0.1 >= 0.25) and the draw is uniform over them
+    ids = draws(flat[0], V, 1.0, 0, 0.25, 3000)
+    assert set(np.unique(ids).tolist()) == {0, 1, 2}
+    np.testing.assert_allclose(np.bincount(ids, minlength=3)[:3] / 3000, [1 / 3] * 3, atol=2e-3)
+    # top-k on equal logits keeps the k smallest ids
+    assert set(np.unique(draws(flat[0], V, 1.0, 4, 1.0, 2000)).tolist()) == {0, 1, 2, 3}
+    rng = np.random.default_rng(4)
+    z = rng.normal(size=(3, 200)).astype(np.float32)
+    np.testing.assert_array_equal(oracle.sample(z, 200, 1.0, 0, 1e-6, [0.5, 0.9, 0.0]),
+                                  np.argmax(z, axis=1))
+    # u = 0 gives the smallest kept id, u just below 1 the largest
+    lo = oracle.sample(z, 200, 1.0, 10, 1.0, np.zeros(3))
+    hi = oracle.sample(z, 200, 1.0, 10, 1.0, np.full(3, np.nextafter(np.float32(1), np.float32(0))))
+    top10 = np.argsort(-z, axis=1)[:, :10]
+    np.testing.assert_array_equal(lo, top10.min(axis=1))
+    np.testing.assert_array_equal(hi, top10.max(axis=1))
+
+
+def test_weights_are_exact_integers():
+    """The weights of the draw are rint(p * 2^36): their sum is exact in
+    float64 for any vocabulary up to 2^16 ids, so cumulative comparisons do not
+    depend on the order of summation."""
+    rng = np.random.default_rng(5)
+    z = (rng.normal(size=50257) * 4).astype(np.float32)
+    p = np.exp(z - z.max()).astype(np.float32)
+    w = np.rint(p.astype(np.float64) * oracle.SAMPLE_WEIGHT_SCALE).astype(np.int64)
+    assert w.max() == 2 ** 36 and w.sum() < 2 ** 53
+    perm = rng.permutation(w.size)
+    assert float(np.cumsum(w)[-1]) == float(np.cumsum(w[perm])[-1])
