@@ -249,13 +249,14 @@ int gpt2_logits_last(gpt2_handle* h, const int32_t* x, int B, int T, int tokens_
  * temperature and top-p; LECTURE: top-k]:
  *   temperature == 0 or top_k == 1: the highest logit (the smaller id on ties);
  *   otherwise p_i = exp((z_i - max z) / temperature) in fp32 over the first V
- *   columns (the real vocabulary: padding columns are never drawn); ids are
- *   ordered by p, the smaller id first among equal p; top_k > 0 keeps the
- *   first top_k of that order; top_p < 1 keeps its shortest prefix whose mass
- *   reaches top_p times the kept mass (the crossing id included); the draw
- *   walks the kept ids in increasing id order, summing p in fp64, and returns
- *   the first id at which the sum exceeds uniform[b] * (kept mass) (the last
- *   kept id if rounding leaves the target unreached).
+ *   columns (the real vocabulary: padding columns are never drawn) and the
+ *   weight of id i is the integer w_i = rint(p_i * 2^36), so every cumulative
+ *   probability below is an exact integer sum; ids are ordered by p, the
+ *   smaller id first among equal p; top_k > 0 keeps the first top_k of that
+ *   order; top_p < 1 keeps its shortest prefix whose weight reaches top_p
+ *   times the kept weight (the crossing id included); the draw walks the kept
+ *   ids in increasing id order and returns the first id at which the running
+ *   weight exceeds uniform[b] * (kept weight) (the last kept id if none does).
  * logits: device fp32, row b at logits + b*ld (ld >= V).  uniform: device fp32
  * [B] in [0, 1) (values outside are clamped; may be NULL for greedy choices).
  * out: device int32, out[b*out_stride].  Deterministic.  GPT2_ERR_ARG unless
