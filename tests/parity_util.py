@@ -50,12 +50,16 @@ def gpu_model(s: Shape, bf16: bool, max_B=None, max_Tseq=None):
 
 
 def inputs(s: Shape, seed=0, stream_seed=1, uniform=True):
+    """Seeded weights and a B*T+1 token stream cut into x, y.  uniform=False
+    draws the web-text stand-in instead: Zipf(1.1) ids with the last id of the
+    vocabulary as the end-of-text separator before every document (id 0 is
+    then about 14% of the tokens at V = 50257, more at small V)."""
     om = oracle_model(s)
     named = synth.init_params(seed, om.shapes())
     n = s.B * s.T + 1
     if uniform:
         stream = synth.uniform_stream(stream_seed, n, s.vocab_size)
     else:
-        stream = synth.token_stream(stream_seed, n)
+        stream = synth.token_stream(stream_seed, n, eot=s.vocab_size - 1)
     x, y = oracle.batch_from_stream(stream, 0, s.B, s.T)
     return om, named, stream, x, y
