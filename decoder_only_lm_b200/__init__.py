@@ -26,6 +26,7 @@ F32, BF16 = 0, 1
 
 ALLOC_FN = C.CFUNCTYPE(C.c_void_p, C.c_size_t, C.c_void_p)
 FREE_FN = C.CFUNCTYPE(None, C.c_void_p, C.c_void_p)
+BUCKET_FN = C.CFUNCTYPE(None, C.c_void_p, C.c_int)
 
 
 class Config(C.Structure):
@@ -69,6 +70,11 @@ SIGNATURES = {
     "gpt2_stream_end": (_i, [_P, C.POINTER(_i64)]),
     "gpt2_synchronize": (_i, [_P]),
     "gpt2_arena": (_i, [_P, _i, C.POINTER(C.POINTER(_f)), C.POINTER(_i64)]),
+    "gpt2_arena_layout": (_i, [C.POINTER(Config), _i, C.c_char_p, _i, C.POINTER(_i64),
+                               C.POINTER(_i64), C.POINTER(_i)]),
+    "gpt2_grad_buckets": (_i, [C.POINTER(Config), _i, C.POINTER(_i), C.POINTER(_i64),
+                               C.POINTER(_i64), C.POINTER(_i)]),
+    "gpt2_set_bucket_callback": (_i, [_P, BUCKET_FN, _P]),
     "gpt2_profile_enable": (_i, [_P, _i]),
     "gpt2_profile_reset": (_i, [_P]),
     "gpt2_profile_read": (_i, [_P, _i, C.POINTER(_i64), C.POINTER(C.c_double), C.POINTER(C.c_double),
@@ -132,6 +138,38 @@ def _stream_ptr(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream
+
+
+def make_config(n_layer, n_embd, n_head, vocab_size, padded_vocab=None, max_T=1024, bf16=True,
+                max_B=1, max_Tseq=None, ln_eps=1e-5):
+    """A gpt2_config without stream or allocator (for the host-only calls)."""
+    return Config(n_layer, n_embd, n_head, vocab_size, padded_vocab or vocab_size, max_T,
+                  1 if bf16 else 0, ln_eps, max_B, max_Tseq or max_T, 0, None, ALLOC_FN(),
+                  FREE_FN(), None)
+
+
+def arena_layout(cfg):
+    """[(name, offset, n_elems)] of every tensor in the arenas (gpt2_arena_layout;
+    host only)."""
+    n = C.c_int()
+    _check(lib.gpt2_arena_layout(C.byref(cfg), -1, None, 0, None, None, C.byref(n)))
+    out = []
+    buf = C.create_string_buffer(128)
+    for i in range(n.value):
+        off, cnt = C.c_int64(), C.c_int64()
+        _check(lib.gpt2_arena_layout(C.byref(cfg), i, buf, 128, C.byref(off), C.byref(cnt), None))
+        out.append((buf.value.decode(), off.value, cnt.value))
+    return out
+
+
+def grad_buckets(cfg):
+    """[(bucket, offset, count)] of the gradient arena in the order the
+    backward finishes the buckets (gpt2_grad_buckets; host only)."""
+    n = C.c_int()
+    _check(lib.gpt2_grad_buckets(C.byref(cfg), 0, C.byref(n), None, None, None))
+    off, cnt, b = (C.c_int64 * n.value)(), (C.c_int64 * n.value)(), (C.c_int * n.value)()
+    _check(lib.gpt2_grad_buckets(C.byref(cfg), n.value, C.byref(n), off, cnt, b))
+    return [(b[k], off[k], cnt[k]) for k in range(n.value)]
 
 
 class GPT2:
@@ -334,6 +372,16 @@ class GPT2:
             __cuda_array_interface__ = {"shape": (n.value,), "typestr": "<f4",
                                         "data": (addr, False), "version": 2}
         return self.torch.as_tensor(_View(), device="cuda")
+
+    def set_bucket_callback(self, fn):
+        """gpt2_set_bucket_callback: fn(bucket) is called as the backward makes
+        each gradient bucket final (None clears it)."""
+        if fn is None:
+            self._bucket_cb = None
+            _check(lib.gpt2_set_bucket_callback(self.h, BUCKET_FN(), None), self.h)
+            return
+        self._bucket_cb = BUCKET_FN(lambda user, b: fn(b))
+        _check(lib.gpt2_set_bucket_callback(self.h, self._bucket_cb, None), self.h)
 
     def profile(self, enable=True):
         _check(lib.gpt2_profile_enable(self.h, int(enable)), self.h)

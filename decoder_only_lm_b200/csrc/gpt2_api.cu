@@ -105,7 +105,7 @@ struct gpt2_handle {
   // side stream: weight-gradient GEMMs overlap the input-gradient GEMMs they
   // are independent of (own workspace; joined back before anything else runs)
   cudaStream_t st2 = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_join2 = nullptr;
   float* ws2 = nullptr;
   void* ws_emb = nullptr;
   double* ws_norm = nullptr;
@@ -129,6 +129,11 @@ struct gpt2_handle {
     std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending;
   };
   bool prof_on = false;
+  // data-parallel exchange: called as each gradient bucket becomes final in a
+  // backward issued call by call (never while a step is being captured)
+  gpt2_bucket_fn bucket_fn = nullptr;
+  void* bucket_user = nullptr;
+  bool capturing = false;
   Cat cats[GPT2_PROF_NCAT];
   std::vector<cudaEvent_t> ev_pool;
   int64_t launches_total = 0;
@@ -238,6 +243,32 @@ void free_all(gpt2_handle* h) {
       cudaFree(p);
   }
   h->allocs.clear();
+}
+
+// Empty string when cfg is a valid configuration, else why not.
+std::string config_problem(const gpt2_config& c) {
+  if (c.n_layer < 1 || c.n_embd < 8 || c.n_head < 1 || c.n_embd % c.n_head || c.n_embd % 8 ||
+      c.vocab_size < 1 || c.padded_vocab < c.vocab_size || c.padded_vocab % 8 || c.max_T < 1 ||
+      c.max_B < 1 || c.max_Tseq < 1 || c.max_Tseq > c.max_T || !(c.ln_eps > 0.f) ||
+      c.n_embd > 1024 || c.resid_init_scale != 0 || (c.alloc && !c.free))
+    return "invalid gpt2_config";
+  const int D = c.n_embd / c.n_head;
+  if (D != 16 && D != 32 && D != 64) return "head size must be 16, 32 or 64";
+  if (int64_t(c.max_B) * c.max_Tseq > (int64_t(1) << 26)) return "max_B * max_Tseq too large";
+  return "";
+}
+
+void set_shape(gpt2_handle* h, const gpt2_config& c) {
+  h->cfg = c;
+  h->L = c.n_layer;
+  h->C = c.n_embd;
+  h->H = c.n_head;
+  h->V = c.vocab_size;
+  h->Vp = c.padded_vocab;
+  h->Tmax = c.max_T;
+  h->F = 4 * c.n_embd;
+  h->use_bf16 = c.bf16 ? 1 : 0;
+  h->Mcap = int64_t(c.max_B) * c.max_Tseq;
 }
 
 void build_layout(gpt2_handle* h) {
@@ -529,6 +560,12 @@ int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save,
 }
 
 // ------------------------------------------------------------------ backward
+// Tells the caller (data-parallel exchange) that bucket b of the gradient
+// arena is final once the work enqueued so far on the handle's stream is done.
+void bucket_ready(gpt2_handle* h, int b) {
+  if (h->bucket_fn && !h->capturing) h->bucket_fn(h->bucket_user, b);
+}
+
 template <typename A>
 int backward_t(gpt2_handle* h, float grad_scale) {
   const int B = h->fB, T = h->fT;
@@ -553,7 +590,8 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     if (!h->prof_on) {
       side.st = h->st2;
       side.e_fork = h->ev_fork;
-      side.e_join = h->ev_join;
+      side.e_join[0] = h->ev_join;
+      side.e_join[1] = h->ev_join2;
       side.ws = h->ws2;
       side.ws_bytes = h->ws_bytes;
     }
@@ -657,6 +695,8 @@ int backward_t(gpt2_handle* h, float grad_scale) {
                                             l > 0 ? G + h->lo[l - 1].fpb : nullptr, acc, h->ws,
                                             h->st)));
     }
+    // layer l's weight matrices are final on st (every side-stream writer joined)
+    bucket_ready(h, h->L - 1 - l);
   }
   {
     // embedding: both uses of the tied matrix add into one gradient [LECTURE]
@@ -664,6 +704,7 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     H_TRY(h, launch_embed_bwd(h->xbuf, h->dres, B, T, C, h->V, G + h->off_wte, G + h->off_wpe,
                               acc, h->ws_emb, h->st));
   }
+  bucket_ready(h, h->L);  // wte, wpe and every vector
   h->grads_zero = false;
   return GPT2_OK;
 }
@@ -691,28 +732,11 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
   *out = nullptr;
   if (!cfg) return fail(nullptr, GPT2_ERR_ARG, "cfg is NULL");
   const gpt2_config& c = *cfg;
-  if (c.n_layer < 1 || c.n_embd < 8 || c.n_head < 1 || c.n_embd % c.n_head || c.n_embd % 8 ||
-      c.vocab_size < 1 || c.padded_vocab < c.vocab_size || c.padded_vocab % 8 || c.max_T < 1 ||
-      c.max_B < 1 || c.max_Tseq < 1 || c.max_Tseq > c.max_T || !(c.ln_eps > 0.f) ||
-      c.n_embd > 1024 || c.resid_init_scale != 0 || (c.alloc && !c.free))
-    return fail(nullptr, GPT2_ERR_ARG, "invalid gpt2_config");
-  const int D = c.n_embd / c.n_head;
-  if (D != 16 && D != 32 && D != 64)
-    return fail(nullptr, GPT2_ERR_ARG, "head size must be 16, 32 or 64");
-  if (int64_t(c.max_B) * c.max_Tseq > (int64_t(1) << 26))
-    return fail(nullptr, GPT2_ERR_ARG, "max_B * max_Tseq too large");
+  const std::string bad = config_problem(c);
+  if (!bad.empty()) return fail(nullptr, GPT2_ERR_ARG, bad);
   gpt2_handle* h = new gpt2_handle();
-  h->cfg = c;
+  set_shape(h, c);
   h->st = static_cast<cudaStream_t>(c.stream);
-  h->L = c.n_layer;
-  h->C = c.n_embd;
-  h->H = c.n_head;
-  h->V = c.vocab_size;
-  h->Vp = c.padded_vocab;
-  h->Tmax = c.max_T;
-  h->F = 4 * c.n_embd;
-  h->use_bf16 = c.bf16 ? 1 : 0;
-  h->Mcap = int64_t(c.max_B) * c.max_Tseq;
   build_layout(h);
 
   const int64_t M = h->Mcap, C = h->C, F = h->F, L = h->L, Vp = h->Vp;
@@ -789,8 +813,10 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
   }
   if (cudaStreamCreateWithFlags(&h->st2, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&h->ev_join2, cudaEventDisableTiming) != cudaSuccess) {
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
     if (h->st2) cudaStreamDestroy(h->st2);
     free_all(h);
     delete h;
@@ -823,6 +849,7 @@ int gpt2_destroy(gpt2_handle* h) {
   }
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->ev_join2) cudaEventDestroy(h->ev_join2);
   prof_collect(h);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   free_all(h);
@@ -1255,8 +1282,10 @@ int gpt2_stream_begin(gpt2_handle* h, const uint16_t* d_stream, int64_t stream_l
   cudaGraph_t g = nullptr;
   cudaError_t ec = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
   if (ec == cudaSuccess) {
+    h->capturing = true;
     rc = stream_step_body(h, d_stream, stream_len, stride, B, T, accum, beta1, beta2, eps,
                           weight_decay, max_norm);
+    h->capturing = false;
     ec = cudaStreamEndCapture(cs, &g);
   }
   h->st = user;
@@ -1295,6 +1324,68 @@ int gpt2_stream_end(gpt2_handle* h, int64_t* cursor_out) {
   h->graph_exec = nullptr;
   h->graph = nullptr;
   return check_status(h);
+}
+
+int gpt2_arena_layout(const gpt2_config* cfg, int i, char* name, int name_len, int64_t* offset,
+                      int64_t* n_elems, int* n_tensors) {
+  if (!cfg) return fail(nullptr, GPT2_ERR_ARG, "cfg is NULL");
+  const std::string bad = config_problem(*cfg);
+  if (!bad.empty()) return fail(nullptr, GPT2_ERR_ARG, bad);
+  gpt2_handle t;  // host-side layout only: nothing is allocated
+  set_shape(&t, *cfg);
+  build_layout(&t);
+  if (n_tensors) *n_tensors = int(t.tensors.size());
+  if (i < 0) return GPT2_OK;
+  if (i >= int(t.tensors.size())) return fail(nullptr, GPT2_ERR_ARG, "tensor index out of range");
+  const TensorInfo& x = t.tensors[i];
+  if (name && name_len > 0) {
+    const size_t n = std::min(size_t(name_len - 1), x.name.size());
+    memcpy(name, x.name.data(), n);
+    name[n] = 0;
+  }
+  if (offset) *offset = x.off;
+  if (n_elems) *n_elems = x.rows * x.cols;
+  return GPT2_OK;
+}
+
+int gpt2_grad_buckets(const gpt2_config* cfg, int max_ranges, int* n_ranges, int64_t* offset,
+                      int64_t* count, int* bucket) {
+  if (!cfg || !n_ranges) return fail(nullptr, GPT2_ERR_ARG, "NULL argument");
+  const std::string bad = config_problem(*cfg);
+  if (!bad.empty()) return fail(nullptr, GPT2_ERR_ARG, bad);
+  gpt2_handle t;
+  set_shape(&t, *cfg);
+  build_layout(&t);
+  struct R {
+    int64_t off, n;
+    int b;
+  };
+  std::vector<R> r;
+  // bucket L-1-l: the four matrices of layer l, one contiguous range of the
+  // 2-D part of the arena (qkv, proj, fc, fc-proj in that order)
+  for (int l = t.L - 1; l >= 0; --l) {
+    const TensorInfo* q = &t.tensors[2 + 12 * l];
+    const int64_t a = q[2].off, e = q[10].off + align_up(q[10].rows * q[10].cols, kAlign);
+    r.push_back({a, e - a, t.L - 1 - l});
+  }
+  // bucket L: wte and wpe (the arena's first range) and every vector (its last)
+  r.push_back({0, t.tensors[2 + 2].off, t.L});
+  r.push_back({t.n_decay, t.n_arena - t.n_decay, t.L});
+  *n_ranges = int(r.size());
+  if (max_ranges < int(r.size())) return GPT2_OK;  // the count only
+  for (size_t k = 0; k < r.size(); ++k) {
+    if (offset) offset[k] = r[k].off;
+    if (count) count[k] = r[k].n;
+    if (bucket) bucket[k] = r[k].b;
+  }
+  return GPT2_OK;
+}
+
+int gpt2_set_bucket_callback(gpt2_handle* h, gpt2_bucket_fn fn, void* user) {
+  if (!h) return GPT2_ERR_ARG;
+  h->bucket_fn = fn;
+  h->bucket_user = user;
+  return GPT2_OK;
 }
 
 int gpt2_arena(gpt2_handle* h, int which, float** ptr, int64_t* n_elems) {

@@ -9,12 +9,15 @@
 //            the target logit; a merge kernel combines the partials of a row in
 //            order: lse = M + log sum_t s_t exp(m_t - M), loss = lse - z_y.
 //            No logit is ever written to memory.
-//   backward per chunk of <= 16384 rows: the recomputed logits go straight
+//   backward per chunk of kChunkBf16 rows: the recomputed logits go straight
 //            from TMEM through dz = scale (exp(z - lse) - onehot) to a bf16
-//            chunk buffer (1.6 GB at Vp = 50304), then dh = dz W and
-//            dW (+)= dz^T h.  Large chunks keep the weight-gradient GEMM long
-//            in K instead of re-accumulating the fp32 [Vp, C] gradient once
-//            per chunk.
+//            chunk buffer, then dh[chunk] = dz W (K = Vp, split along K) and
+//            dW (+)= dz^T h[chunk] (fp32, one add per element and chunk, in
+//            chunk order).  kRingBf16 chunk buffers: with a side stream the
+//            next chunk's logits are recomputed while the previous chunk's
+//            weight gradient still reads its buffer.  The live part of dz is
+//            kRingBf16 x kChunkBf16 x Vp bf16 (206 MB at Vp = 50304), whatever
+//            the number of rows.
 // fp32 path (parity mode, CUDA cores): per chunk of <= 2048 rows, logits in an
 // fp32 chunk buffer, a row kernel for lse / loss / dz, then the same two
 // contractions.
@@ -25,10 +28,11 @@
 
 namespace {
 
-constexpr int kChunkBf16 = 16384, kChunkF32 = 2048;
+constexpr int kChunkBf16 = 1024, kRingBf16 = 2, kChunkF32 = 2048;
 constexpr int kTileN = 256;  // column tile of the LSE-partial tensor-core GEMM
 
 int chunk_rows(int bf16) { return bf16 ? kChunkBf16 : kChunkF32; }
+int ring(int bf16) { return bf16 ? kRingBf16 : 1; }
 
 size_t r256(size_t b) { return (b + 255) / 256 * 256; }
 
@@ -43,10 +47,10 @@ Layout layout(int M, int C, int Vp, int bf16) {
   L.part = bf16 ? r256(size_t(M) * nt * 4) : 0;  // each of part_max, part_sum
   L.tgt = bf16 ? r256(size_t(M) * 4) : 0;
   L.z = bf16 ? 0 : r256(size_t(mc) * Vp * 4);
-  L.dz = r256(size_t(mc) * Vp * (bf16 ? 2 : 4));
+  L.dz = r256(size_t(mc) * Vp * (bf16 ? 2 : 4));  // one chunk buffer (ring() of them)
   L.gws = r256(std::max({gemm_workspace_bytes(mc, Vp, C), gemm_workspace_bytes(mc, C, Vp),
                          gemm_workspace_bytes(Vp, C, mc), gemm_workspace_bytes(M, Vp, C)}));
-  L.total = 2 * L.part + L.tgt + L.z + L.dz + L.gws + 256;
+  L.total = 2 * L.part + L.tgt + L.z + size_t(ring(bf16)) * L.dz + L.gws + 256;
   return L;
 }
 
@@ -88,7 +92,7 @@ int lmhead_fwd(const void* h, const void* W, const int32_t* y, int M, int C, int
   float* psum = reinterpret_cast<float*>(w + L.part);
   float* tgt = reinterpret_cast<float*>(w + 2 * L.part);
   float* z = reinterpret_cast<float*>(w + 2 * L.part + L.tgt);
-  float* gws = reinterpret_cast<float*>(w + 2 * L.part + L.tgt + L.z + L.dz);
+  float* gws = reinterpret_cast<float*>(w + 2 * L.part + L.tgt + L.z + ring(bf16) * L.dz);
   if (bf16) {
     EpiParams e;
     e.kind = EPI_LSE_PARTIAL;
@@ -135,13 +139,20 @@ int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse,
   }
   char* w = static_cast<char*>(ws);
   float* z = reinterpret_cast<float*>(w + 2 * L.part + L.tgt);
-  void* dz = w + 2 * L.part + L.tgt + L.z;
-  float* gws = reinterpret_cast<float*>(w + 2 * L.part + L.tgt + L.z + L.dz);
+  char* dz0 = w + 2 * L.part + L.tgt + L.z;
+  const int nbuf = ring(bf16);
+  float* gws = reinterpret_cast<float*>(dz0 + nbuf * L.dz);
   const size_t a = bf16 ? 2 : 4;
   const int chunk = chunk_rows(bf16);
-  for (int64_t r0 = 0; r0 < M; r0 += chunk) {
+  const bool par = side && side->st && dh && dW;
+  int c = 0;
+  for (int64_t r0 = 0; r0 < M; r0 += chunk, ++c) {
     const int mc = int(std::min<int64_t>(chunk, M - r0));
     const void* hr = static_cast<const char*>(h) + r0 * C * int64_t(a);
+    void* dz = dz0 + (c % nbuf) * L.dz;
+    // the weight gradient of the chunk that last used this buffer (side
+    // stream) has finished reading it; dH of that chunk ran before on st
+    if (par && c >= nbuf) GPT2_CUDA_TRY(cudaStreamWaitEvent(st, side->e_join[c % nbuf], 0));
     int rc;
     if (bf16) {
       EpiParams e;
@@ -166,7 +177,6 @@ int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse,
                                        st);
     }
     if (rc) return rc;
-    const bool par = side && side->st && dh && dW;
     if (par) {  // dz of this chunk complete: dW may start beside dH
       GPT2_CUDA_TRY(cudaEventRecord(side->e_fork, st));
       GPT2_CUDA_TRY(cudaStreamWaitEvent(side->st, side->e_fork, 0));
@@ -182,7 +192,7 @@ int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse,
       if (rc) return rc;
     }
     if (dW) {
-      // dH and dW only read dz: with a side stream, dW fills dH's last wave
+      // chunks add into dW one after the other (stream order): deterministic
       EpiParams e;
       e.kind = EPI_ACC;
       e.out = dW;
@@ -192,11 +202,10 @@ int lmhead_bwd(const void* h, const void* W, const int32_t* y, const float* lse,
                  par ? side->ws_bytes : L.gws};
       rc = gemm_launch(g, par ? side->st : st);
       if (rc) return rc;
-      if (par) {  // dz is rewritten by the next chunk
-        GPT2_CUDA_TRY(cudaEventRecord(side->e_join, side->st));
-        GPT2_CUDA_TRY(cudaStreamWaitEvent(st, side->e_join, 0));
-      }
+      if (par) GPT2_CUDA_TRY(cudaEventRecord(side->e_join[c % nbuf], side->st));
     }
   }
+  // the side stream runs in order: its last weight-gradient GEMM done means all are
+  if (par && c > 0) GPT2_CUDA_TRY(cudaStreamWaitEvent(st, side->e_join[(c - 1) % nbuf], 0));
   return GPT2_OK;
 }

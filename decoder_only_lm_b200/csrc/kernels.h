@@ -143,17 +143,19 @@ int launch_attn_bwd(const T* dout, const T* qkv, const T* out, const float* lse,
 // ---------------------------------------------------------------- tied LM head + CE
 // Forward: lse[m] = logsumexp_v (h[m] . W[v]) over all Vp rows of W,
 // row_loss[m] = lse[m] - h[m] . W[y[m]].  Backward: with dz = scale (softmax -
-// onehot(y)): dh = dz W (overwritten), dW (+)= dz^T h.  At most a bounded row
-// chunk of dz (never the whole [M, Vp]) lives in the workspace.
+// onehot(y)): dh = dz W (overwritten), dW (+)= dz^T h.  dz exists only as a
+// bounded ring of row-chunk buffers in the workspace (never the whole [M, Vp]
+// once M is above one chunk).
 size_t lmhead_workspace(int M, int C, int Vp, int bf16);
 int lmhead_fwd(const void* h, const void* W, const int32_t* y, int M, int C, int Vp, int bf16,
                float* lse, float* row_loss, void* ws, size_t ws_bytes, cudaStream_t st);
 // With side != nullptr the dW GEMM of each chunk runs on that stream (its own
-// split-K workspace side_ws of ws-sized need), forked after the chunk's dz and
-// joined before the next chunk rewrites dz (events e_fork, e_join).
+// split-K workspace side_ws of ws-sized need), forked after the chunk's dz
+// (event e_fork); e_join[b] is recorded after the dW GEMM that read chunk
+// buffer b, and st waits on it before buffer b is rewritten and at the end.
 struct LmSide {
   cudaStream_t st = nullptr;
-  cudaEvent_t e_fork = nullptr, e_join = nullptr;
+  cudaEvent_t e_fork = nullptr, e_join[2] = {nullptr, nullptr};
   float* ws = nullptr;
   size_t ws_bytes = 0;
 };

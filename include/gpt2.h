@@ -306,6 +306,45 @@ int gpt2_synchronize(gpt2_handle* h);
  * right after gpt2_zero_grad first materialises the zeros. */
 int gpt2_arena(gpt2_handle* h, int which, float** ptr, int64_t* n_elems);
 
+/* ---------------------------------------------------------------- data parallel */
+/* The data-parallel step [LECTURE: DDP; CH28 §28.3, rank offsets]: every rank
+ * runs forward and backward on its own windows, the ranks' gradients are
+ * averaged (an all-reduce of the gradient arena), and every rank applies the
+ * same clip + AdamW.  These calls let the caller overlap the exchange with
+ * the backward pass: the arena is cut into buckets in the order the backward
+ * finishes them, and the handle reports each one as it becomes final.  The
+ * exchange itself is the caller's (e.g. NCCL through torch.distributed). */
+
+/* Host-only layout of the arenas for configuration cfg (no handle, no device
+ * call): tensor i (the order of gpt2_tensor_info) starts at element *offset
+ * and holds *n_elems elements; its name is copied to name (name_len bytes,
+ * NUL-terminated, nullable).  *n_tensors (nullable) receives the tensor count;
+ * i = -1 asks for the count only. */
+int gpt2_arena_layout(const gpt2_config* cfg, int i, char* name, int name_len, int64_t* offset,
+                      int64_t* n_elems, int* n_tensors);
+
+/* Host-only bucket plan of the gradient arena for configuration cfg, as
+ * contiguous element ranges (offset[k], count[k]) each tagged with its bucket
+ * bucket[k].  Bucket b < n_layer holds the four weight matrices of layer
+ * n_layer-1-b (final once that layer's backward is done); bucket n_layer holds
+ * wte, wpe and every vector (final after the embedding backward, the last
+ * step of the backward).  The ranges cover the whole arena once, padding
+ * included.  *n_ranges receives the number of ranges; the arrays are filled
+ * only when max_ranges >= *n_ranges. */
+int gpt2_grad_buckets(const gpt2_config* cfg, int max_ranges, int* n_ranges, int64_t* offset,
+                      int64_t* count, int* bucket);
+
+/* While fn is set (NULL clears it), gpt2_backward calls fn(user, b) on the
+ * calling thread for b = 0 .. n_layer, in that order, each time right after it
+ * has enqueued on the handle's stream the last work that writes bucket b: work
+ * the callback enqueues on another stream after an event recorded on the
+ * handle's stream at that moment sees bucket b final.  The callback must not
+ * call into the handle.  It is not called while gpt2_stream_begin records a
+ * step.  With gradient accumulation, set it before the last micro-batch's
+ * backward only. */
+typedef void (*gpt2_bucket_fn)(void* user, int bucket);
+int gpt2_set_bucket_callback(gpt2_handle* h, gpt2_bucket_fn fn, void* user);
+
 /* ---------------------------------------------------------------- profiling */
 /* Kernel groups timed by the built-in profiler. */
 #define GPT2_PROF_GEMM 0        /* linear-layer contractions (fwd, dX, dW) */
@@ -341,8 +380,10 @@ int gpt2_profile_read(gpt2_handle* h, int cat, int64_t* launches, double* ms, do
  * y: device int32 [M] in [0, V).  d_loss: device fp32 [1].  d_lse (nullable):
  * device fp32 [M] log-normalisers.  d_dh (nullable, same type as hidden) and
  * d_dw (nullable, fp32 [Vp,C]) request the backward.  The [M,Vp] logits are
- * never stored whole: at most a row chunk of dz (16384 rows for GPT2_BF16,
- * 2048 for GPT2_F32) lives in the workspace.
+ * never stored: the forward reduces them tile by tile to per-row partials,
+ * and the backward recomputes them chunk by chunk into a fixed-size ring of
+ * dz chunk buffers (GPT2_BF16: two chunks of 1024 rows, 2 x 1024 x Vp bf16,
+ * 206 MB at Vp = 50304, whatever M is; GPT2_F32: one chunk of 2048 rows).
  * workspace: device memory of at least gpt2_lmhead_ce_workspace() bytes.
  * C must be a multiple of 64 for GPT2_BF16.  Asynchronous on `stream`. */
 int gpt2_lmhead_ce_workspace(int M, int C, int Vp, int dtype, size_t* bytes);
@@ -394,6 +435,9 @@ int gpt2_attention_bwd(const void* dout, const void* qkv, const void* out, const
  *   - Limit: B*H*T <= 1,048,576 rows, else GPT2_ERR_ARG and a message.
  *   - The first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
+ *     The address is then kept for the rest of the process: resetting the
+ *     device (cudaDeviceReset) or calling from a context other than the
+ *     device's primary one is not supported.
  *   - Every call uses the same array, which keeps the last call's contents
  *     (each call writes what it reads first, so nothing needs clearing):
  *     calls that overlap on the GPU, e.g. on two streams, race. */

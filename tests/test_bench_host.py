@@ -19,20 +19,36 @@ def test_parameter_counts_and_step_flops():
 
 
 def test_stored_traffic_follows_the_source_hash(tmp_path, monkeypatch):
-    per, src = bench.stored_traffic("gemm", "gpt2-124m", 192)
-    assert per is not None and per > 1e6 and "per launch" in src
+    """The record is used only while the kernel sources hash to the ones it was
+    captured on: a copy of the record stamped with the current sources' hash is
+    accepted, the same record stamped with another hash is refused."""
+    import hashlib
     assert bench.stored_traffic("gemm", "gpt2-350m", 192) == (None, None)
-    # a record taken on other sources is refused
     rec = json.load(open(os.path.join(bench.ROOT, "profiles",
                                       "gemm_dram_traffic_gpt2_124m_b16_t1024.json")))
-    rec["kernel_sources_sha256"] = "0" * 64
     root = tmp_path / "r"
     (root / "profiles").mkdir(parents=True)
-    (root / "profiles" / "gemm_dram_traffic_gpt2_124m_b16_t1024.json").write_text(json.dumps(rec))
-    for f in rec["kernel_sources"]:
+    h = hashlib.sha256()
+    for f in sorted(rec["kernel_sources"]):
         dst = root / f
         dst.parent.mkdir(parents=True, exist_ok=True)
-        dst.write_bytes(open(os.path.join(bench.ROOT, f), "rb").read())
+        data = open(os.path.join(bench.ROOT, f), "rb").read()
+        dst.write_bytes(data)
+        h.update(data)
     monkeypatch.setattr(bench, "ROOT", str(root))
+    path = root / "profiles" / "gemm_dram_traffic_gpt2_124m_b16_t1024.json"
+    rec["kernel_sources_sha256"] = h.hexdigest()
+    path.write_text(json.dumps(rec))
+    per, src = bench.stored_traffic("gemm", "gpt2-124m", 192)
+    assert per is not None and per > 1e6 and "per launch" in src
+    rec["kernel_sources_sha256"] = "0" * 64
+    path.write_text(json.dumps(rec))
     per, why = bench.stored_traffic("gemm", "gpt2-124m", 192)
     assert per is None and "changed" in why
+
+
+def test_metric_names_the_workload_model():
+    assert set(bench.METRICS) == set(bench.WORKLOADS)
+    base = json.load(open(os.path.join(bench.ROOT, "BASELINE.json")))
+    assert bench.METRICS["gpt2-124m"] == base["metric"]
+    assert bench.METRICS["gpt2-350m"].startswith("GPT-2 350M")
