@@ -50,6 +50,10 @@ WORKLOADS = {
     "gpt2-124m-accum": dict(n_layer=12, n_embd=768, n_head=12, vocab_size=50257,
                             padded_vocab=50304, max_T=1024, B=64, T=1024, accum=8, eval_batches=20),
 }
+# the fused LM head + cross-entropy alone (forward loss, backward dHidden and dW), bf16:
+# hidden [8192, 768] ~ N(0, 1), tied weight [50304, 768] ~ N(0, 0.02), targets uniform in
+# [0, 50257), all from seed 2
+LMHEAD = {"lmhead-ce-8192": dict(M=8192, C=768, Vp=50304, V=50257)}
 # schedule of the accumulation workload: max 6e-4, min 6e-5, 100 warmup steps; the decay
 # length is the run's choice (its token budget), 10,000 optimizer steps here
 LR_SCHEDULE = dict(max_lr=6e-4, min_lr=6e-5, warmup_steps=100, total_steps=10000)
@@ -57,6 +61,7 @@ METRIC = "GPT-2 124M training tokens/s (fwd+bwd+AdamW, T=1024, bf16) and MFU"
 # the line's metric names the model the workload trains
 METRICS = {"gpt2-124m": METRIC,
            "gpt2-124m-accum": METRIC,
+           "lmhead-ce-8192": "fused LM-head + cross-entropy fwd+bwd TFLOP/s (8192x768x50304, bf16)",
            "gpt2-350m": "GPT-2 350M training tokens/s (fwd+bwd+AdamW, T=1024, bf16) and MFU"}
 DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -76,9 +81,11 @@ def flops_per_token(w):
 
 def stored_traffic(group, workload, launches_per_step):
     """DRAM bytes per launch of a kernel group from the committed ncu capture
-    (profiles/gemm_dram_traffic_*.json), or None when that capture was taken on
-    another workload or on kernel sources that have changed since."""
-    path = os.path.join(ROOT, "profiles", "gemm_dram_traffic_gpt2_124m_b16_t1024.json")
+    (profiles/gemm_dram_traffic_*.json: one block's GEMMs run standalone at the
+    step's shapes, so bytes per launch carry over to the 12-block step), or None
+    when that capture was taken on another workload or on kernel sources that
+    have changed since."""
+    path = os.path.join(ROOT, "profiles", "gemm_dram_traffic_gpt2_124m_layer_m16384.json")
     if workload != "gpt2-124m" or not os.path.exists(path):
         return None, None
     rec = json.load(open(path))
@@ -91,9 +98,10 @@ def stored_traffic(group, workload, launches_per_step):
         return None, "kernel sources changed since the capture"
     g = rec[group]
     per_launch = g["dram_bytes_per_step"] / max(1.0, launches_per_step)
-    return per_launch, ("ncu dram__bytes_read.sum + dram__bytes_write.sum over one step "
-                        f"({g['kernel_launches_per_step']} launches), per launch; "
-                        "profiles/gemm_dram_traffic_gpt2_124m_b16_t1024.json")
+    return per_launch, ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one block's "
+                        f"{rec['per_layer']['launches']} GEMM launches captured standalone "
+                        "(opbench layer_gemms at M=16384), per launch; "
+                        "profiles/gemm_dram_traffic_gpt2_124m_layer_m16384.json")
 
 
 def load_peaks():
@@ -234,6 +242,146 @@ def run_reference(args, w, wname):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- LM head alone
+def lmhead_inputs(w):
+    """The seed-2 inputs of the LM-head workload (float32 host arrays)."""
+    M, Cc, Vp, V = w["M"], w["C"], w["Vp"], w["V"]
+    h = synth.normal(synth.derive_key(2, 1), M * Cc, 1.0).reshape(M, Cc).astype(np.float32)
+    W = synth.normal(synth.derive_key(2, 2), Vp * Cc, 0.02).reshape(Vp, Cc).astype(np.float32)
+    y = synth.randint(synth.derive_key(2, 3), M, V).astype(np.int32)
+    return h, W, y
+
+
+def lmhead_cpu_baseline(w, h, W, y, rows=64):
+    """The oracle (fp32) on the first `rows` rows, scaled to all M rows (the work
+    per row does not depend on the other rows)."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.lmhead_ce(h[:rows], W, y[:rows], w["V"])
+    dt = (time.perf_counter() - t0) * w["M"] / rows
+    fl = 3 * 2.0 * w["M"] * w["C"] * w["Vp"]
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"oracle fp32 forward + backward on {rows} of the {w['M']} rows "
+                      f"({dt * rows / w['M']:.1f} s), scaled to all rows"}
+
+
+def run_lmhead(args, w, wname):
+    """Config 2: the tied head with mean cross-entropy alone, forward and backward,
+    as one op-level call (gpt2_lmhead_ce) per step on device-resident inputs."""
+    import ctypes
+    import torch
+    import decoder_only_lm_b200 as g
+    M, Cc, Vp, V = w["M"], w["C"], w["Vp"], w["V"]
+    h_np, W_np, y_np = lmhead_inputs(w)
+    h = torch.from_numpy(h_np).cuda().bfloat16()
+    W = torch.from_numpy(W_np).cuda().bfloat16()
+    y = torch.from_numpy(y_np).cuda()
+    ws_b = ctypes.c_size_t()
+    g._check(g.lib.gpt2_lmhead_ce_workspace(M, Cc, Vp, g.BF16, ctypes.byref(ws_b)))
+    ws = torch.empty(ws_b.value, dtype=torch.uint8, device="cuda")
+    loss = torch.empty(1, device="cuda")
+    lse = torch.empty(M, device="cuda")
+    dh = torch.empty_like(h)
+    dW = torch.zeros((Vp, Cc), device="cuda")  # accumulated into by every call
+    st = torch.cuda.current_stream()
+
+    def call(hh=h, yy=y):
+        g._check(g.lib.gpt2_lmhead_ce(hh.data_ptr(), W.data_ptr(), yy.data_ptr(), M, Cc, Vp, V, g.BF16,
+                                      1.0, loss.data_ptr(), lse.data_ptr(), dh.data_ptr(),
+                                      dW.data_ptr(), ws.data_ptr(), ws_b.value, st.cuda_stream))
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = g.launch_count()
+    e0.record(st)
+    for _ in range(args.steps):
+        call()
+    e1.record(st)
+    torch.cuda.synchronize()
+    n1 = g.launch_count()
+    clk = clocks.stop()
+    assert g.device_error() == 0
+    ms = e0.elapsed_time(e1) / args.steps
+    fl = 3 * 2.0 * M * Cc * Vp  # forward, dHidden, dW (the recompute is extra work)
+    tflops = fl / (ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    # end to end: hidden and targets from pinned host memory, the loss read back
+    hh = torch.from_numpy(h_np).bfloat16().pin_memory()
+    yh = torch.from_numpy(y_np).pin_memory()
+    hd, yd = torch.empty_like(h), torch.empty_like(y)
+    times = []
+    lh = torch.empty(1, pin_memory=True)
+    for i in range(max(3, args.steps // 2) + 1):
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        hd.copy_(hh, non_blocking=True)
+        yd.copy_(yh, non_blocking=True)
+        call(hd, yd)
+        lh.copy_(loss, non_blocking=True)
+        b.record(st)
+        torch.cuda.synchronize()
+        if i > 0:
+            times.append(a.elapsed_time(b))
+    e_ms = sum(times) / len(times)
+    line = {
+        "metric": METRICS[wname], "value": tflops, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (hidden N(0,1), weight N(0,0.02), targets uniform, seed 2)",
+        "config": {"workload": wname, "rows": M, "hidden": Cc, "padded_vocab": Vp, "vocab": V,
+                   "flops_per_step": fl, "flops": "algorithmic: 3 x 2 M C Vp (forward, dHidden, "
+                   "dW); the backward's recompute of the logits is extra",
+                   "l2": "working set (weights 77 MB, fp32 dW 155 MB, workspace 230 MB) > 126 MB L2;"
+                         " no flush"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "gpt2_lmhead_ce (LSE-partial GEMM, merge, per 2048-row chunk: "
+                               "CE-gradient GEMM, dHidden GEMM + split reduction, dW GEMM)",
+                     "peak_source": f"{peak_src} bf16 burst (op timed alone)",
+                     "measured": "CUDA events around the timed calls on the launching stream"},
+        "clocks": clk,
+        "gpu_launches": n1 - n0,
+        "e2e": {"value": fl / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * Cc * 2 + M * 4, "d2h_bytes_per_step": 4, "ms_per_step": e_ms,
+                "api": "gpt2_lmhead_ce (host bf16 hidden + int32 targets in, loss out)"},
+        "cpu_baseline": None if args.no_cpu_baseline else lmhead_cpu_baseline(w, h_np, W_np, y_np),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_lmhead_reference(args, w, wname):
+    """The oracle on the LM-head workload, each step a 16-row sample scaled to
+    all rows."""
+    import oracle
+    h, W, y = lmhead_inputs(w)
+    rows = 16
+    fl = 3 * 2.0 * w["M"] * w["C"] * w["Vp"]
+    times = []
+    for i in range(args.warmup + args.steps):
+        r0 = (i * rows) % w["M"]
+        t0 = time.perf_counter()
+        oracle.lmhead_ce(h[r0:r0 + rows], W, y[r0:r0 + rows], w["V"])
+        if i >= args.warmup:
+            times.append((time.perf_counter() - t0) * w["M"] / rows)
+    step_s = sum(times) / len(times)
+    value = fl / step_s / 1e12
+    sample = (f"oracle fp32 forward + backward on {rows} rows per step, scaled to all {w['M']} rows")
+    print(json.dumps({
+        "impl": "reference", "metric": METRICS[wname], "value": value, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seed 2)", "config": {"workload": wname, "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+        flush=True)
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -241,13 +389,19 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--workload", default="gpt2-124m", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="gpt2-124m", choices=sorted(WORKLOADS) + sorted(LMHEAD))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
-    w = WORKLOADS[args.workload]
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload in LMHEAD:
+        if int(os.environ.get("RANK", "0")) != 0:
+            return  # one GPU's op; further ranks have nothing to do
+        if args.impl == "reference":
+            return run_lmhead_reference(args, LMHEAD[args.workload], args.workload)
+        return run_lmhead(args, LMHEAD[args.workload], args.workload)
+    w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w, args.workload)
 

@@ -93,6 +93,7 @@ SIGNATURES = {
                          _sz, _P]),
     "gpt2_linear": (_i, [_i, _P, _P, _i, _P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "gpt2_device_error": (_i, [C.POINTER(_i)]),
+    "gpt2_launch_count": (_i, [C.POINTER(_i64)]),
 }
 
 
@@ -577,6 +578,13 @@ def cosine_lr(t, max_lr, min_lr, warmup_steps, total_steps):
         return max_lr * (t / warmup_steps)
     phase = math.pi * (t - warmup_steps) / (total_steps - warmup_steps)
     return min_lr + (max_lr - min_lr) * (1.0 + math.cos(phase)) / 2.0
+
+
+def launch_count():
+    """Kernel launches issued by the library from this thread so far."""
+    n = C.c_int64()
+    _check(lib.gpt2_launch_count(C.byref(n)))
+    return n.value
 
 
 def device_error():

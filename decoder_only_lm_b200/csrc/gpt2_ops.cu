@@ -259,6 +259,12 @@ int gpt2_sample(const float* logits, int64_t ld, int B, int V, float temperature
                        static_cast<cudaStream_t>(stream));
 }
 
+int gpt2_launch_count(int64_t* n) {
+  if (!n) return GPT2_ERR_ARG;
+  *n = gpt2_internal::launches();
+  return GPT2_OK;
+}
+
 int gpt2_device_error(int* code) {
   if (!code) return GPT2_ERR_ARG;
   int* w = device_error_word();

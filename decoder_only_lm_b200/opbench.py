@@ -5,6 +5,7 @@
     python -m decoder_only_lm_b200.opbench attention --B 16 --T 1024 --C 768 --H 12 [--bwd]
     python -m decoder_only_lm_b200.opbench layernorm --M 16384 --C 768 [--bwd]
     python -m decoder_only_lm_b200.opbench linear --M 16384 --N 3072 --K 768 --epi gelu [--graph]
+    python -m decoder_only_lm_b200.opbench layer_gemms --M 16384 --C 768 (one block's linear layers)
     python -m decoder_only_lm_b200.opbench sample --B 16 --V 50257 [--temperature 0.8 --top-k 0 --top-p 0.9]
     python -m decoder_only_lm_b200.opbench generate --B 16 --T0 64 --new 64 [--cached] (GPT-2 124M, bf16)
 
@@ -63,7 +64,7 @@ EPIS = {"bias": g.LINEAR_BIAS, "gelu": g.LINEAR_BIAS_GELU, "resid": g.LINEAR_RES
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("op", choices=["matmul", "lmhead", "attention", "layernorm", "linear",
-                                   "sample", "generate"])
+                                   "sample", "generate", "layer_gemms"])
     ap.add_argument("--temperature", type=float, default=0.8)
     ap.add_argument("--top-k", type=int, default=0)
     ap.add_argument("--top-p", type=float, default=0.9)
@@ -124,6 +125,43 @@ def main():
         ms = timed(fn, a.iters, a.warmup)
         fl = 2.0 * a.M * a.N * a.K
         out.update(M=a.M, N=a.N, K=a.K, epi=a.epi, ms=ms, tflops=fl / ms / 1e9)
+    elif a.op == "layer_gemms":
+        # the twelve contractions of one transformer block as the training step
+        # issues them (M = B*T rows, C, F = 4C, bf16 operands): forward QKV + bias,
+        # attention projection + residual, fc + bias + GELU, fc projection +
+        # residual; backward per layer in reverse: fc projection dX with GELU',
+        # its dW, fc dX, its dW, projection dX, its dW, QKV dX, its dW (fp32 dW
+        # accumulated, split along the rows where the cost model picks it)
+        M, Cc = a.M, a.C
+        F = 4 * Cc
+        bf = torch.bfloat16
+        r = lambda *s_: torch.randn(*s_, device=dev).to(bf)
+        x, att, g_, u = r(M, Cc), r(M, Cc), r(M, F), r(M, F)
+        Wqkv, Wp, Wfc, Wfp = r(3 * Cc, Cc), r(Cc, Cc), r(F, Cc), r(Cc, F)
+        bq, bp, bfc, bfp = (torch.randn(n, device=dev) for n in (3 * Cc, Cc, F, Cc))
+        res = torch.randn(M, Cc, device=dev)
+        res2 = torch.empty_like(res)
+        qkv, fc_u, fc_g = torch.empty(M, 3 * Cc, device=dev, dtype=bf), torch.empty(M, F, device=dev, dtype=bf), torch.empty(M, F, device=dev, dtype=bf)
+        dres, du, dln, dqkv = r(M, Cc), torch.empty(M, F, device=dev, dtype=bf), torch.empty(M, Cc, device=dev, dtype=bf), r(M, 3 * Cc)
+        dWqkv, dWp, dWfc, dWfp = (torch.zeros(*w.shape, device=dev) for w in (Wqkv, Wp, Wfc, Wfp))
+
+        def fn():
+            g.linear(g.LINEAR_BIAS, x, Wqkv, bias=bq, out=qkv)
+            g.linear(g.LINEAR_RESIDUAL, att, Wp, bias=bp, inp=res, out=res2)
+            g.linear(g.LINEAR_BIAS_GELU, x, Wfc, bias=bfc, out=fc_g, out2=fc_u)
+            g.linear(g.LINEAR_RESIDUAL, g_, Wfp, bias=bfp, inp=res2, out=res)
+            g.linear(g.LINEAR_GELU_BWD, dres, Wfp, inp=u, w_kn=True, out=du)
+            g.matmul(dres, g_, a_kmajor=False, b_kmajor=False, M=Cc, N=F, K=M, out=dWfp, accumulate=True)
+            g.matmul(du, Wfc, a_kmajor=True, b_kmajor=False, M=M, N=Cc, K=F, out=dln)
+            g.matmul(du, x, a_kmajor=False, b_kmajor=False, M=F, N=Cc, K=M, out=dWfc, accumulate=True)
+            g.matmul(dres, Wp, a_kmajor=True, b_kmajor=False, M=M, N=Cc, K=Cc, out=dln)
+            g.matmul(dres, att, a_kmajor=False, b_kmajor=False, M=Cc, N=Cc, K=M, out=dWp, accumulate=True)
+            g.matmul(dqkv, Wqkv, a_kmajor=True, b_kmajor=False, M=M, N=Cc, K=3 * Cc, out=dln)
+            g.matmul(dqkv, x, a_kmajor=False, b_kmajor=False, M=3 * Cc, N=Cc, K=M, out=dWqkv, accumulate=True)
+
+        ms = timed(fn, a.iters, a.warmup)
+        fl = 3 * 2.0 * M * 12 * Cc * Cc
+        out.update(M=M, C=Cc, ms=ms, tflops=fl / ms / 1e9)
     elif a.op == "sample":
         # next-token choice over B rows of fp32 logits (the padded width, V drawn)
         z = 3.0 * torch.randn((a.B, a.Vp), device=dev)

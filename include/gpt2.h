@@ -381,9 +381,9 @@ int gpt2_profile_read(gpt2_handle* h, int cat, int64_t* launches, double* ms, do
  * device fp32 [M] log-normalisers.  d_dh (nullable, same type as hidden) and
  * d_dw (nullable, fp32 [Vp,C]) request the backward.  The [M,Vp] logits are
  * never stored: the forward reduces them tile by tile to per-row partials,
- * and the backward recomputes them chunk by chunk into a fixed-size ring of
- * dz chunk buffers (GPT2_BF16: two chunks of 1024 rows, 2 x 1024 x Vp bf16,
- * 206 MB at Vp = 50304, whatever M is; GPT2_F32: one chunk of 2048 rows).
+ * and the backward recomputes them chunk by chunk into one fixed-size dz
+ * chunk buffer (2048 rows: 2048 x Vp bf16 = 206 MB at Vp = 50304 for
+ * GPT2_BF16, fp32 for GPT2_F32), whatever M is.
  * workspace: device memory of at least gpt2_lmhead_ce_workspace() bytes.
  * C must be a multiple of 64 for GPT2_BF16.  Asynchronous on `stream`. */
 int gpt2_lmhead_ce_workspace(int M, int C, int Vp, int dtype, size_t* bytes);
@@ -482,6 +482,13 @@ int gpt2_matmul(const void* A, int a_kmajor, int64_t lda, const void* B, int b_k
 int gpt2_linear(int epi, const void* x, const void* w, int w_kn, const float* bias,
                 const void* in, void* out, void* out2, int M, int N, int K, int dtype,
                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Kernel launches the library has issued from the calling thread since the
+ * process started, op-level calls and handle calls alike.  Kernels recorded
+ * into a graph by gpt2_stream_begin count once, when recorded; replays by
+ * gpt2_stream_steps are not counted here (gpt2_profile_read(h, -1) counts
+ * them per handle). */
+int gpt2_launch_count(int64_t* n);
 
 /* Reads and clears the device error word shared by the op-level calls
  * (bounded-wait timeouts).  *code = GPT2_OK when nothing was recorded.

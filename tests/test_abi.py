@@ -76,7 +76,7 @@ def test_null_arguments_are_refused(g):
     assert g.lib.gpt2_lmhead_ce_workspace(128, 768, 50304, g.BF16, C.byref(ws)) == g.OK
     assert ws.value >= 128 * 50304 * 2  # holds the rows' dz (bf16)
     assert ws.value < 8192 * 50304 * 2  # ... and less than the full [8192, 50304] bf16 logits
-    # the live dz is a ring of two 1024-row chunks whatever M is: at the GPT-2
+    # the live dz is one 2048-row chunk whatever M is: at the GPT-2
     # 124M batch (16 x 1024 rows) the whole workspace stays within 256 MB, and
     # from there on it grows only by the per-row partials of the forward
     # (197 column tiles x 2 x 4 B) and the per-row target logit
@@ -88,7 +88,7 @@ def test_null_arguments_are_refused(g):
     assert sizes[16384] < 16384 * 50304 * 2 // 6
     per_row = (sizes[65536] - sizes[16384]) / (65536 - 16384)
     assert per_row <= 197 * 2 * 4 + 4 + 8 + 1  # (two lse/loss words of the op-level call)
-    assert sizes[2048] >= 2 * 1024 * 50304 * 2
+    assert sizes[2048] >= 2048 * 50304 * 2
     # fused linear layer: missing inputs and unknown epilogues are refused on the host
     buf = C.c_void_p(16)  # never dereferenced: the arguments are rejected first
     L = g.lib.gpt2_linear

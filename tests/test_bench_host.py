@@ -25,7 +25,7 @@ def test_stored_traffic_follows_the_source_hash(tmp_path, monkeypatch):
     import hashlib
     assert bench.stored_traffic("gemm", "gpt2-350m", 192) == (None, None)
     rec = json.load(open(os.path.join(bench.ROOT, "profiles",
-                                      "gemm_dram_traffic_gpt2_124m_b16_t1024.json")))
+                                      "gemm_dram_traffic_gpt2_124m_layer_m16384.json")))
     root = tmp_path / "r"
     (root / "profiles").mkdir(parents=True)
     h = hashlib.sha256()
@@ -36,7 +36,7 @@ def test_stored_traffic_follows_the_source_hash(tmp_path, monkeypatch):
         dst.write_bytes(data)
         h.update(data)
     monkeypatch.setattr(bench, "ROOT", str(root))
-    path = root / "profiles" / "gemm_dram_traffic_gpt2_124m_b16_t1024.json"
+    path = root / "profiles" / "gemm_dram_traffic_gpt2_124m_layer_m16384.json"
     rec["kernel_sources_sha256"] = h.hexdigest()
     path.write_text(json.dumps(rec))
     per, src = bench.stored_traffic("gemm", "gpt2-124m", 192)
@@ -48,7 +48,7 @@ def test_stored_traffic_follows_the_source_hash(tmp_path, monkeypatch):
 
 
 def test_metric_names_the_workload_model():
-    assert set(bench.METRICS) == set(bench.WORKLOADS)
+    assert set(bench.METRICS) == set(bench.WORKLOADS) | set(bench.LMHEAD)
     base = json.load(open(os.path.join(bench.ROOT, "BASELINE.json")))
     assert bench.METRICS["gpt2-124m"] == base["metric"]
     assert bench.METRICS["gpt2-350m"].startswith("GPT-2 350M")
