@@ -11,11 +11,12 @@ starts at B*T*r and advances B*T*N).  Weights are random (N(0, 0.02)); the
 stream is Zipf(1.1) ids with an end-of-text id before every document of
 geometric length (mean 600): a stand-in for a tokenised web corpus.
 
-With N > 1 (torchrun) every rank trains its own shard and the gradient arena
-is averaged bucket by bucket (one NCCL all-reduce per layer's weight matrices,
-issued on a side stream as the backward finishes that layer, then one for the
-embeddings and vectors) before clip + AdamW (data parallel; per-GPU work is
-fixed, so scaling is weak).
+With N > 1 (torchrun) every rank trains its own shard and the library
+averages the gradient arena bucket by bucket (one NCCL all-reduce per layer's
+weight matrices, issued on its communication stream as the backward finishes
+that layer, then one for the embeddings and vectors; recorded into the step's
+CUDA graph) before clip + AdamW (data parallel; per-GPU work is fixed, so
+scaling is weak).
 
 `--impl reference` times the CPU oracle (test infrastructure) on the same
 workload, each step a bounded sample of it.  Rank 0 prints one JSON line.
@@ -428,12 +429,11 @@ def main():
     model = g.GPT2(w["n_layer"], w["n_embd"], w["n_head"], w["vocab_size"], w["padded_vocab"],
                    w["max_T"], bf16=True, max_B=B, max_Tseq=T)
     model.set_params(synth.init_params(0, model.shapes()))
-    # data parallel: the gradient buckets are averaged (NCCL all-reduce) on a side
-    # stream as the last micro-batch's backward finishes each of them
-    exchange = None
+    # data parallel: the library averages each gradient bucket (NCCL all-reduce on
+    # its communication stream) as the last micro-batch's backward finishes it
     if world > 1:
-        from decoder_only_lm_b200.dp import nccl_exchange
-        exchange = nccl_exchange(model)
+        from decoder_only_lm_b200.dp import init_library_exchange
+        init_library_exchange(model)
 
     def hp_at(i):
         hp = dict(HP)
@@ -449,27 +449,20 @@ def main():
             off = ((i * acc + a) * world + rank) * B * T
             x, y = model.batch_from_stream(stream, off, B, T)
             model.forward_loss(x, y, loss=False)
-            if exchange and a == acc - 1:
-                exchange.arm()
+            if world > 1:
+                model.dp_sync(a == acc - 1)  # exchange after the last micro-batch only
             model.backward(1.0 / acc)
-        if exchange:
-            exchange.finish()
         model.clip_adamw_step(**hp_at(i), norm=False)
 
-    # One GPU: each optimizer step is replayed from a CUDA graph recorded by
+    # Each optimizer step is replayed from a CUDA graph recorded by
     # gpt2_stream_begin (windows cut at a device cursor that advances through
-    # the stream; the learning rate is set before each replay).  Several GPUs:
-    # the same calls one by one, with the bucketed exchange overlapping the
-    # last backward.
-    use_graph = world == 1
+    # the stream: rank r starts at B*T*r and advances B*T*N; the learning rate is
+    # set before each replay).  With N > 1 the graph holds the bucketed
+    # gradient exchange too.
     lrs = [hp_at(i)["lr"] for i in range(steps_total)]
-    if use_graph:
-        model.stream_begin(stream, 0, B * T, B, T, accum=acc,
-                           **{k: v for k, v in HP.items() if k != "lr"})
-        model.stream_steps(lrs[:args.warmup])
-    else:
-        for i in range(args.warmup):
-            step(i)
+    model.stream_begin(stream, rank * B * T, world * B * T, B, T, accum=acc,
+                       **{k: v for k, v in HP.items() if k != "lr"})
+    model.stream_steps(lrs[:args.warmup])
     model.synchronize()
     torch.cuda.synchronize()
     if world > 1:
@@ -484,18 +477,13 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(st)
-    if use_graph:
-        model.stream_steps(lrs[args.warmup:])
-    else:
-        for i in range(args.warmup, steps_total):
-            step(i)
+    model.stream_steps(lrs[args.warmup:])
     e1.record(st)
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    if use_graph:
-        cursor = model.stream_end()  # also surfaces any device-side error of the timed steps
-        assert cursor == steps_total * acc * B * T, cursor
+    cursor = model.stream_end()  # also surfaces any device-side error of the timed steps
+    assert cursor == (rank + steps_total * acc * world) * B * T, cursor
     if world > 1:
         t = torch.tensor([ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -568,11 +556,9 @@ def main():
                 model.zero_grad()
                 for m_ in range(acc):
                     model.forward_loss(xh.numpy()[m_], yh.numpy()[m_], loss=(m_ == acc - 1))
-                    if exchange and m_ == acc - 1:
-                        exchange.arm()
+                    if world > 1:
+                        model.dp_sync(m_ == acc - 1)
                     model.backward(1.0 / acc)
-                if exchange:
-                    exchange.finish()
                 model.clip_adamw_step(**hp_at(steps_total + i), norm=True)
             b.record(st)
             torch.cuda.synchronize()
@@ -623,8 +609,8 @@ def main():
             "data": "synthetic (Zipf(1.1)/EOT token stream seed 3, N(0,0.02) weights seed 0)",
             "config": {"workload": args.workload, "global_batch": acc * B * world, "seq_len": T,
                        "micro_batch_per_gpu": B, "accumulation": acc, "parallelism": f"dp{world}",
-                       "step_launch": ("CUDA graph of one optimizer step, replayed (gpt2_stream_steps)"
-                                       if use_graph else "one library call per operation"),
+                       "step_launch": "CUDA graph of one optimizer step, replayed (gpt2_stream_steps)"
+                                      + (", bucketed NCCL gradient exchange inside" if world > 1 else ""),
                        "l2": "working set (saved activations and weights + optimizer state, GBs) "
                              ">> 126 MB L2; no flush"},
             # MFU is against the dense bf16 datasheet peak (2250 TFLOP/s per GPU);

@@ -75,6 +75,9 @@ SIGNATURES = {
     "gpt2_grad_buckets": (_i, [C.POINTER(Config), _i, C.POINTER(_i), C.POINTER(_i64),
                                C.POINTER(_i64), C.POINTER(_i)]),
     "gpt2_set_bucket_callback": (_i, [_P, BUCKET_FN, _P]),
+    "gpt2_dp_unique_id": (_i, [C.c_char_p]),
+    "gpt2_dp_init": (_i, [_P, C.c_char_p, _i, _i]),
+    "gpt2_dp_sync": (_i, [_P, _i]),
     "gpt2_profile_enable": (_i, [_P, _i]),
     "gpt2_profile_reset": (_i, [_P]),
     "gpt2_profile_read": (_i, [_P, _i, C.POINTER(_i64), C.POINTER(C.c_double), C.POINTER(C.c_double),
@@ -161,6 +164,18 @@ def arena_layout(cfg):
         _check(lib.gpt2_arena_layout(C.byref(cfg), i, buf, 128, C.byref(off), C.byref(cnt), None))
         out.append((buf.value.decode(), off.value, cnt.value))
     return out
+
+
+DP_ID_BYTES = 128
+
+
+def dp_unique_id():
+    """gpt2_dp_unique_id: the bytes every rank passes to GPT2.dp_init (made on
+    one rank, sent to the others)."""
+    import torch  # noqa: F401  (NCCL: the process's own copy, as PyTorch loads it)
+    buf = C.create_string_buffer(DP_ID_BYTES)
+    _check(lib.gpt2_dp_unique_id(buf))
+    return buf.raw
 
 
 def grad_buckets(cfg):
@@ -373,6 +388,18 @@ class GPT2:
             __cuda_array_interface__ = {"shape": (n.value,), "typestr": "<f4",
                                         "data": (addr, False), "version": 2}
         return self.torch.as_tensor(_View(), device="cuda")
+
+    def dp_init(self, unique_id, rank, world):
+        """gpt2_dp_init: average the gradient buckets over `world` ranks (NCCL)
+        inside every backward from now on."""
+        if len(unique_id) != DP_ID_BYTES:
+            raise ValueError("unique_id must be the bytes of dp_unique_id()")
+        _check(lib.gpt2_dp_init(self.h, C.c_char_p(bytes(unique_id)), int(rank), int(world)),
+               self.h)
+
+    def dp_sync(self, on=True):
+        """gpt2_dp_sync: whether the backward calls that follow exchange."""
+        _check(lib.gpt2_dp_sync(self.h, int(bool(on))), self.h)
 
     def set_bucket_callback(self, fn):
         """gpt2_set_bucket_callback: fn(bucket) is called as the backward makes

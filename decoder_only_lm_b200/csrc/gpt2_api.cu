@@ -134,6 +134,15 @@ struct gpt2_handle {
   gpt2_bucket_fn bucket_fn = nullptr;
   void* bucket_user = nullptr;
   bool capturing = false;
+  // in-library exchange (gpt2_dp_init): NCCL communicator, communication
+  // stream, the ranges of each bucket, whether the next backward exchanges
+  void* dp_comm = nullptr;
+  int dp_world = 1;
+  bool dp_sync = true;
+  bool dp_pending = false;  // this backward has enqueued exchanges to join
+  cudaStream_t st_comm = nullptr;
+  cudaEvent_t ev_dp = nullptr, ev_dp_join = nullptr;
+  std::vector<std::vector<std::pair<int64_t, int64_t>>> dp_ranges;
   Cat cats[GPT2_PROF_NCAT];
   std::vector<cudaEvent_t> ev_pool;
   int64_t launches_total = 0;
@@ -560,10 +569,40 @@ int forward_t(gpt2_handle* h, int B, int T, float* d_row_loss, bool save,
 }
 
 // ------------------------------------------------------------------ backward
-// Tells the caller (data-parallel exchange) that bucket b of the gradient
-// arena is final once the work enqueued so far on the handle's stream is done.
-void bucket_ready(gpt2_handle* h, int b) {
+// Gradient buckets in the order the backward finishes them (see
+// gpt2_grad_buckets): bucket L-1-l is the four matrices of layer l, one
+// contiguous range of the 2-D part of the arena (qkv, proj, fc, fc-proj in
+// that order); bucket L is wte and wpe (the arena's first range) and every
+// vector (its last).
+struct BucketRange {
+  int64_t off, n;
+  int b;
+};
+std::vector<BucketRange> bucket_plan(const gpt2_handle& t) {
+  std::vector<BucketRange> r;
+  for (int l = t.L - 1; l >= 0; --l) {
+    const TensorInfo* q = &t.tensors[2 + 12 * l];
+    const int64_t a = q[2].off, e = q[10].off + align_up(q[10].rows * q[10].cols, kAlign);
+    r.push_back({a, e - a, t.L - 1 - l});
+  }
+  r.push_back({0, t.tensors[2 + 2].off, t.L});
+  r.push_back({t.n_decay, t.n_arena - t.n_decay, t.L});
+  return r;
+}
+
+// Bucket b of the gradient arena is final once the work enqueued so far on
+// the handle's stream is done: start its exchange (in-library NCCL) and tell
+// the caller's callback, if any.
+int bucket_ready(gpt2_handle* h, int b) {
+  if (h->dp_comm && h->dp_sync) {
+    // the communication stream picks up here: bucket b is final on st
+    H_CUDA(h, cudaEventRecord(h->ev_dp, h->st));
+    H_CUDA(h, cudaStreamWaitEvent(h->st_comm, h->ev_dp, 0));
+    H_TRY(h, gpt2_internal::dp_allreduce_ranges(h->dp_comm, h->dp_ranges[b], h->G, h->st_comm));
+    h->dp_pending = true;
+  }
   if (h->bucket_fn && !h->capturing) h->bucket_fn(h->bucket_user, b);
+  return GPT2_OK;
 }
 
 template <typename A>
@@ -696,7 +735,7 @@ int backward_t(gpt2_handle* h, float grad_scale) {
                                             h->st)));
     }
     // layer l's weight matrices are final on st (every side-stream writer joined)
-    bucket_ready(h, h->L - 1 - l);
+    H_TRY(h, bucket_ready(h, h->L - 1 - l));
   }
   {
     // embedding: both uses of the tied matrix add into one gradient [LECTURE]
@@ -704,7 +743,12 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     H_TRY(h, launch_embed_bwd(h->xbuf, h->dres, B, T, C, h->V, G + h->off_wte, G + h->off_wpe,
                               acc, h->ws_emb, h->st));
   }
-  bucket_ready(h, h->L);  // wte, wpe and every vector
+  H_TRY(h, bucket_ready(h, h->L));  // wte, wpe and every vector
+  if (h->dp_pending) {  // the averaged gradients are what the next step reads
+    H_CUDA(h, cudaEventRecord(h->ev_dp_join, h->st_comm));
+    H_CUDA(h, cudaStreamWaitEvent(h->st, h->ev_dp_join, 0));
+    h->dp_pending = false;
+  }
   h->grads_zero = false;
   return GPT2_OK;
 }
@@ -850,6 +894,13 @@ int gpt2_destroy(gpt2_handle* h) {
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   if (h->ev_join) cudaEventDestroy(h->ev_join);
   if (h->ev_join2) cudaEventDestroy(h->ev_join2);
+  if (h->st_comm) {
+    cudaStreamSynchronize(h->st_comm);
+    cudaStreamDestroy(h->st_comm);
+  }
+  if (h->ev_dp) cudaEventDestroy(h->ev_dp);
+  if (h->ev_dp_join) cudaEventDestroy(h->ev_dp_join);
+  gpt2_internal::dp_comm_destroy(h->dp_comm);
   prof_collect(h);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   free_all(h);
@@ -1229,7 +1280,9 @@ int stream_step_body(gpt2_handle* h, const uint16_t* tok, int64_t len, int64_t s
                      float max_norm) {
   const int64_t n = int64_t(B) * T;
   h->grads_zero = true;
+  const bool sync = h->dp_sync;
   for (int a = 0; a < accum; ++a) {
+    h->dp_sync = sync && a == accum - 1;  // exchange after the last micro-batch only
     H_TRY(h, launch_slice_batch_cursor(tok, len, h->d_cursor, n, h->xbuf, h->ybuf, h->status,
                                        h->st));
     H_TRY(h, launch_advance_cursor(h->d_cursor, stride, h->st));
@@ -1237,11 +1290,14 @@ int stream_step_body(gpt2_handle* h, const uint16_t* tok, int64_t len, int64_t s
       H_TRY(h, forward_t<bf16>(h, B, T, nullptr, true));
     else
       H_TRY(h, forward_t<float>(h, B, T, nullptr, true));
-    if (h->use_bf16)
-      H_TRY(h, backward_t<bf16>(h, 1.f / float(accum)));
-    else
-      H_TRY(h, backward_t<float>(h, 1.f / float(accum)));
+    int rc = h->use_bf16 ? backward_t<bf16>(h, 1.f / float(accum))
+                         : backward_t<float>(h, 1.f / float(accum));
+    if (rc) {
+      h->dp_sync = sync;
+      return rc;
+    }
   }
+  h->dp_sync = sync;
   H_TRY(h, launch_gradnorm(h->G, h->n_arena, h->ws_norm, h->d_norm, h->st));
   H_TRY(h, launch_clip_adamw(h->P, h->G, h->Mo, h->Vo, h->Pb, h->n_arena, h->n_decay, h->d_norm,
                              h->status, 0.f, h->d_lr, beta1, beta2, eps, wd, max_norm, h->st));
@@ -1356,21 +1412,7 @@ int gpt2_grad_buckets(const gpt2_config* cfg, int max_ranges, int* n_ranges, int
   gpt2_handle t;
   set_shape(&t, *cfg);
   build_layout(&t);
-  struct R {
-    int64_t off, n;
-    int b;
-  };
-  std::vector<R> r;
-  // bucket L-1-l: the four matrices of layer l, one contiguous range of the
-  // 2-D part of the arena (qkv, proj, fc, fc-proj in that order)
-  for (int l = t.L - 1; l >= 0; --l) {
-    const TensorInfo* q = &t.tensors[2 + 12 * l];
-    const int64_t a = q[2].off, e = q[10].off + align_up(q[10].rows * q[10].cols, kAlign);
-    r.push_back({a, e - a, t.L - 1 - l});
-  }
-  // bucket L: wte and wpe (the arena's first range) and every vector (its last)
-  r.push_back({0, t.tensors[2 + 2].off, t.L});
-  r.push_back({t.n_decay, t.n_arena - t.n_decay, t.L});
+  const std::vector<BucketRange> r = bucket_plan(t);
   *n_ranges = int(r.size());
   if (max_ranges < int(r.size())) return GPT2_OK;  // the count only
   for (size_t k = 0; k < r.size(); ++k) {
@@ -1385,6 +1427,34 @@ int gpt2_set_bucket_callback(gpt2_handle* h, gpt2_bucket_fn fn, void* user) {
   if (!h) return GPT2_ERR_ARG;
   h->bucket_fn = fn;
   h->bucket_user = user;
+  return GPT2_OK;
+}
+
+int gpt2_dp_init(gpt2_handle* h, const char* id, int rank, int world) {
+  if (!h || !id) return fail(h, GPT2_ERR_ARG, "NULL argument");
+  if (world < 1 || rank < 0 || rank >= world) return fail(h, GPT2_ERR_ARG, "bad rank or world");
+  if (h->dp_comm) return fail(h, GPT2_ERR_STATE, "dp_init: already initialised");
+  if (h->graph_exec) return fail(h, GPT2_ERR_STATE, "dp_init: end the recorded stream first");
+  H_CUDA(h, cudaStreamSynchronize(h->st));
+  if (!h->st_comm) {
+    H_CUDA(h, cudaStreamCreateWithFlags(&h->st_comm, cudaStreamNonBlocking));
+    H_CUDA(h, cudaEventCreateWithFlags(&h->ev_dp, cudaEventDisableTiming));
+    H_CUDA(h, cudaEventCreateWithFlags(&h->ev_dp_join, cudaEventDisableTiming));
+  }
+  void* comm = nullptr;
+  const int rc = gpt2_internal::dp_comm_init(&comm, id, rank, world);
+  if (rc) return fail(h, rc, gpt2_internal::get_error());
+  h->dp_ranges.assign(h->L + 1, {});
+  for (const BucketRange& r : bucket_plan(*h)) h->dp_ranges[r.b].push_back({r.off, r.n});
+  h->dp_comm = comm;
+  h->dp_world = world;
+  h->dp_sync = true;
+  return GPT2_OK;
+}
+
+int gpt2_dp_sync(gpt2_handle* h, int on) {
+  if (!h) return GPT2_ERR_ARG;
+  h->dp_sync = on != 0;
   return GPT2_OK;
 }
 

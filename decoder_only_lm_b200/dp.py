@@ -8,12 +8,18 @@ and every rank applies the same clip + AdamW.
 
 The library cuts the gradient arena into buckets in the order its backward
 finishes them (gpt2_grad_buckets: one per layer's weight matrices, last
-layer first, then the embeddings and every vector) and calls back as each one
-becomes final (gpt2_set_bucket_callback).  GradExchange averages a bucket as
-soon as it is reported, so all but the last bucket cross NVLink while the
-earlier layers' backward still runs.  Averaging a range of elements in place
-is the caller's collective: NCCL all-reduce with ReduceOp.AVG on a side
-stream for GPUs (nccl_exchange), any callable for tests.
+layer first, then the embeddings and every vector).  Two ways to average them:
+
+* inside the library (init_library_exchange -> gpt2_dp_init): the backward
+  itself enqueues an NCCL all-reduce of each bucket on its communication
+  stream as soon as the bucket is final; this is stream-ordered, so it is also
+  recorded into the graph of gpt2_stream_begin (what bench.py uses);
+* by the caller, through gpt2_set_bucket_callback: GradExchange averages a
+  bucket as soon as it is reported with any collective (NCCL all-reduce with
+  ReduceOp.AVG on a side stream in nccl_exchange, gloo in the CPU tests).
+
+Either way all but the last bucket cross NVLink while the earlier layers'
+backward still runs.
 """
 from __future__ import annotations
 
@@ -93,3 +99,14 @@ def nccl_exchange(model, group=None):
         dist.all_reduce(view, op=dist.ReduceOp.AVG, group=group)
 
     return CudaGradExchange(model, average)
+
+
+def init_library_exchange(model, group=None):
+    """gpt2_dp_init over the ranks of `group` (torch.distributed, initialised):
+    rank 0 makes the NCCL id and broadcasts it; every rank joins."""
+    import torch.distributed as dist
+    from decoder_only_lm_b200 import dp_unique_id
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    box = [dp_unique_id() if rank == 0 else None]
+    dist.broadcast_object_list(box, src=0, group=group)
+    model.dp_init(box[0], rank, world)

@@ -345,6 +345,28 @@ int gpt2_grad_buckets(const gpt2_config* cfg, int max_ranges, int* n_ranges, int
 typedef void (*gpt2_bucket_fn)(void* user, int bucket);
 int gpt2_set_bucket_callback(gpt2_handle* h, gpt2_bucket_fn fn, void* user);
 
+/* The exchange inside the library (NCCL, opened at run time): every rank
+ * calls gpt2_dp_init with the same id (made by gpt2_dp_unique_id on one rank
+ * and sent to the others, e.g. by torch.distributed) and its rank.  From then
+ * on every backward that exchanges averages each gradient bucket over the
+ * ranks as soon as it is final: an NCCL all-reduce (average) of the bucket's
+ * ranges on the handle's communication stream, which first waits for the
+ * handle's stream at that point; the handle's stream waits for the
+ * communication stream at the end of the backward.  This includes the
+ * backward recorded by gpt2_stream_begin, so one replayed graph holds a whole
+ * data-parallel optimizer step (all ranks must replay the same number of
+ * steps).  gpt2_dp_sync(h, 0) turns the exchange off for the backward calls
+ * that follow (the micro-batches of an accumulation before the last one),
+ * gpt2_dp_sync(h, 1) back on; gpt2_stream_begin exchanges on the last
+ * micro-batch of each step only.  The communicator is destroyed by
+ * gpt2_destroy (release every graph first, then destroy the handles, then
+ * the caller's own process group).  GPT2_ERR_CUDA when NCCL cannot be
+ * opened or fails. */
+#define GPT2_DP_ID_BYTES 128
+int gpt2_dp_unique_id(char* id);
+int gpt2_dp_init(gpt2_handle* h, const char* id, int rank, int world);
+int gpt2_dp_sync(gpt2_handle* h, int on);
+
 /* ---------------------------------------------------------------- profiling */
 /* Kernel groups timed by the built-in profiler. */
 #define GPT2_PROF_GEMM 0        /* linear-layer contractions (fwd, dX, dW) */

@@ -86,3 +86,43 @@ def test_no_reports_while_a_step_is_recorded(torch):
     assert seen == list(range(TINY.n_layer + 1))
     gm.set_bucket_callback(None)
     gm.close()
+
+
+def test_library_exchange_one_rank_is_exact(torch):
+    """gpt2_dp_init over one rank (NCCL): every bucket's all-reduce (average)
+    is an identity, so the exchanging backward, and steps recorded as a graph
+    with the exchange inside, must give bit for bit what the same calls give
+    without it; and dp_sync(0) must leave the exchange out."""
+    import decoder_only_lm_b200 as g
+    om, named, stream, x, y = inputs(RAGGED)
+    xs, ys = torch.from_numpy(x).cuda(), torch.from_numpy(y).cuda()
+
+    def grads(model):
+        model.zero_grad()
+        model.forward_loss(xs, ys, loss=False)
+        model.backward()
+        model.synchronize()
+        return model.arena(g.GRAD).clone()
+
+    ref = gpu_model(RAGGED, True)
+    ref.set_params(named)
+    gm = gpu_model(RAGGED, True)
+    gm.set_params(named)
+    gm.dp_init(g.dp_unique_id(), 0, 1)
+    assert torch.equal(grads(gm), grads(ref))
+    gm.dp_sync(False)
+    assert torch.equal(grads(gm), grads(ref))
+    gm.dp_sync(True)
+    # two optimizer steps of two micro-batches each, replayed from the graph
+    bt = RAGGED.B * RAGGED.T
+    s = synth.uniform_stream(7, 6 * bt + 1, RAGGED.vocab_size)
+    ds = torch.from_numpy(s.astype(np.int16).view(np.int16)).cuda()
+    for m in (ref, gm):
+        m.stream_begin(ds, 0, bt, RAGGED.B, RAGGED.T, accum=2)
+        m.stream_steps([6e-4, 5e-4])
+        assert m.stream_end() == 4 * bt
+    for name in ("wte", "h.0.attn.qkv.w", "h.1.mlp.proj.b", "lnf.w"):
+        assert np.array_equal(gm.get_tensor(name), ref.get_tensor(name)), name
+    assert gm.step == ref.step == 2
+    gm.close()
+    ref.close()
