@@ -25,6 +25,7 @@
 #include <string>
 #include <vector>
 
+#include "dp_internal.h"
 #include "kernels.h"
 
 namespace gpt2_internal {

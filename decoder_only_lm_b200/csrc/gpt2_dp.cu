@@ -26,6 +26,7 @@
 #include <mutex>
 #include <string>
 
+#include "dp_internal.h"
 #include "kernels.h"
 
 namespace {

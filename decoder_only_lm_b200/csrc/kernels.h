@@ -166,15 +166,3 @@ bool gemm_tc_supported(const GemmArgs& g);
 
 // device error word of the op-level calls (bounded waits)
 int* device_error_word();
-
-// ---------------------------------------------------------------- data parallel
-#include <utility>
-#include <vector>
-namespace gpt2_internal {
-// NCCL communicator over `world` ranks from a unique id (GPT2_DP_ID_BYTES)
-int dp_comm_init(void** comm, const char* id, int rank, int world);
-void dp_comm_destroy(void* comm);
-// in-place average over the ranks of grad[off .. off + n) for each (off, n), on st
-int dp_allreduce_ranges(void* comm, const std::vector<std::pair<int64_t, int64_t>>& ranges,
-                        float* grad, cudaStream_t st);
-}  // namespace gpt2_internal
