@@ -462,6 +462,7 @@ def main():
     lrs = [hp_at(i)["lr"] for i in range(steps_total)]
     model.stream_begin(stream, rank * B * T, world * B * T, B, T, accum=acc,
                        **{k: v for k, v in HP.items() if k != "lr"})
+    kernels_per_step = model.stream_kernels()  # what each replay launches
     model.stream_steps(lrs[:args.warmup])
     model.synchronize()
     torch.cuda.synchronize()
@@ -626,7 +627,11 @@ def main():
                                 "measured_peak_source": peak_src}},
             "roofline": roof,
             "clocks": clk,
-            "gpu_launches": prof["total_launches"],
+            # kernels launched in the timed region: the step graph's kernels, once per
+            # replayed step (the per-call profiled repeat launches the same set)
+            "gpu_launches": kernels_per_step * args.steps,
+            "gpu_launches_per_step": kernels_per_step,
+            "profiled_pass_launches": prof["total_launches"],
             "profiled_pass_ms_per_step": sum(v["ms"] for v in groups.values()) / args.steps,
             "kernel_groups_ms_per_step": {k: round(v["ms"] / args.steps, 4) for k, v in groups.items()},
             "e2e": e2e,

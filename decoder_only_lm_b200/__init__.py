@@ -68,6 +68,7 @@ SIGNATURES = {
     "gpt2_stream_begin": (_i, [_P, _P, _i64, _i64, _i64, _i, _i, _i, _f, _f, _f, _f, _f]),
     "gpt2_stream_steps": (_i, [_P, _i, C.POINTER(_f)]),
     "gpt2_stream_end": (_i, [_P, C.POINTER(_i64)]),
+    "gpt2_stream_kernels": (_i, [_P, C.POINTER(_i64)]),
     "gpt2_synchronize": (_i, [_P]),
     "gpt2_arena": (_i, [_P, _i, C.POINTER(C.POINTER(_f)), C.POINTER(_i64)]),
     "gpt2_arena_layout": (_i, [C.POINTER(Config), _i, C.c_char_p, _i, C.POINTER(_i64),
@@ -336,6 +337,12 @@ class GPT2:
         """gpt2_stream_steps: one replayed optimizer step per learning rate in lrs."""
         arr = (C.c_float * len(lrs))(*[float(v) for v in lrs])
         _check(lib.gpt2_stream_steps(self.h, len(lrs), arr), self.h)
+
+    def stream_kernels(self):
+        """gpt2_stream_kernels: kernels one replay of the recorded step runs."""
+        n = C.c_int64()
+        _check(lib.gpt2_stream_kernels(self.h, C.byref(n)), self.h)
+        return n.value
 
     def stream_end(self):
         """gpt2_stream_end: returns the cursor (offset of the next window)."""

@@ -147,6 +147,7 @@ struct gpt2_handle {
   Cat cats[GPT2_PROF_NCAT];
   std::vector<cudaEvent_t> ev_pool;
   int64_t launches_total = 0;
+  int64_t graph_kernels = 0;  // kernel launches recorded into the step graph
 
   size_t act_size() const { return use_bf16 ? 2 : 4; }
 };
@@ -1340,8 +1341,10 @@ int gpt2_stream_begin(gpt2_handle* h, const uint16_t* d_stream, int64_t stream_l
   cudaError_t ec = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
   if (ec == cudaSuccess) {
     h->capturing = true;
+    const int64_t k0 = gpt2_internal::launches();
     rc = stream_step_body(h, d_stream, stream_len, stride, B, T, accum, beta1, beta2, eps,
                           weight_decay, max_norm);
+    h->graph_kernels = gpt2_internal::launches() - k0;
     h->capturing = false;
     ec = cudaStreamEndCapture(cs, &g);
   }
@@ -1367,6 +1370,12 @@ int gpt2_stream_steps(gpt2_handle* h, int n_steps, const float* lr) {
     H_CUDA(h, cudaGraphLaunch(h->graph_exec, h->st));
     h->launches_total += 1;
   }
+  return GPT2_OK;
+}
+
+int gpt2_stream_kernels(const gpt2_handle* h, int64_t* n) {
+  if (!h || !n) return GPT2_ERR_ARG;
+  *n = h->graph_exec ? h->graph_kernels : 0;
   return GPT2_OK;
 }
 

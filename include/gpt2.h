@@ -193,6 +193,11 @@ int gpt2_train_step(gpt2_handle* h, const int32_t* x, const int32_t* y, int B, i
                     int tokens_on_device, float lr, float beta1, float beta2, float eps,
                     float weight_decay, float max_norm, float* loss_out, float* grad_norm_out);
 
+/* Kernel launches recorded into the step graph of gpt2_stream_begin (each
+ * replay by gpt2_stream_steps runs exactly these); 0 when no step is
+ * recorded.  Host only. */
+int gpt2_stream_kernels(const gpt2_handle* h, int64_t* n);
+
 /* Training on consecutive windows of a device-resident token stream, each
  * optimizer step replayed from a CUDA graph recorded once (no counterpart on
  * the pages, which launch every operation from Python; the step itself is

@@ -48,8 +48,14 @@ def test_graph_steps_equal_eager_steps(bf16, torch):
     ge, gg = gpu_model(TINY, bf16), gpu_model(TINY, bf16)
     ge.set_params(named)
     gg.set_params(named)
+    import decoder_only_lm_b200 as g
     end = eager_steps(ge, stream, bt, accum, lrs)
+    n0 = g.launch_count()
     gg.stream_begin(stream, 0, bt, TINY.B, TINY.T, accum=accum, **HP)
+    recorded = g.launch_count() - n0
+    # every kernel issued while recording is in the graph (the bf16 weight
+    # mirror is refreshed once before recording)
+    assert gg.stream_kernels() == recorded - (1 if bf16 else 0) and gg.stream_kernels() > 50
     gg.stream_steps(lrs)
     assert gg.stream_end() == end
     assert gg.step == ge.step == len(lrs)
