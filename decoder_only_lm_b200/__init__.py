@@ -98,6 +98,7 @@ SIGNATURES = {
     "gpt2_linear": (_i, [_i, _P, _P, _i, _P, _P, _P, _P, _i, _i, _i, _i, _P, _sz, _P]),
     "gpt2_device_error": (_i, [C.POINTER(_i)]),
     "gpt2_launch_count": (_i, [C.POINTER(_i64)]),
+    "gpt2_wait_selfcheck": (_i, [C.POINTER(_i)]),
 }
 
 
@@ -619,6 +620,14 @@ def launch_count():
     n = C.c_int64()
     _check(lib.gpt2_launch_count(C.byref(n)))
     return n.value
+
+
+def wait_selfcheck():
+    """gpt2_wait_selfcheck: True when a deliberately unmet device wait gave up
+    (after its 2 s budget) and was recorded."""
+    e = C.c_int()
+    _check(lib.gpt2_wait_selfcheck(C.byref(e)))
+    return bool(e.value)
 
 
 def device_error():

@@ -510,6 +510,16 @@ int gpt2_linear(int epi, const void* x, const void* w, int w_kn, const float* bi
                 const void* in, void* out, void* out2, int M, int N, int K, int dtype,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Self-check of the bounded device waits (no counterpart on the pages: the
+ * failure handling of this library).  Every wait of the tensor-core kernels on
+ * a barrier gives up after 2 s of device time, records a timeout (read back
+ * as GPT2_ERR_TIMEOUT) and lets the kernel end.  This call runs one thread
+ * that waits for a barrier phase nothing completes, synchronises the current
+ * device (about 2 s), and sets *expired = 1 when the wait gave up and was
+ * recorded, 0 otherwise; it clears the record afterwards, so the device and
+ * the library stay usable.  Allocates 4 bytes with cudaMalloc. */
+int gpt2_wait_selfcheck(int* expired);
+
 /* Kernel launches the library has issued from the calling thread since the
  * process started, op-level calls and handle calls alike.  Kernels recorded
  * into a graph by gpt2_stream_begin count once, when recorded; replays by
