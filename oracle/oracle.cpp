@@ -565,9 +565,21 @@ int clip_adamw(const oracle_cfg* cp, S* params, const S* grads, S* m, S* v, int 
   if (!cfg_ok(cp) || t < 1) return ERR_ARG;
   auto tl = tensor_list(*cp);
   const int64_t N = param_count(*cp);
+  // the sum of squares in a fixed order, whatever the thread count: blocks
+  // of 4096 elements summed one by one, then the block sums in block order
+  // (an OpenMP reduction would combine the threads' sums in arrival order)
+  constexpr int64_t kBlk = 4096;
+  const int64_t nblk = (N + kBlk - 1) / kBlk;
+  std::vector<double> part(size_t(std::max<int64_t>(nblk, 1)), 0.0);
+#pragma omp parallel for schedule(static)
+  for (int64_t bI = 0; bI < nblk; ++bI) {
+    double acc = 0;
+    const int64_t end = std::min(N, (bI + 1) * kBlk);
+    for (int64_t i = bI * kBlk; i < end; ++i) acc += double(grads[i]) * double(grads[i]);
+    part[size_t(bI)] = acc;
+  }
   double n2 = 0;
-#pragma omp parallel for reduction(+ : n2) schedule(static)
-  for (int64_t i = 0; i < N; ++i) n2 += double(grads[i]) * double(grads[i]);
+  for (int64_t bI = 0; bI < nblk; ++bI) n2 += part[size_t(bI)];
   const double n = std::sqrt(n2);
   if (norm_out) *norm_out = n;
   if (!std::isfinite(n)) return ERR_NONFINITE;

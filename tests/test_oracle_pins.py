@@ -430,3 +430,40 @@ def test_tiny_mod17_task_learns():
         losses.append(loss)
         m.clip_adamw(p, g, mm, vv, t + 1, lr=1e-2, wd=0.0)
     assert losses[0] > 2.5 and losses[-1] < 0.5 * losses[0]
+
+
+_NORM_CHILD = r"""
+import sys, numpy as np
+sys.path.insert(0, sys.argv[1])
+import oracle, synth
+m = oracle.Model(2, 64, 4, 512, 512, 64)
+p = m.pack(synth.init_params(0, m.shapes()))
+g = synth.normal(synth.derive_key(31), p.size, 1.0).astype(np.float64)
+mm, vv = np.zeros_like(p), np.zeros_like(p)
+n = m.clip_adamw(p, g, mm, vv, 1)
+sys.stdout.write(repr(n) + " " + str(oracle.num_threads()) + " " + p.tobytes().hex()[:0])
+np.save(sys.argv[2], p)
+"""
+
+
+def test_clip_adamw_identical_for_any_thread_count(tmp_path):
+    """The gradient norm is one sum of squares over every element, taken in a
+    fixed order, so that data-parallel ranks (each applying the same averaged
+    gradient) end with bit-identical parameters: the same update computed in
+    two processes with 1 and 5 OpenMP threads must agree bit for bit."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = []
+    for nt in (1, 5):
+        f = tmp_path / f"p{nt}.npy"
+        env = dict(os.environ, OMP_NUM_THREADS=str(nt))
+        r = subprocess.run([sys.executable, "-c", _NORM_CHILD, root, str(f)], env=env,
+                           capture_output=True, text=True, timeout=120)
+        assert r.returncode == 0, r.stderr
+        norm, threads = r.stdout.split()[:2]
+        assert int(threads) == nt
+        out.append((norm, np.load(f)))
+    assert out[0][0] == out[1][0]
+    assert np.array_equal(out[0][1], out[1][1])
