@@ -23,8 +23,10 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <type_traits>
 #include <vector>
 
+#include "attn_internal.h"
 #include "dp_internal.h"
 #include "kernels.h"
 
@@ -108,6 +110,7 @@ struct gpt2_handle {
   cudaStream_t st2 = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_join2 = nullptr;
   float* ws2 = nullptr;
+  bf16* ads = nullptr;  // attention score gradients (bf16 tcgen05 path), one layer at a time
   void* ws_emb = nullptr;
   double* ws_norm = nullptr;
   DevStatus* status = nullptr;
@@ -708,8 +711,12 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     }
     {
       PROF(GPT2_PROF_ATTN_BWD, attn_bwd_flops, a * 9.0 * M * C + 8.0 * M * Hh);
-      H_TRY(h, launch_attn_bwd<A>(datt, static_cast<A*>(h->qkv[l]), static_cast<A*>(h->att[l]),
-                                  h->alse[l], B, T, C, Hh, dqkv, h->ws, h->st));
+      if constexpr (std::is_same<A, bf16>::value)
+        H_TRY(h, launch_attn_bwd_ds(datt, static_cast<A*>(h->qkv[l]), static_cast<A*>(h->att[l]),
+                                    h->alse[l], B, T, C, Hh, dqkv, h->ws, h->ads, h->st));
+      else
+        H_TRY(h, launch_attn_bwd<A>(datt, static_cast<A*>(h->qkv[l]), static_cast<A*>(h->att[l]),
+                                    h->alse[l], B, T, C, Hh, dqkv, h->ws, h->st));
       H_TRY(h, sd.join());  // attn.proj's weight gradient ran beside the attention backward
     }
     {
@@ -847,6 +854,8 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
   h->ws_bytes = ws;
   h->ws = static_cast<float*>(A(ws));
   h->ws2 = static_cast<float*>(A(ws));
+  if (h->use_bf16 && attn_tc_supported(c.max_B, c.max_Tseq, int(C), H))
+    h->ads = static_cast<bf16*>(A(attn_tc_ds_bytes(c.max_B, c.max_Tseq, H)));
   h->ws_emb = A(embed_bwd_workspace(M, int(C)));
   h->ws_norm = static_cast<double*>(A(gradnorm_workspace()));
   h->status = static_cast<DevStatus*>(A(sizeof(DevStatus)));

@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <string>
 
+#include "attn_internal.h"
 #include "kernels.h"
 
 using gpt2_internal::set_error;
@@ -134,10 +135,8 @@ int gpt2_attention_fwd(const void* qkv, int dtype, int B, int T, int C, int H, v
 }
 
 int gpt2_attention_bwd_workspace(int B, int T, int C, int H, int dtype, size_t* bytes) {
-  (void)C;
-  (void)dtype;
   if (!bytes || B < 1 || T < 1 || H < 1) return GPT2_ERR_ARG;
-  *bytes = attn_bwd_workspace(B, T, H);
+  *bytes = attn_bwd_workspace_total(B, T, C, H, dtype == GPT2_BF16);
   return GPT2_OK;
 }
 
@@ -145,16 +144,22 @@ int gpt2_attention_bwd(const void* dout, const void* qkv, const void* out, const
                        int dtype, int B, int T, int C, int H, void* dqkv, void* workspace,
                        size_t workspace_bytes, void* stream) {
   if (!dout || !qkv || !out || !lse || !dqkv || B < 1 || T < 1 || H < 1 || C % H || !workspace ||
-      workspace_bytes < attn_bwd_workspace(B, T, H)) {
+      workspace_bytes < attn_bwd_workspace_total(B, T, C, H, dtype == GPT2_BF16)) {
     set_error("attention_bwd: bad arguments or workspace too small");
     return GPT2_ERR_ARG;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
-  if (dtype == GPT2_BF16)
-    return launch_attn_bwd<bf16>(static_cast<const bf16*>(dout), static_cast<const bf16*>(qkv),
-                                 static_cast<const bf16*>(out), lse, B, T, C, H,
-                                 static_cast<bf16*>(dqkv), ws, st);
+  if (dtype == GPT2_BF16) {
+    // the score-gradient buffer follows Delta when the workspace holds one
+    const size_t delta = (attn_bwd_workspace(B, T, H) + 1023) / 1024 * 1024;
+    bf16* ds = attn_bwd_workspace_total(B, T, C, H, true) > attn_bwd_workspace(B, T, H)
+                   ? reinterpret_cast<bf16*>(static_cast<char*>(workspace) + delta)
+                   : nullptr;
+    return launch_attn_bwd_ds(static_cast<const bf16*>(dout), static_cast<const bf16*>(qkv),
+                              static_cast<const bf16*>(out), lse, B, T, C, H,
+                              static_cast<bf16*>(dqkv), ws, ds, st);
+  }
   if (dtype == GPT2_F32)
     return launch_attn_bwd<float>(static_cast<const float*>(dout), static_cast<const float*>(qkv),
                                   static_cast<const float*>(out), lse, B, T, C, H,

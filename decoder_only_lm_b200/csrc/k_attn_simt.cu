@@ -9,6 +9,7 @@
 // and dq kernel (one thread per query) both recompute p_ij, so no two threads
 // add into the same element and the result is deterministic.
 
+#include "attn_internal.h"
 #include "kernels.h"
 
 namespace {
@@ -322,11 +323,10 @@ template int launch_attn_simt_bwd<bf16>(const bf16*, const bf16*, const bf16*, c
 
 // Dispatch: bf16 with head size 64 runs on the tcgen05 kernels (k_attn_tc.cu);
 // fp32 (the parity mode) and other head sizes run on the kernels above.
-bool attn_tc_supported(int B, int T, int C, int H);
 int launch_attn_tc_fwd(const bf16* qkv, int B, int T, int C, int H, bf16* out, float* lse,
                        cudaStream_t st);
 int launch_attn_tc_bwd(const bf16* dout, const bf16* qkv, const float* lse, const float* delta,
-                       int B, int T, int C, int H, bf16* dqkv, cudaStream_t st);
+                       int B, int T, int C, int H, bf16* dqkv, bf16* ds, cudaStream_t st);
 
 template <>
 int launch_attn_fwd<float>(const float* qkv, int B, int Tn, int C, int H, float* out, float* lse,
@@ -344,13 +344,22 @@ int launch_attn_bwd<float>(const float* dout, const float* qkv, const float* out
                            int B, int Tn, int C, int H, float* dqkv, float* ws, cudaStream_t st) {
   return launch_attn_simt_bwd<float>(dout, qkv, out, lse, B, Tn, C, H, dqkv, ws, st);
 }
-template <>
-int launch_attn_bwd<bf16>(const bf16* dout, const bf16* qkv, const bf16* out, const float* lse,
-                          int B, int Tn, int C, int H, bf16* dqkv, float* ws, cudaStream_t st) {
+int launch_attn_bwd_ds(const bf16* dout, const bf16* qkv, const bf16* out, const float* lse, int B,
+                       int Tn, int C, int H, bf16* dqkv, float* ws, bf16* ds, cudaStream_t st) {
   if (!attn_tc_supported(B, Tn, C, H))
     return launch_attn_simt_bwd<bf16>(dout, qkv, out, lse, B, Tn, C, H, dqkv, ws, st);
   const int64_t rows = int64_t(B) * H * Tn;
   attn_delta64_kernel<<<int(cdiv64(rows * 8, 256)), 256, 0, st>>>(dout, out, B, Tn, C, H, ws);
   COUNT_LAUNCH(1);
-  return launch_attn_tc_bwd(dout, qkv, lse, ws, B, Tn, C, H, dqkv, st);
+  return launch_attn_tc_bwd(dout, qkv, lse, ws, B, Tn, C, H, dqkv, ds, st);
+}
+template <>
+int launch_attn_bwd<bf16>(const bf16* dout, const bf16* qkv, const bf16* out, const float* lse,
+                          int B, int Tn, int C, int H, bf16* dqkv, float* ws, cudaStream_t st) {
+  return launch_attn_bwd_ds(dout, qkv, out, lse, B, Tn, C, H, dqkv, ws, nullptr, st);
+}
+size_t attn_bwd_workspace_total(int B, int T, int C, int H, bool bf16_path) {
+  const size_t delta = attn_bwd_workspace(B, T, H);
+  if (!bf16_path || H < 1 || C % H || !attn_tc_supported(B, T, C, H)) return delta;
+  return (delta + 1023) / 1024 * 1024 + attn_tc_ds_bytes(B, T, H);
 }

@@ -30,10 +30,15 @@
 //   dK/dV kernel (per 128 keys, 64-query tiles i >= keys): S^T, dP^T = V dO^T,
 //   dS^T = P^T (dP^T - Delta); dV += P^T dO, dK += dS^T Q / sqrt(D);
 //   dQ kernel (per 128 queries, 64-key tiles): S, dP, dS; dQ += dS K / sqrt(D).
-// Both recompute P, so no two CTAs add into one element (deterministic).
+//   With a score-gradient buffer the dK/dV kernel also writes dS^T (bf16, the
+//   values its dK MMA takes) and dQ is one contraction over it (no
+//   exponentials, no second S or dP); without one (the no-allocation entry
+//   point) the dQ kernel recomputes P and dS as above.
+// Every output element is written by one CTA, no atomics (deterministic).
 // Every wait is bounded (2 s of global time) and reports a timeout in the
 // error word instead of hanging.
 
+#include "attn_internal.h"
 #include "tc_common.cuh"
 
 using namespace tc;
@@ -355,6 +360,12 @@ struct BwdParams {
   const float* lse;
   const float* delta;
   bf16* dqkv;
+  // score gradients kept for the dQ contraction (null: the dQ kernel
+  // recomputes them): dS^T in 128 x 128 bf16 tiles [key][query], one per
+  // (key block kb, query block qb >= kb), tile kb + qb (qb + 1) / 2 of
+  // (batch, head) b * H + h, ntri = nqb (nqb + 1) / 2 tiles per (batch, head)
+  bf16* dst;
+  int ntri;
   int* err;
 };
 
@@ -366,20 +377,35 @@ struct BwdParams {
 // step i: dV(i-1) (after P^T_{i-1} is written); S^T_i; dK(i-1) (after dS^T_{i-1});
 // dP^T_i: each MMA that overwrites a TMEM region is issued after the one
 // that last reads it.
-constexpr int NSK = 4;  // Q/dO stages
-constexpr int kDkdvSmem = 2 * kRowTile + NSK * 2 * kStrTile + 2 * BS * 4 + 256 + 1024;
+// KEEP: the warpgroup writes dS^T_i (bf16) into a 128-byte-swizzled 16 KB
+// shared-memory tile instead of TMEM; dK += dS^T_i Q_i reads it from there
+// (A K-major) and the MMA thread stores it into the score-gradient buffer with
+// one TMA store, then waits for that store to have read the tile and tells the
+// warpgroup (ds_free) that tile i+1 may be written.  The tile takes one Q/dO
+// stage, so that two CTAs still share an SM.
+template <bool KEEP>
+struct DkdvCfg {
+  static constexpr int NSK = KEEP ? 3 : 4;  // Q/dO stages
+  static constexpr int kStage = KEEP ? kRowTile : 0;
+  static constexpr int kSmem = 2 * kRowTile + NSK * 2 * kStrTile + kStage + 2 * BS * 4 + 256 + 1024;
+};
 
+template <bool KEEP>
 __global__ void __launch_bounds__(kThreads, 2)
     fa_tc_dkdv_kernel(const __grid_constant__ CUtensorMap q128, const __grid_constant__ CUtensorMap q64,
-                      const __grid_constant__ CUtensorMap o64, const BwdParams p) {
+                      const __grid_constant__ CUtensorMap o64, const __grid_constant__ CUtensorMap ds_map,
+                      const BwdParams p) {
+  constexpr int NSK = DkdvCfg<KEEP>::NSK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sK = smem_u32(smem), sV = sK + kRowTile;
   const uint32_t sQ = sV + kRowTile;            // NSK x 8 KB
   const uint32_t sO = sQ + NSK * kStrTile;      // dO, NSK x 8 KB
-  float* sLD = reinterpret_cast<float*>(smem + 2 * kRowTile + 2 * NSK * kStrTile);  // [64] -lse*log2e, [64] -delta
+  uint8_t* sDs = smem + 2 * kRowTile + 2 * NSK * kStrTile;  // KEEP: dS^T, 128 x 64 bf16
+  float* sLD = reinterpret_cast<float*>(sDs + DkdvCfg<KEEP>::kStage);  // [64] -lse*log2e, [64] -delta
   uint64_t* bars = reinterpret_cast<uint64_t*>(sLD + 2 * BS);
-  // kv_full | qo_full[NSK] | qo_empty[NSK] | s_full | p_full | dp_full | ds_full | mm_done | slot
+  // kv_full | qo_full[NSK] | qo_empty[NSK] | s_full | p_full | dp_full | ds_full | mm_done |
+  // ds_free | slot
   const uint32_t b_kv = smem_u32(bars);
   auto b_qf = [&](int s) { return smem_u32(bars + 1 + s); };
   auto b_qe = [&](int s) { return smem_u32(bars + 1 + NSK + s); };
@@ -388,7 +414,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t b_dpf = smem_u32(bars + 3 + 2 * NSK);
   const uint32_t b_df = smem_u32(bars + 4 + 2 * NSK);
   const uint32_t b_mm = smem_u32(bars + 5 + 2 * NSK);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * NSK);
+  const uint32_t b_dsf = smem_u32(bars + 6 + 2 * NSK);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * NSK);
 
   const int kb = blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -410,6 +437,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(b_dpf, 1);
     mbar_init(b_df, 128);
     mbar_init(b_mm, 1);
+    mbar_init(b_dsf, 1);
     init_bar_fence();
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -472,16 +500,32 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
-        mma_ts4(tKd, tP, desc_offset(dQm, si * kStrTile), id_o, 128, i > 1);
+        if (KEEP) {
+          mma_ss4(tKd, desc_kmajor(smem_u32(sDs), 0), desc_offset(dQm, si * kStrTile), id_o, 2,
+                  128, i > 1);
+        } else {
+          mma_ts4(tKd, tP, desc_offset(dQm, si * kStrTile), id_o, 128, i > 1);
+        }
         umma_commit(b_mm);
         umma_commit(b_qe(si));
         ++mm;
+        if (KEEP) {  // dS^T_{i-1} into its tile of the score-gradient buffer
+          const int qt = qt0 + i - 1, qbt = qt >> 1;
+          const int y = int((int64_t(b * p.H + h) * p.ntri + qbt * (qbt + 1) / 2 + kb) * BR);
+          tma_store_2d(&ds_map, smem_u32(sDs), (qt & 1) * BS, y);
+          bulk_commit();
+        }
       }
       if (i < n) {  // dP^T_i = V dO_i^T
         mma_ss4(tP, dV, desc_offset(dO, s * kStrTile), id_s, 2, 2, false);
         umma_commit(b_dpf);
+        if (KEEP && i >= 1) {  // the store of dS^T_{i-1} has read the tile
+          bulk_wait_read<0>();
+          mbar_arrive(b_dsf);
+        }
       }
     }
+    if (KEEP) bulk_wait_all();
     if (mm > 0) mbar_wait(b_mm, uint32_t((mm - 1) & 1), p.err, 26);
   } else if (warp >= 2) {
     const int e = (warp & 3) * 32 + lane;  // key row in the block = TMEM lane
@@ -563,8 +607,20 @@ __global__ void __launch_bounds__(kThreads, 2)
           pd[qc >> 1] = pack2(g0, g1);
         }
       }
-      tmem_st32_async(tP + lo, pd);  // dS^T over the first 32 columns of dP^T
-      tmem_wait_st();
+      if (KEEP) {
+        // row e of the dS^T tile (K-major, 128-byte swizzle), once the dK MMA
+        // (done before dP^T_i) and the store of dS^T_{i-1} have read it
+        if (i > 0 && ok) ok = mbar_wait(b_dsf, (i - 1) & 1, p.err, 30);
+        uint8_t* row = sDs + e * 128;
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          *reinterpret_cast<uint4*>(row + ((v ^ (e & 7)) << 4)) =
+              make_uint4(pd[4 * v], pd[4 * v + 1], pd[4 * v + 2], pd[4 * v + 3]);
+        fence_proxy_async();  // visible to the MMA and the bulk copy
+      } else {
+        tmem_st32_async(tP + lo, pd);  // dS^T over the first 32 columns of dP^T
+        tmem_wait_st();
+      }
       tc_fence_before();
       mbar_arrive(b_df);
       wg_bar();  // sLD may be rewritten for the next tile
@@ -806,7 +862,111 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---------------------------------------------------------------- dQ from kept dS
+// With the score gradients kept by the dK/dV kernel, dQ is a plain contraction,
+// dQ_i = sum_j dS_ij K_j / sqrt(D), with no exponentials and no recomputed S
+// or dP.  CTA: 128 queries, 64-key steps up to the diagonal; one TMA stage =
+// dS^T of the 64 keys x 128 queries (two 64-query chunks: A MN-major) and K_j
+// (64 keys x 64 channels: B MN-major); TMEM: one 128 x 64 fp32 accumulator.
+constexpr int NSG = 3;                            // stages (three CTAs per SM)
+constexpr int kGStage = kRowTile + kStrTile;      // 16 KB dS^T + 8 KB K
+constexpr int kDqgSmem = NSG * kGStage + 256 + 1024;
+constexpr int kDqgTmemCols = 64;
+
+__global__ void __launch_bounds__(kThreads, 3)
+    fa_tc_dq_ds_kernel(const __grid_constant__ CUtensorMap ds_map,
+                       const __grid_constant__ CUtensorMap q64, const BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NSG * kGStage);
+  // full[NSG] | empty[NSG] | acc_done | slot
+  auto b_full = [&](int s) { return smem_u32(bars + s); };
+  auto b_empty = [&](int s) { return smem_u32(bars + NSG + s); };
+  const uint32_t b_acc = smem_u32(bars + 2 * NSG);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NSG + 1);
+  const int qb = gridDim.x - 1 - blockIdx.x;
+  // (batch, head) in the reverse of the dK/dV kernel's launch order: the first
+  // CTAs read the score gradients written last, the ones most likely in L2
+  const int h = gridDim.y - 1 - blockIdx.y, b = gridDim.z - 1 - blockIdx.z;
+  const int T = p.T, C = p.C;
+  const int last_key = min(T, (qb + 1) * BR) - 1;
+  const int nkt = last_key / BS + 1;
+  const int row_base = b * T;
+  const int64_t tile0 = (int64_t(b) * p.H + h) * p.ntri + qb * (qb + 1) / 2;  // (kb 0, qb)
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSG; ++s) {
+      mbar_init(b_full(s), 1);
+      mbar_init(b_empty(s), 1);
+    }
+    mbar_init(b_acc, 1);
+    init_bar_fence();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kDqgTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp == 0 && lane == 0) {
+    int issued = 0;
+    for (int j = 0; j < nkt; ++j) {
+      const int s = j % NSG;
+      if (!mbar_wait(b_empty(s), ((j / NSG) & 1) ^ 1, p.err, 41)) break;
+      const uint32_t sa = sbase + s * kGStage;
+      const int y = int((tile0 + (j >> 1)) * BR + (j & 1) * BS);  // first key row of step j
+      mbar_expect_tx(b_full(s), kGStage);
+      tma_load_2d(sa, &ds_map, b_full(s), 0, y);
+      tma_load_2d(sa + BK * 128, &ds_map, b_full(s), BS, y);
+      tma_load_2d(sa + kRowTile, &q64, b_full(s), C + h * D, row_base + j * BS);
+      ++issued;
+    }
+    for (int q = 1; q <= min(issued, NSG); ++q) {
+      const int idx = issued - q;
+      mbar_wait(b_full(idx % NSG), uint32_t((idx / NSG) & 1), p.err, 45);
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t id = idesc_bf16(BR, D, 1, 1);
+    const uint64_t dA = desc_mnmajor(sbase, 0), dB = desc_mnmajor(sbase + kRowTile, 0);
+    for (int j = 0; j < nkt; ++j) {
+      const int s = j % NSG;
+      if (!mbar_wait(b_full(s), (j / NSG) & 1, p.err, 42)) break;
+      tc_fence_after();
+      mma_ss4(tmem, desc_offset(dA, s * kGStage), desc_offset(dB, s * kGStage), id, 128, 128,
+              j > 0);
+      umma_commit(b_empty(s));
+    }
+    // tracks every MMA issued, so the accumulator is released only after them
+    umma_commit(b_acc);
+    mbar_wait(b_acc, 0, p.err, 43);
+  } else if (warp >= 2) {
+    const int e = (warp & 3) * 32 + lane;  // query row in the block = TMEM lane
+    const int q = qb * BR + e;
+    const uint32_t lo = uint32_t((warp & 3) * 32) << 16;
+    const bool w = mbar_wait(b_acc, 0, p.err, 44);
+    if (__all_sync(0xffffffffu, w)) {
+      tc_fence_after();
+      uint32_t a0[32], a1[32];
+      tmem_ld32_async(tmem + lo, a0);
+      tmem_ld32_async(tmem + lo + 32, a1);
+      tmem_wait_ld(a0);
+      reg_after_wait(a1);
+      if (q < T)
+        store_row64(p.dqkv + (int64_t(row_base) + q) * 3 * C + h * D, a0, a1, rsqrtf(float(D)));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kDqgTmemCols);
+}
+
 }  // namespace
+
+size_t attn_tc_ds_bytes(int B, int T, int H) {
+  const int64_t nqb = cdiv(T, BR);
+  return size_t(B) * H * (nqb * (nqb + 1) / 2) * BR * BR * sizeof(bf16);
+}
 
 bool attn_tc_supported(int B, int T, int C, int H) {
   return C / H == D && C % H == 0 && C % 8 == 0 && int64_t(B) * T < (int64_t(1) << 31);
@@ -835,12 +995,22 @@ int launch_attn_tc_fwd(const bf16* qkv, int B, int T, int C, int H, bf16* out, f
 }
 
 int launch_attn_tc_bwd(const bf16* dout, const bf16* qkv, const float* lse, const float* delta,
-                       int B, int T, int C, int H, bf16* dqkv, cudaStream_t st) {
+                       int B, int T, int C, int H, bf16* dqkv, bf16* ds, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(fa_tc_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDkdvSmem);
+    cudaFuncSetAttribute(fa_tc_dkdv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         DkdvCfg<false>::kSmem);
+    cudaFuncSetAttribute(fa_tc_dkdv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         DkdvCfg<true>::kSmem);
     cudaFuncSetAttribute(fa_tc_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
+    cudaFuncSetAttribute(fa_tc_dq_ds_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqgSmem);
     attr = true;
+  }
+  const int nqb = cdiv(T, BR), ntri = nqb * (nqb + 1) / 2;
+  const int64_t ds_rows = int64_t(B) * H * ntri * BR;
+  if (ds && (reinterpret_cast<uintptr_t>(ds) % 16 || ds_rows >= (int64_t(1) << 31))) {
+    gpt2_internal::set_error("attention: score-gradient buffer misaligned or too large");
+    return GPT2_ERR_ARG;
   }
   CUtensorMap q128, q64, o128, o64;
   const int64_t rows = int64_t(B) * T;
@@ -851,11 +1021,24 @@ int launch_attn_tc_bwd(const bf16* dout, const bf16* qkv, const float* lse, cons
     gpt2_internal::set_error("attention: tensor map encoding failed");
     return GPT2_ERR_CUDA;
   }
-  BwdParams p{T, C, H, lse, delta, dqkv, device_error_word()};
-  dim3 grid(cdiv(T, BR), H, B);
-  fa_tc_dkdv_kernel<<<grid, kThreads, kDkdvSmem, st>>>(q128, q64, o64, p);
-  COUNT_LAUNCH(1);
-  fa_tc_dq_kernel<<<grid, kThreads, kDqSmem, st>>>(q128, q64, o128, p);
+  // score-gradient buffer: stored as 128-key x 64-query boxes, read as 64 x 64
+  CUtensorMap ds_st, ds_ld;
+  if (ds && (!make_map_bf16(&ds_st, ds, BR, ds_rows, BR, BR) ||
+             !make_map_bf16(&ds_ld, ds, BR, ds_rows, BR, BS))) {
+    gpt2_internal::set_error("attention: tensor map encoding failed");
+    return GPT2_ERR_CUDA;
+  }
+  BwdParams p{T, C, H, lse, delta, dqkv, ds, ntri, device_error_word()};
+  dim3 grid(nqb, H, B);
+  if (ds) {
+    fa_tc_dkdv_kernel<true><<<grid, kThreads, DkdvCfg<true>::kSmem, st>>>(q128, q64, o64, ds_st, p);
+    COUNT_LAUNCH(1);
+    fa_tc_dq_ds_kernel<<<grid, kThreads, kDqgSmem, st>>>(ds_ld, q64, p);
+  } else {
+    fa_tc_dkdv_kernel<false><<<grid, kThreads, DkdvCfg<false>::kSmem, st>>>(q128, q64, o64, q64, p);
+    COUNT_LAUNCH(1);
+    fa_tc_dq_kernel<<<grid, kThreads, kDqSmem, st>>>(q128, q64, o128, p);
+  }
   COUNT_LAUNCH(1);
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;

@@ -445,7 +445,12 @@ int gpt2_attention_fwd(const void* qkv, int dtype, int B, int T, int C, int H, v
 
 /* Backward of gpt2_attention_fwd: dqkv [B,T,3C] (overwritten) from dout
  * [B,T,C], qkv, out and lse of the forward.  workspace >=
- * gpt2_attention_bwd_workspace(). */
+ * gpt2_attention_bwd_workspace(), device memory owned by the caller: one
+ * float per (batch, head, position) for Delta = rowsum(dO o O), and, for bf16
+ * with head size 64, after it (at a 1 KB offset) the causal half of the score
+ * gradients dS in bf16 (B*H*n(n+1)/2 tiles of 128 x 128, n = ceil(T/128);
+ * 226 MB at B=16, T=1024, H=12), written by the dK/dV step and read by the dQ
+ * step instead of recomputing them.  GPT2_ERR_ARG if the workspace is smaller. */
 int gpt2_attention_bwd_workspace(int B, int T, int C, int H, int dtype, size_t* bytes);
 int gpt2_attention_bwd(const void* dout, const void* qkv, const void* out, const float* lse,
                        int dtype, int B, int T, int C, int H, void* dqkv, void* workspace,

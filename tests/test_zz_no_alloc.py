@@ -27,9 +27,12 @@ def test_noalloc_matches_workspace_entry_point(bf16):
     assert torch.cuda.is_available()
     dt = torch.bfloat16 if bf16 else torch.float32
     tol = 3e-2 if bf16 else 1e-4
-    # head size 64 (the tensor-core kernels in bf16), then head size 32 (the
-    # CUDA-core kernels, which read the same fixed scratch)
-    for call, (B, T, C, H) in enumerate([(2, 200, 128, 2), (3, 77, 128, 2), (2, 100, 64, 2)]):
+    # head size 64 (the tensor-core kernels in bf16: here dQ recomputes the
+    # score gradients, where the workspace entry point keeps them from the
+    # dK/dV kernel), then head size 32 (the CUDA-core kernels, which read the
+    # same fixed scratch)
+    shapes = [(2, 200, 128, 2), (3, 77, 128, 2), (2, 1024, 768, 12), (2, 100, 64, 2)]
+    for call, (B, T, C, H) in enumerate(shapes):
         rng = np.random.default_rng(100 + call)
         qkv = torch.from_numpy(rng.normal(size=(B, T, 3 * C)).astype(np.float32)).cuda().to(dt)
         dout = torch.from_numpy(rng.normal(size=(B, T, C)).astype(np.float32)).cuda().to(dt)
