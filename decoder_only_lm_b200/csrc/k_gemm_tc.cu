@@ -642,8 +642,10 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
         }
         row_put<OutT>(b0, e, v);
       } else if constexpr (EPI == EPI_ACC) {
+        if (!p.ws) {  // split partial sums stay raw (alpha applied by the reduction)
 #pragma unroll
-        for (int j = 0; j < CW; ++j) v[j] *= ep.alpha;
+          for (int j = 0; j < CW; ++j) v[j] *= ep.alpha;
+        }
         row_put<OutT>(b0, e, v);
       } else if constexpr (EPI == EPI_CE_GRAD) {
         const float cs = ep.ce_scale, l2 = row_l * kLog2e;
@@ -666,7 +668,9 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
       epi_bar(bar_id);
       if (leader) {
         const uint32_t src = eb + slot * T::ARR * 8192;
-        if (EPI == EPI_ACC && ep.accumulate)
+        if (EPI == EPI_ACC && p.ws)  // split sp's partial: rows sp * M .. of [splits * M, N]
+          tma_store_2d(mo, src, n0, m0 + sp * p.M);
+        else if (EPI == EPI_ACC && ep.accumulate)
           tma_reduce_add_2d(mo, src, n0, m0);
         else
           tma_store_2d(mo, src, n0, m0);
@@ -1062,10 +1066,17 @@ int pair_slots() {
 }
 
 // The TMA epilogue needs 16-byte aligned arrays and rows (tensor-map rules);
-// split-K partial tiles and the LSE-partial epilogue use the staged path.
+// split-K partial tiles (but those of weight gradients over whole 256-row
+// tiles) and the LSE-partial epilogue use the staged path.
 bool te_eligible(const GemmArgs& g, int splits) {
-  if (splits != 1 || g.ep.kind == EPI_LSE_PARTIAL) return false;
   auto al16 = [](const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  if (splits != 1) {
+    // fp32 weight-gradient partial sums by TMA into the workspace viewed as
+    // [splits * M, N]: whole 256-row tiles only, so no tile reaches into the
+    // next split's rows
+    return g.ep.kind == EPI_ACC && g.M % BM2 == 0 && (g.N * 4) % 16 == 0 && al16(g.ws);
+  }
+  if (g.ep.kind == EPI_LSE_PARTIAL) return false;
   const int eb = (g.ep.kind == EPI_RESID || g.ep.kind == EPI_ACC || !g.ep.out_bf16) ? 4 : 2;
   if ((g.ep.ldo * eb) % 16 != 0) return false;
   switch (g.ep.kind) {
@@ -1101,7 +1112,10 @@ int launch_tc(const GemmArgs& g, int splits, cudaStream_t st) {
   if (TE) {
     constexpr int eb = int(sizeof(OutT));
     const void* o = EPI == EPI_RESID ? static_cast<const void*>(g.ep.rout) : g.ep.out;
-    ok = ok && tc::make_map_epi(&mo, o, eb, g.N, g.M, g.ep.ldo);
+    if (EPI == EPI_ACC && splits > 1)
+      ok = ok && tc::make_map_epi(&mo, g.ws, 4, g.N, int64_t(splits) * g.M, g.N);
+    else
+      ok = ok && tc::make_map_epi(&mo, o, eb, g.N, g.M, g.ep.ldo);
     if (EPI == EPI_GELU) ok = ok && tc::make_map_epi(&mo2, g.ep.out2, eb, g.N, g.M, g.ep.ldo);
     if (EPI == EPI_RESID) ok = ok && tc::make_map_epi(&mi, g.ep.rin, 4, g.N, g.M, g.ep.ldo);
     if (EPI == EPI_GELU_BWD) ok = ok && tc::make_map_epi(&mi, g.ep.aux, eb, g.N, g.M, g.ep.ldo);
