@@ -17,8 +17,19 @@ size_t attn_tc_ds_bytes(int B, int T, int H);
 // contraction over it instead of a second recomputation of S, P and dP.
 // ds == nullptr, or a shape the tcgen05 kernels do not take, gives
 // launch_attn_bwd<bf16>.  ws holds B * H * T floats (Delta), as there.
+// With bias_part (B * attn_bias_parts(T) rows of 3C floats) the kernels also
+// leave per-block column sums of dqkv there (when they keep dS; the return
+// value of attn_bias_parts_written() says whether they did).
 int launch_attn_bwd_ds(const bf16* dout, const bf16* qkv, const bf16* out, const float* lse, int B,
-                       int Tn, int C, int H, bf16* dqkv, float* ws, bf16* ds, cudaStream_t st);
+                       int Tn, int C, int H, bf16* dqkv, float* ws, bf16* ds, cudaStream_t st,
+                       float* bias_part = nullptr);
+// row blocks of 128 per sequence: the partial rows per batch element
+int attn_bias_parts(int T);
+// whether launch_attn_bwd_ds with these arguments writes the partial sums
+bool attn_bias_parts_written(int B, int T, int C, int H, const bf16* ds);
+// out[c] (+)= sum over the `parts` rows of p[r * n + c], rows in a fixed order
+int launch_sum_parts(const float* p, int parts, int n, float* out, int accumulate,
+                     cudaStream_t st);
 // workspace of gpt2_attention_bwd: Delta (rounded up to 1 KB), then, for bf16
 // on the tcgen05 path, the score-gradient buffer
 size_t attn_bwd_workspace_total(int B, int T, int C, int H, bool bf16_path);

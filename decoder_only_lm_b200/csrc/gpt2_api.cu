@@ -111,6 +111,7 @@ struct gpt2_handle {
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_join2 = nullptr;
   float* ws2 = nullptr;
   bf16* ads = nullptr;  // attention score gradients (bf16 tcgen05 path), one layer at a time
+  float* qkvb_parts = nullptr;  // per-block column sums of dqkv left by those kernels
   void* ws_emb = nullptr;
   double* ws_norm = nullptr;
   DevStatus* status = nullptr;
@@ -657,6 +658,8 @@ int backward_t(gpt2_handle* h, float grad_scale) {
   A* datt = static_cast<A*>(h->datt);
   A* dqkv = static_cast<A*>(h->dqkv);
   const double attn_bwd_flops = 4.0 * B * Hh * double(T) * T * (C / Hh);
+  // the attention kernels leave the attn.qkv bias column sums (bf16 tcgen05 path)
+  const bool qkvb_fused = h->qkvb_parts && attn_bias_parts_written(B, T, C, Hh, h->ads);
   // Each weight-gradient GEMM (and the bias column sum beside it) is
   // independent of the input-gradient GEMM of the same layer: they run on the
   // side stream, launched after it, so that they fill its last partial wave;
@@ -711,10 +714,15 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     }
     {
       PROF(GPT2_PROF_ATTN_BWD, attn_bwd_flops, a * 9.0 * M * C + 8.0 * M * Hh);
-      if constexpr (std::is_same<A, bf16>::value)
+      if constexpr (std::is_same<A, bf16>::value) {
         H_TRY(h, launch_attn_bwd_ds(datt, static_cast<A*>(h->qkv[l]), static_cast<A*>(h->att[l]),
-                                    h->alse[l], B, T, C, Hh, dqkv, h->ws, h->ads, h->st));
-      else
+                                    h->alse[l], B, T, C, Hh, dqkv, h->ws, h->ads, h->st,
+                                    h->qkvb_parts));
+        // attn.qkv bias gradient from the kernels' per-block column sums
+        if (qkvb_fused)
+          H_TRY(h, launch_sum_parts(h->qkvb_parts, B * attn_bias_parts(T), 3 * C, G + o.qkvb, acc,
+                                    h->st));
+      } else
         H_TRY(h, launch_attn_bwd<A>(datt, static_cast<A*>(h->qkv[l]), static_cast<A*>(h->att[l]),
                                     h->alse[l], B, T, C, Hh, dqkv, h->ws, h->st));
       H_TRY(h, sd.join());  // attn.proj's weight gradient ran beside the attention backward
@@ -732,7 +740,8 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     }
     {
       PROF(GPT2_PROF_OTHER, 0, a * 3.0 * M * C);
-      H_TRY(h, launch_colsum<A>(dqkv, M, 3 * C, G + o.qkvb, acc, sd.ws(), sd.st()));
+      if (!qkvb_fused)
+        H_TRY(h, launch_colsum<A>(dqkv, M, 3 * C, G + o.qkvb, acc, sd.ws(), sd.st()));
       H_TRY(h, sd.join());
     }
     {
@@ -854,8 +863,11 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
   h->ws_bytes = ws;
   h->ws = static_cast<float*>(A(ws));
   h->ws2 = static_cast<float*>(A(ws));
-  if (h->use_bf16 && attn_tc_supported(c.max_B, c.max_Tseq, int(C), H))
+  if (h->use_bf16 && attn_tc_supported(c.max_B, c.max_Tseq, int(C), H)) {
     h->ads = static_cast<bf16*>(A(attn_tc_ds_bytes(c.max_B, c.max_Tseq, H)));
+    h->qkvb_parts = static_cast<float*>(
+        A(size_t(c.max_B) * attn_bias_parts(c.max_Tseq) * 3 * C * sizeof(float)));
+  }
   h->ws_emb = A(embed_bwd_workspace(M, int(C)));
   h->ws_norm = static_cast<double*>(A(gradnorm_workspace()));
   h->status = static_cast<DevStatus*>(A(sizeof(DevStatus)));

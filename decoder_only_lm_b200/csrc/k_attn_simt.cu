@@ -326,7 +326,8 @@ template int launch_attn_simt_bwd<bf16>(const bf16*, const bf16*, const bf16*, c
 int launch_attn_tc_fwd(const bf16* qkv, int B, int T, int C, int H, bf16* out, float* lse,
                        cudaStream_t st);
 int launch_attn_tc_bwd(const bf16* dout, const bf16* qkv, const float* lse, const float* delta,
-                       int B, int T, int C, int H, bf16* dqkv, bf16* ds, cudaStream_t st);
+                       int B, int T, int C, int H, bf16* dqkv, bf16* ds, float* bias_part,
+                       cudaStream_t st);
 
 template <>
 int launch_attn_fwd<float>(const float* qkv, int B, int Tn, int C, int H, float* out, float* lse,
@@ -344,14 +345,19 @@ int launch_attn_bwd<float>(const float* dout, const float* qkv, const float* out
                            int B, int Tn, int C, int H, float* dqkv, float* ws, cudaStream_t st) {
   return launch_attn_simt_bwd<float>(dout, qkv, out, lse, B, Tn, C, H, dqkv, ws, st);
 }
+int attn_bias_parts(int T) { return int(cdiv64(T, 128)); }
+bool attn_bias_parts_written(int B, int T, int C, int H, const bf16* ds) {
+  return ds && H >= 1 && C % H == 0 && attn_tc_supported(B, T, C, H);
+}
 int launch_attn_bwd_ds(const bf16* dout, const bf16* qkv, const bf16* out, const float* lse, int B,
-                       int Tn, int C, int H, bf16* dqkv, float* ws, bf16* ds, cudaStream_t st) {
+                       int Tn, int C, int H, bf16* dqkv, float* ws, bf16* ds, cudaStream_t st,
+                       float* bias_part) {
   if (!attn_tc_supported(B, Tn, C, H))
     return launch_attn_simt_bwd<bf16>(dout, qkv, out, lse, B, Tn, C, H, dqkv, ws, st);
   const int64_t rows = int64_t(B) * H * Tn;
   attn_delta64_kernel<<<int(cdiv64(rows * 8, 256)), 256, 0, st>>>(dout, out, B, Tn, C, H, ws);
   COUNT_LAUNCH(1);
-  return launch_attn_tc_bwd(dout, qkv, lse, ws, B, Tn, C, H, dqkv, ds, st);
+  return launch_attn_tc_bwd(dout, qkv, lse, ws, B, Tn, C, H, dqkv, ds, bias_part, st);
 }
 template <>
 int launch_attn_bwd<bf16>(const bf16* dout, const bf16* qkv, const bf16* out, const float* lse,

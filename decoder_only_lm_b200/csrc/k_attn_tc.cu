@@ -416,7 +416,36 @@ struct BwdParams {
   bf16* dst;
   int ntri;
   int* err;
+  // column sums of this CTA's 128 rows of dq, dk, dv (rows past T excluded)
+  // -> bias_part[(b * gridDim.x + block) * 3C + column] (null: not computed)
+  float* bias_part = nullptr;
 };
+
+// Sum over the 128 rows of the warpgroup of a 64-column row per thread into
+// out[0..63], in a fixed order: thread e adds column e % 64 over rows
+// 64 (e / 64) .. + 63 in eight interleaved chains (rows r = 8 i + k into chain
+// k), the chains in order, then the two halves.  All 128 threads call it
+// (named barriers); stg holds 128 x 65 floats of shared memory that nothing
+// else uses at this point.
+__device__ __forceinline__ void wg_colsum64(float* stg, int e, const float (&v)[64], float* out) {
+#pragma unroll
+  for (int c = 0; c < 64; ++c) stg[e * 65 + c] = v[c];
+  wg_bar();
+  const float* col = stg + (e >> 6) * 64 * 65 + (e & 63);
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = col[k * 65];
+#pragma unroll
+  for (int i = 1; i < 8; ++i)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] += col[(8 * i + k) * 65];
+  const float half = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+  wg_bar();  // every read of stg done
+  stg[e] = half;
+  wg_bar();
+  if (e < 64) out[e] = stg[e] + stg[64 + e];
+  wg_bar();  // stg may be rewritten
+}
 
 // ---------------------------------------------------------------- dK, dV
 // CTA: 128 keys kb*128 ..; 64-query tiles i from the diagonal to the end.
@@ -679,21 +708,37 @@ __global__ void __launch_bounds__(kThreads, 2)
       wg_bar();  // sLD may be rewritten for the next tile
     }
     ok = __all_sync(0xffffffffu, ok);
+    bool have = false;
     if (ok && n > 0) {
-      bool w = mbar_wait(b_mm, (n - 1) & 1, p.err, 29);
-      if (__all_sync(0xffffffffu, w)) {
-        tc_fence_after();
-        bf16* drow = p.dqkv + (int64_t(row_base) + key) * 3 * C + h * D;
-        // dV then dK, one 64-column row each
+      const bool w = mbar_wait(b_mm, (n - 1) & 1, p.err, 29);
+      have = __all_sync(0xffffffffu, w);
+    }
+    if (have) tc_fence_after();
+    bf16* drow = p.dqkv + (int64_t(row_base) + key) * 3 * C + h * D;
+    // dV then dK, one 64-column row each (and their column sums: every
+    // thread of the warpgroup takes part, whatever the waits gave)
+#pragma unroll 1
+    for (int w2 = 0; w2 < 2; ++w2) {
+      uint32_t a0[32], a1[32];
+      if (have) {
+        tmem_ld32_async((w2 ? tKd : tV) + lo, a0);
+        tmem_ld32_async((w2 ? tKd : tV) + lo + 32, a1);
+        tmem_wait_ld(a0);
+        reg_after_wait(a1);
+        if (key < T) store_row64(drow + (w2 ? C : 2 * C), a0, a1, w2 ? scale : 1.f);
+      }
+      if (p.bias_part) {  // the K / V rows of the keys past T are excluded
+        const float f = (have && key < T) ? (w2 ? scale : 1.f) : 0.f;
+        float v[64];
 #pragma unroll
-        for (int w2 = 0; w2 < 2; ++w2) {
-          uint32_t a0[32], a1[32];
-          tmem_ld32_async((w2 ? tKd : tV) + lo, a0);
-          tmem_ld32_async((w2 ? tKd : tV) + lo + 32, a1);
-          tmem_wait_ld(a0);
-          reg_after_wait(a1);
-          if (key < T) store_row64(drow + (w2 ? C : 2 * C), a0, a1, w2 ? scale : 1.f);
+        for (int c = 0; c < 32; ++c) {
+          v[c] = have ? __uint_as_float(a0[c]) * f : 0.f;
+          v[32 + c] = have ? __uint_as_float(a1[c]) * f : 0.f;
         }
+        // the K/V tiles' shared memory: every MMA that read it has completed
+        wg_colsum64(reinterpret_cast<float*>(smem), e, v,
+                    p.bias_part + (int64_t(b) * gridDim.x + kb) * 3 * C + (w2 ? C : 2 * C) +
+                        h * D);
       }
     }
   }
@@ -997,15 +1042,28 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int q = qb * BR + e;
     const uint32_t lo = uint32_t((warp & 3) * 32) << 16;
     const bool w = mbar_wait(b_acc, 0, p.err, 44);
-    if (__all_sync(0xffffffffu, w)) {
+    const bool have = __all_sync(0xffffffffu, w);
+    const float scale = rsqrtf(float(D));
+    uint32_t a0[32], a1[32];
+    if (have) {
       tc_fence_after();
-      uint32_t a0[32], a1[32];
       tmem_ld32_async(tmem + lo, a0);
       tmem_ld32_async(tmem + lo + 32, a1);
       tmem_wait_ld(a0);
       reg_after_wait(a1);
-      if (q < T)
-        store_row64(p.dqkv + (int64_t(row_base) + q) * 3 * C + h * D, a0, a1, rsqrtf(float(D)));
+      if (q < T) store_row64(p.dqkv + (int64_t(row_base) + q) * 3 * C + h * D, a0, a1, scale);
+    }
+    if (p.bias_part) {  // the rows of the queries past T are excluded
+      const float f = (have && q < T) ? scale : 0.f;
+      float v[64];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        v[c] = have ? __uint_as_float(a0[c]) * f : 0.f;
+        v[32 + c] = have ? __uint_as_float(a1[c]) * f : 0.f;
+      }
+      // the stage ring: every copy into it has been consumed by the MMAs
+      wg_colsum64(reinterpret_cast<float*>(smem), e, v,
+                  p.bias_part + (int64_t(b) * gridDim.x + qb) * 3 * C + h * D);
     }
   }
   tc_fence_before();
@@ -1048,7 +1106,8 @@ int launch_attn_tc_fwd(const bf16* qkv, int B, int T, int C, int H, bf16* out, f
 }
 
 int launch_attn_tc_bwd(const bf16* dout, const bf16* qkv, const float* lse, const float* delta,
-                       int B, int T, int C, int H, bf16* dqkv, bf16* ds, cudaStream_t st) {
+                       int B, int T, int C, int H, bf16* dqkv, bf16* ds, float* bias_part,
+                       cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(fa_tc_dkdv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1081,7 +1140,7 @@ int launch_attn_tc_bwd(const bf16* dout, const bf16* qkv, const float* lse, cons
     gpt2_internal::set_error("attention: tensor map encoding failed");
     return GPT2_ERR_CUDA;
   }
-  BwdParams p{T, C, H, lse, delta, dqkv, ds, ntri, device_error_word()};
+  BwdParams p{T, C, H, lse, delta, dqkv, ds, ntri, device_error_word(), ds ? bias_part : nullptr};
   dim3 grid(nqb, H, B);
   if (ds) {
     fa_tc_dkdv_kernel<true><<<grid, kThreads, DkdvCfg<true>::kSmem, st>>>(q128, q64, o64, ds_st, p);

@@ -15,6 +15,7 @@
 
 #include <algorithm>
 
+#include "attn_internal.h"
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -1090,6 +1091,14 @@ __global__ void __launch_bounds__(256) colsum_vec_kernel(const InT* __restrict__
     for (int k = 0; k < 8; ++k) t += sh[k][c];
     ws[int64_t(blockIdx.y) * N + n] = t;
   }
+}
+
+int launch_sum_parts(const float* p, int parts, int n, float* out, int accumulate,
+                     cudaStream_t st) {
+  reduce_rows_kernel<<<cdiv(n, 32), 256, 0, st>>>(p, parts, n, out, nullptr, n, accumulate);
+  COUNT_LAUNCH(1);
+  GPT2_LAUNCH_CHECK();
+  return GPT2_OK;
 }
 
 size_t colsum_workspace(int64_t M, int N) { return size_t(cdiv64(M, kColRows)) * N * sizeof(float); }
