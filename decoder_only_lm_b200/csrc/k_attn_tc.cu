@@ -2,7 +2,8 @@
 // TMEM accumulators, operands loaded by TMA), head size 64, bf16 in / fp32
 // accumulate [ZERO: Attention, OpFlashAttention recomputes the scores in the
 // backward; LECTURE: flash attention, causal mask].  The [T, T] scores and
-// probabilities never leave TMEM and registers.
+// probabilities never leave TMEM and registers; the backward may keep the
+// causal half of the score gradients (bf16) for its dQ step.
 //
 // Every kernel: one CTA of 192 threads per block of 128 rows (queries, or keys
 // in dK/dV) = the 128 TMEM lanes, streaming 64-row tiles of the other operand:
@@ -15,7 +16,7 @@
 //                      as bf16 over the first 32 columns of that tile, where
 //                      the next MMA takes them as its A operand (kind::f16
 //                      with A in TMEM), so they never pass through shared
-//                      memory.
+//                      memory (except the kept score gradients, below).
 // 256 TMEM columns and < 100 KB of shared memory let two CTAs share an SM, so
 // one CTA's elementwise work overlaps the other's MMAs; the shared memory is
 // a deep ring of streamed K/V (or Q/dO) tiles that hides load latency.
@@ -33,7 +34,9 @@
 //   With a score-gradient buffer the dK/dV kernel also writes dS^T (bf16, the
 //   values its dK MMA takes) and dQ is one contraction over it (no
 //   exponentials, no second S or dP); without one (the no-allocation entry
-//   point) the dQ kernel recomputes P and dS as above.
+//   point) the dQ kernel recomputes P and dS as above.  Both backward kernels
+//   may also leave per-block column sums of dq, dk, dv (the qkv bias gradient).
+// CTAs take the longest causal row blocks first (work_item).
 // Every output element is written by one CTA, no atomics (deterministic).
 // Every wait is bounded (2 s of global time) and reports a timeout in the
 // error word instead of hanging.
