@@ -35,6 +35,8 @@ GPT2_124M_T1024 = Shape(12, 768, 12, 50257, 50304, 1024, 1, 1024)
 # of its 24 layers: a different number of tiles per row, K=1024 for the head
 # and the fc layer, and LayerNorm rows of 1024 columns
 GPT2_350M_2L_T1024 = Shape(2, 1024, 16, 50257, 50304, 1024, 1, 1024)
+# the benchmark's own configuration: 16 sequences of 1024 tokens per step
+GPT2_124M_B16 = Shape(12, 768, 12, 50257, 50304, 1024, 16, 1024)
 
 
 @pytest.fixture(scope="module")
@@ -68,6 +70,49 @@ def test_step_t1024_zipf(torch, s):
     gm.synchronize()
     check_step(om, gm, named, flat, go, lo, rlo, lg, rl.cpu().numpy(), True)
     gm.close()
+
+
+def test_step_b16_as_benchmarked(torch):
+    """GPT-2 124M at B=16, T=1024, the launch configuration of the benchmark
+    (16384 rows: eight 2048-row LM-head chunks, 1536 CTAs per attention kernel,
+    the M = 16384 tilings and split counts).  Forward: nothing couples the
+    sequences of a batch, so the row losses of sampled sequences must match the
+    oracle run on each of those sequences alone.  Backward: the mean loss is
+    linear in the sequences' losses, so the gradient must equal the mean of
+    the 16 single-sequence gradients, accumulated here at B=1 (the path that
+    test_step_t1024_zipf checks against the oracle) with grad_scale = 1/16."""
+    s = GPT2_124M_B16
+    om, named, stream, x, y = inputs(s, seed=0, stream_seed=3, uniform=False)
+    tol = TOL[True]
+    gm = gpu_model(s, True)
+    gm.set_params(named)
+    rl = torch.empty(s.B * s.T, dtype=torch.float32, device="cuda")
+    gm.zero_grad()
+    lg = gm.forward_loss(torch.from_numpy(x).cuda(), torch.from_numpy(y).cuda(), row_loss=rl)
+    gm.backward()
+    gm.synchronize()
+    rows = rl.cpu().numpy().reshape(s.B, s.T)
+    assert abs(lg - rows.mean()) <= 1e-4
+    flat = om.pack(named)
+    for b in (0, 9, 15):
+        lo_b, rlo_b, _, _ = om.fwd_bwd(flat, x[b:b + 1], y[b:b + 1], grads=False, row_loss=True)
+        assert abs(rows[b].mean() - lo_b) <= tol["loss"], (b, rows[b].mean(), lo_b)
+        assert np.max(np.abs(rows[b] - rlo_b)) <= 10 * tol["loss"], b
+    g16 = {n: gm.get_tensor(n, which=1) for n, _ in om.shapes()}
+    gm.close()
+    one = Shape(s.n_layer, s.n_embd, s.n_head, s.vocab_size, s.padded_vocab, s.max_T, 1, s.T)
+    g1 = gpu_model(one, True)
+    g1.set_params(named)
+    g1.zero_grad()
+    for b in range(s.B):
+        g1.forward_loss(torch.from_numpy(x[b:b + 1]).cuda(), torch.from_numpy(y[b:b + 1]).cuda(),
+                        loss=False)
+        g1.backward(1.0 / s.B)
+    g1.synchronize()
+    for name, _ in om.shapes():
+        r = rel_l2(g16[name], g1.get_tensor(name, which=1))
+        assert r <= tol["grad"], (name, r)
+    g1.close()
 
 
 @pytest.mark.parametrize("scale", [1.0, 6.0], ids=["qkv_x1", "qkv_x6"])
