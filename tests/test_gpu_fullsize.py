@@ -35,8 +35,11 @@ GPT2_124M_T1024 = Shape(12, 768, 12, 50257, 50304, 1024, 1, 1024)
 # of its 24 layers: a different number of tiles per row, K=1024 for the head
 # and the fc layer, and LayerNorm rows of 1024 columns
 GPT2_350M_2L_T1024 = Shape(2, 1024, 16, 50257, 50304, 1024, 1, 1024)
-# the benchmark's own configuration: 16 sequences of 1024 tokens per step
+# the benchmarked configurations: 16 sequences of 1024 tokens per step
 GPT2_124M_B16 = Shape(12, 768, 12, 50257, 50304, 1024, 16, 1024)
+GPT2_350M_B16 = Shape(24, 1024, 16, 50257, 50304, 1024, 16, 1024)
+# the micro-batch of the accumulation workload: 64 sequences (65536 rows)
+GPT2_124M_B64 = Shape(12, 768, 12, 50257, 50304, 1024, 64, 1024)
 
 
 @pytest.fixture(scope="module")
@@ -72,16 +75,19 @@ def test_step_t1024_zipf(torch, s):
     gm.close()
 
 
-def test_step_b16_as_benchmarked(torch):
-    """GPT-2 124M at B=16, T=1024, the launch configuration of the benchmark
-    (16384 rows: eight 2048-row LM-head chunks, 1536 CTAs per attention kernel,
-    the M = 16384 tilings and split counts).  Forward: nothing couples the
+@pytest.mark.parametrize("s,sampled", [(GPT2_124M_B16, (0, 9, 15)), (GPT2_350M_B16, (5,)),
+                                       (GPT2_124M_B64, (63,))],
+                         ids=["124m_b16", "350m_b16", "124m_b64"])
+def test_step_as_benchmarked(torch, s, sampled):
+    """GPT-2 124M and 350M at B=16, T=1024, and the 124M micro-batch of 64
+    sequences of the accumulation workload: the launch configurations of the
+    benchmark (16384 or 65536 rows: 8 or 32 LM-head chunks of 2048 rows, 1536
+    or 6144 CTAs per attention kernel, the GEMM tilings and split counts).  Forward: nothing couples the
     sequences of a batch, so the row losses of sampled sequences must match the
     oracle run on each of those sequences alone.  Backward: the mean loss is
     linear in the sequences' losses, so the gradient must equal the mean of
-    the 16 single-sequence gradients, accumulated here at B=1 (the path that
-    test_step_t1024_zipf checks against the oracle) with grad_scale = 1/16."""
-    s = GPT2_124M_B16
+    the B single-sequence gradients, accumulated here at B=1 (the path that
+    test_step_t1024_zipf checks against the oracle) with grad_scale = 1/B."""
     om, named, stream, x, y = inputs(s, seed=0, stream_seed=3, uniform=False)
     tol = TOL[True]
     gm = gpu_model(s, True)
@@ -94,7 +100,7 @@ def test_step_b16_as_benchmarked(torch):
     rows = rl.cpu().numpy().reshape(s.B, s.T)
     assert abs(lg - rows.mean()) <= 1e-4
     flat = om.pack(named)
-    for b in (0, 9, 15):
+    for b in sampled:
         lo_b, rlo_b, _, _ = om.fwd_bwd(flat, x[b:b + 1], y[b:b + 1], grads=False, row_loss=True)
         assert abs(rows[b].mean() - lo_b) <= tol["loss"], (b, rows[b].mean(), lo_b)
         assert np.max(np.abs(rows[b] - rlo_b)) <= 10 * tol["loss"], b
