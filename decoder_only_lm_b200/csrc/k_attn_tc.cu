@@ -730,13 +730,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         reg_after_wait(a1);
         if (key < T) store_row64(drow + (w2 ? C : 2 * C), a0, a1, w2 ? scale : 1.f);
       }
-      if (p.bias_part) {  // the K / V rows of the keys past T are excluded
-        const float f = (have && key < T) ? (w2 ? scale : 1.f) : 0.f;
+      if (p.bias_part) {
+        // the K / V rows of the keys past T are excluded by selection (a
+        // product with 0 would keep a NaN of a row nothing defines)
+        const bool use = have && key < T;
+        const float f = w2 ? scale : 1.f;
         float v[64];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          v[c] = have ? __uint_as_float(a0[c]) * f : 0.f;
-          v[32 + c] = have ? __uint_as_float(a1[c]) * f : 0.f;
+          v[c] = use ? __uint_as_float(a0[c]) * f : 0.f;
+          v[32 + c] = use ? __uint_as_float(a1[c]) * f : 0.f;
         }
         // the K/V tiles' shared memory: every MMA that read it has completed
         wg_colsum64(reinterpret_cast<float*>(smem), e, v,
@@ -1056,13 +1059,16 @@ __global__ void __launch_bounds__(kThreads, 3)
       reg_after_wait(a1);
       if (q < T) store_row64(p.dqkv + (int64_t(row_base) + q) * 3 * C + h * D, a0, a1, scale);
     }
-    if (p.bias_part) {  // the rows of the queries past T are excluded
-      const float f = (have && q < T) ? scale : 0.f;
+    if (p.bias_part) {
+      // the rows of the queries past T are excluded by selection: their score
+      // gradients may be memory nothing has written (a product with 0 would
+      // keep a NaN)
+      const bool use = have && q < T;
       float v[64];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        v[c] = have ? __uint_as_float(a0[c]) * f : 0.f;
-        v[32 + c] = have ? __uint_as_float(a1[c]) * f : 0.f;
+        v[c] = use ? __uint_as_float(a0[c]) * scale : 0.f;
+        v[32 + c] = use ? __uint_as_float(a1[c]) * scale : 0.f;
       }
       // the stage ring: every copy into it has been consumed by the MMAs
       wg_colsum64(reinterpret_cast<float*>(smem), e, v,

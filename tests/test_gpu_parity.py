@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 import synth
-from tests.parity_util import RAGGED, TINY, TOL, gpu_model, inputs, rel_l2
+from tests.parity_util import RAGGED, TINY, TOL, Shape, gpu_model, inputs, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +48,23 @@ def test_step_matches_oracle(shape, bf16, uniform, torch):
     of equal ids to sum."""
     om, gm, named, flat, (lo, rlo, go), (lg, rlg, x, y) = run_both(shape, bf16, torch,
                                                                    uniform=uniform)
+    check_step(om, gm, named, flat, go, lo, rlo, lg, rlg, bf16)
+
+
+# Degenerate sizes: one-token sequences (a single key, the diagonal block only)
+# with head size 16 (CUDA-core attention) and 64 (tcgen05 attention, one
+# 128 x 128 score-gradient tile per head), and one sequence of two tokens (the
+# LM head and every linear layer on two rows).
+T1_HEAD16 = Shape(2, 64, 4, 512, 512, 64, 3, 1)
+T1_HEAD64 = Shape(2, 128, 2, 1000, 1024, 128, 2, 1)
+B1_T2_HEAD64 = Shape(2, 128, 2, 1000, 1024, 128, 1, 2)
+
+
+@pytest.mark.parametrize("shape", [T1_HEAD16, T1_HEAD64, B1_T2_HEAD64],
+                         ids=["t1_head16", "t1_head64", "b1_t2_head64"])
+@pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
+def test_step_degenerate_sizes(shape, bf16, torch):
+    om, gm, named, flat, (lo, rlo, go), (lg, rlg, x, y) = run_both(shape, bf16, torch)
     check_step(om, gm, named, flat, go, lo, rlo, lg, rlg, bf16)
 
 
