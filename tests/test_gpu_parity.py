@@ -53,15 +53,17 @@ def test_step_matches_oracle(shape, bf16, uniform, torch):
 
 # Degenerate sizes: one-token sequences (a single key, the diagonal block only)
 # with head size 16 (CUDA-core attention) and 64 (tcgen05 attention, one
-# 128 x 128 score-gradient tile per head), and one sequence of two tokens (the
-# LM head and every linear layer on two rows).
+# 128 x 128 score-gradient tile per head), one sequence of two tokens (the
+# LM head and every linear layer on two rows), and T = 130.
 T1_HEAD16 = Shape(2, 64, 4, 512, 512, 64, 3, 1)
 T1_HEAD64 = Shape(2, 128, 2, 1000, 1024, 128, 2, 1)
 B1_T2_HEAD64 = Shape(2, 128, 2, 1000, 1024, 128, 1, 2)
+# T = 130: the second query block's last 64-query half lies wholly past T
+T130_HEAD64 = Shape(2, 128, 2, 1000, 1024, 256, 2, 130)
 
 
-@pytest.mark.parametrize("shape", [T1_HEAD16, T1_HEAD64, B1_T2_HEAD64],
-                         ids=["t1_head16", "t1_head64", "b1_t2_head64"])
+@pytest.mark.parametrize("shape", [T1_HEAD16, T1_HEAD64, B1_T2_HEAD64, T130_HEAD64],
+                         ids=["t1_head16", "t1_head64", "b1_t2_head64", "t130_head64"])
 @pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
 def test_step_degenerate_sizes(shape, bf16, torch):
     om, gm, named, flat, (lo, rlo, go), (lg, rlg, x, y) = run_both(shape, bf16, torch)
