@@ -84,9 +84,11 @@ def test_layernorm_unaligned_view(g):
 # head size 64 (bf16: the tcgen05 kernels) at T = 130 and 320 ends in a query
 # block whose second 64-query half lies wholly past T: the kept score
 # gradients there are never written and must not reach any stored row;
-# T = 2048 runs 16 key blocks per (batch, head), 136 score-gradient tiles
+# T = 2048 runs 16 key blocks per (batch, head), 136 score-gradient tiles;
+# T = 1: one key, the diagonal tile only
 @pytest.mark.parametrize("B,T,C,H", [(2, 37, 64, 4), (1, 200, 128, 2), (2, 64, 96, 3),
-                                     (1, 130, 128, 2), (2, 320, 128, 2), (1, 2048, 128, 2)])
+                                     (1, 130, 128, 2), (2, 320, 128, 2), (1, 2048, 128, 2),
+                                     (3, 1, 128, 2)])
 @pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
 def test_attention(g, B, T, C, H, bf16):
     import torch
