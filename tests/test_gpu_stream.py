@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 
 import synth
-from tests.parity_util import TINY, gpu_model, inputs
+from tests.parity_util import RAGGED, TINY, gpu_model, inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -25,12 +25,12 @@ def torch():
     return torch
 
 
-def eager_steps(gm, stream, bt, accum, lrs, start=0):
+def eager_steps(gm, stream, bt, accum, lrs, start=0, shape=TINY):
     off = start
     for lr in lrs:
         gm.zero_grad()
         for _ in range(accum):
-            x, y = gm.batch_from_stream(stream, off, TINY.B, TINY.T)
+            x, y = gm.batch_from_stream(stream, off, shape.B, shape.T)
             gm.forward_loss(x, y, loss=False)
             gm.backward(1.0 / accum)
             off += bt
@@ -39,19 +39,23 @@ def eager_steps(gm, stream, bt, accum, lrs, start=0):
     return off
 
 
+# TINY has head size 16 (CUDA-core attention); RAGGED head size 64, so in bf16
+# the tcgen05 attention kernels, with the kept score gradients and the qkv bias
+# column sums, are recorded into the graph
+@pytest.mark.parametrize("shape", [TINY, RAGGED], ids=["tiny", "ragged"])
 @pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
-def test_graph_steps_equal_eager_steps(bf16, torch):
-    om, named, _, _, _ = inputs(TINY)
-    bt, accum, lrs = TINY.B * TINY.T, 2, [6e-4, 3e-4, 1e-4]
-    s_np = synth.uniform_stream(5, accum * len(lrs) * bt + 1, TINY.vocab_size)
+def test_graph_steps_equal_eager_steps(bf16, shape, torch):
+    om, named, _, _, _ = inputs(shape)
+    bt, accum, lrs = shape.B * shape.T, 2, [6e-4, 3e-4, 1e-4]
+    s_np = synth.uniform_stream(5, accum * len(lrs) * bt + 1, shape.vocab_size)
     stream = torch.from_numpy(s_np.astype(np.uint16).view(np.int16)).cuda()
-    ge, gg = gpu_model(TINY, bf16), gpu_model(TINY, bf16)
+    ge, gg = gpu_model(shape, bf16), gpu_model(shape, bf16)
     ge.set_params(named)
     gg.set_params(named)
     import decoder_only_lm_b200 as g
-    end = eager_steps(ge, stream, bt, accum, lrs)
+    end = eager_steps(ge, stream, bt, accum, lrs, shape=shape)
     n0 = g.launch_count()
-    gg.stream_begin(stream, 0, bt, TINY.B, TINY.T, accum=accum, **HP)
+    gg.stream_begin(stream, 0, bt, shape.B, shape.T, accum=accum, **HP)
     recorded = g.launch_count() - n0
     # every kernel issued while recording is in the graph (the bf16 weight
     # mirror is refreshed once before recording)
