@@ -459,10 +459,13 @@ int gpt2_attention_bwd(const void* dout, const void* qkv, const void* out, const
 /* gpt2_attention_bwd for callers that cannot allocate device memory: a
  * program that runs under a fixed memory budget already handed to another
  * allocator, or a loop that must not call cudaMalloc / cudaFree because those
- * calls can wait for the whole device to go idle.  Same arguments and result
- * as gpt2_attention_bwd, but no workspace: the per-row scratch lives in a
- * fixed 4 MiB device array declared by the library (held on every device that
- * loads the library until the process exits).  No counterpart on the pages:
+ * calls can wait for the whole device to go idle.  Same arguments and the
+ * same computation as gpt2_attention_bwd, but no workspace: the per-row
+ * scratch lives in a fixed 4 MiB device array declared by the library (held
+ * on every device that loads the library until the process exits), and the
+ * dQ step recomputes the score gradients instead of keeping them (bf16 with
+ * head size 64), so results can differ from gpt2_attention_bwd's in the last
+ * bits.  No counterpart on the pages:
  * an interface variant only.
  *   - Limit: B*H*T <= 1,048,576 rows, else GPT2_ERR_ARG and a message.
  *   - The first call on a device looks up the array's device address with
