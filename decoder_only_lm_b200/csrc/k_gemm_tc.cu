@@ -419,10 +419,10 @@ struct TeCfg {
   static constexpr int ARR = EPI == EPI_GELU ? 2 : 1;  // buffers per chunk
   static constexpr int SLOTS = NBUF / ARR;
   static constexpr bool HAS_IN = epi_has_input<EPI>();
-  static constexpr int DIST = HAS_IN ? SLOTS - 2 : 0;  // input prefetch distance in chunks
-  // bulk groups that may still be reading their buffers when a chunk is done
-  static constexpr int WAITN = HAS_IN ? SLOTS - 1 - DIST : (SLOTS - 2 < 6 ? SLOTS - 2 : 6);
-  static_assert(SLOTS >= 2 && SLOTS <= 16 && WAITN >= 0, "epilogue slots");
+  // bulk groups that may still be reading their buffers when a chunk is
+  // done (with an input: when the issuer takes the next chunk)
+  static constexpr int WAITN = HAS_IN ? 1 : (SLOTS - 2 < 6 ? SLOTS - 2 : 6);
+  static_assert(SLOTS >= 2 && SLOTS <= 8 && WAITN >= 0, "epilogue slots");
 };
 // tcgen05.ld of CW (32 or 16) accumulator columns without waiting; the
 // registers are valid after tmem_wait_cols(r), which names them so that no
@@ -518,21 +518,99 @@ __device__ __forceinline__ void bias_chunk(const float* bias, int n0, int N, flo
   }
 }
 
-// Epilogue warpgroup with TMA stores: thread e owns row 128 r + e of the
-// pair's tile (CTA rank r, TMEM lane e).
-// Per chunk it loads CW accumulator columns, applies the epilogue op (inputs
-// such as the residual or the GELU input arrive by TMA in the chunk's own
-// buffer, DIST chunks ahead), writes the row into the swizzled buffer, and
-// after one named barrier a single thread issues the TMA store (or, for
-// gradient accumulation, the TMA reduce-add: one fp32 add per element, so the
-// result does not depend on timing).  Out-of-range rows and columns of edge
-// tiles are clipped by the tensor map.
+// The epilogue op on one chunk of a row: v holds CW accumulator columns of
+// row e of this CTA's half-tile (first column n0); inputs (residual, GELU
+// input) are read from, and the results written to, the chunk's swizzled
+// buffer(s) at b0.
+template <int EPI, typename OutT, int CW>
+__device__ __forceinline__ void chunk_apply(const TcParams& p, uint8_t* b0, int e, int n0,
+                                            float (&v)[CW], float row_l, int row_t) {
+  const EpiParams& ep = p.ep;
+  if constexpr (EPI == EPI_RESID || EPI == EPI_GELU_BWD) {
+    float r[CW];
+    row_get<OutT>(b0, e, r);
+    if constexpr (EPI == EPI_RESID) {
+      if (ep.bias) {
+        float bb[CW];
+        bias_chunk<CW>(ep.bias, n0, p.N, bb);
+#pragma unroll
+        for (int j = 0; j < CW; ++j) r[j] += bb[j];
+      }
+#pragma unroll
+      for (int j = 0; j < CW; ++j) v[j] += r[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < CW; j += 2) gelu_bwd_pair(v[j], v[j + 1], r[j], r[j + 1]);
+    }
+    row_put<OutT>(b0, e, v);
+  } else if constexpr (EPI == EPI_GELU) {
+    static_assert(CW == 32, "bf16 GELU chunks");
+    float bb[CW];
+    bias_chunk<CW>(ep.bias, n0, p.N, bb);
+    uint32_t pre[CW / 2], act[CW / 2];
+    gelu_chunk32(v, bb, pre, act);
+    row_put_bits(b0, e, pre);
+    row_put_bits(b0 + 8192, e, act);
+  } else if constexpr (EPI == EPI_STORE) {
+    if (ep.bias) {
+      float bb[CW];
+      bias_chunk<CW>(ep.bias, n0, p.N, bb);
+#pragma unroll
+      for (int j = 0; j < CW; ++j) v[j] = v[j] * ep.alpha + bb[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < CW; ++j) v[j] *= ep.alpha;
+    }
+    row_put<OutT>(b0, e, v);
+  } else if constexpr (EPI == EPI_ACC) {
+    if (!p.ws) {  // split partial sums stay raw (alpha applied by the reduction)
+#pragma unroll
+      for (int j = 0; j < CW; ++j) v[j] *= ep.alpha;
+    }
+    row_put<OutT>(b0, e, v);
+  } else if constexpr (EPI == EPI_CE_GRAD) {
+    const float cs = ep.ce_scale, l2 = row_l * kLog2e;
+#pragma unroll
+    for (int j = 0; j < CW; ++j) v[j] = cs * ex2_hw(fmaf(v[j], kLog2e, -l2));
+    if (row_t >= n0 && row_t < n0 + CW) {  // the target column: - scale
+#pragma unroll
+      for (int j = 0; j < CW; ++j)
+        if (n0 + j == row_t) v[j] -= cs;
+    }
+    row_put<OutT>(b0, e, v);
+  }
+}
+
+// Barriers of the TMA epilogue (offsets in tb, one per slot and warpgroup):
+// in[s] the chunk's input landed (TMA transaction count), rdy[s] the chunk is
+// written (4 warp arrivals, epilogues with an input only).
+constexpr int kEpiIn = 4, kEpiRdy = 20, kTmemSlot = 36;
+
+// The pair-local tiles of warpgroup wg (wg, wg+2, ...).
+struct EpiTiles {
+  int pair, npairs, wg, my_tiles;
+  __device__ EpiTiles(const TcParams& p, int wg_) : wg(wg_) {
+    pair = int(blockIdx.x) >> 1;
+    npairs = int(gridDim.x) >> 1;
+    const int pair_tiles = pair < p.total_tiles ? (p.total_tiles - 1 - pair) / npairs + 1 : 0;
+    my_tiles = pair_tiles > wg ? (pair_tiles - wg + 1) / 2 : 0;
+  }
+  __device__ int tile(int j) const { return pair + (wg + 2 * j) * npairs; }
+};
+
+// Epilogue warpgroup with TMA stores, for the epilogues without an input:
+// thread e owns row 128 r + e of the pair's tile (CTA rank r, TMEM lane e).
+// Per chunk it loads CW accumulator columns, applies the epilogue op, writes
+// the row into the swizzled buffer, and after one named barrier a single
+// thread issues the TMA store (for gradient accumulation the TMA reduce-add:
+// one fp32 add per element, so the result does not depend on timing).
+// Out-of-range rows and columns of edge tiles are clipped by the tensor map.
 template <int BN, int EPI, typename OutT, int NBUF>
 __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMap* mo,
-                                             const CUtensorMap* mo2, const CUtensorMap* mi,
-                                             uint8_t* ebuf, uint64_t* tb, uint32_t tmem_base,
-                                             int wg) {
+                                             const CUtensorMap* mo2, uint8_t* ebuf, uint64_t* tb,
+                                             uint32_t tmem_base, int wg) {
   using T = TeCfg<EPI, OutT, NBUF>;
+  static_assert(!T::HAS_IN, "epilogues with an input use epilogue_tma_split");
   constexpr int CW = T::CW, NCH = BN / CW, SL = T::SLOTS;
   const int e = threadIdx.x - 128 - 128 * wg;
   const int bar_id = 1 + wg;
@@ -540,39 +618,19 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
   const bool leader = e == 0;
   const uint32_t eb = smem_u32(ebuf);
   const int rank = int(cluster_ctarank());
-  const int pair = int(blockIdx.x) >> 1, npairs = int(gridDim.x) >> 1;
   auto tfull = [&](int a) { return smem_u32(tb + a); };
   // the even CTA's accumulator-empty barrier (its MMA issuer waits on it)
   auto tempty_pair = [&](int a) { return mapa_shared(smem_u32(tb + 2 + a), 0); };
-  auto lbar = [&](int s) { return smem_u32(tb + 4 + 8 * wg + s); };  // one per slot (<= 8)
-  const EpiParams& ep = p.ep;
-  // warpgroup wg drains accumulator wg: the pair's local tiles wg, wg+2, ...
-  const int pair_tiles = pair < p.total_tiles ? (p.total_tiles - 1 - pair) / npairs + 1 : 0;
-  const int my_tiles = pair_tiles > wg ? (pair_tiles - wg + 1) / 2 : 0;
-  const int total_chunks = my_tiles * NCH;
-  int next_load = 0;  // next chunk whose input is to be fetched (leader only)
-  auto issue_load = [&]() {
-    const int tile = pair + (wg + 2 * (next_load / NCH)) * npairs;
-    int tm, tn, sp;
-    tile_coords(p, tile, tm, tn, sp);
-    const int slot = next_load % SL;
-    mbar_expect_tx(lbar(slot), 8192);
-    tma_load_2d(eb + slot * 8192, mi, lbar(slot), tn * BN + (next_load % NCH) * CW,
-                tm * BM2 + rank * BM);
-    ++next_load;
-  };
-  if (T::HAS_IN && leader)
-    while (next_load < min(T::DIST, total_chunks)) issue_load();
-
+  const EpiTiles et(p, wg);
   // A wait that expires (error word set) poisons the thread: later waits are
   // skipped but every thread still runs the same sequence of named barriers,
   // so no warp is left waiting at one.
   int g = 0;  // chunks done by this warpgroup
   bool ok = true;
-  for (int t_local = wg, tile = pair + wg * npairs; tile < p.total_tiles;
-       t_local += 2, tile += 2 * npairs) {
+  for (int j = 0; j < et.my_tiles; ++j) {
+    const int t_local = wg + 2 * j;
     int tm, tn, sp;
-    tile_coords(p, tile, tm, tn, sp);
+    tile_coords(p, et.tile(j), tm, tn, sp);
     const int acc = wg;
     const int m0 = tm * BM2 + rank * BM;  // first row of this CTA's half
     if (ok) ok = mbar_wait(tfull(acc), (t_local >> 1) & 1, p.err, 4);
@@ -581,8 +639,8 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
     float row_l = 0.f;
     int row_t = -1;
     if (EPI == EPI_CE_GRAD && m < p.M) {
-      row_l = ep.lse[m];
-      row_t = ep.tgt[m];
+      row_l = p.ep.lse[m];
+      row_t = p.ep.tgt[m];
     }
     const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
     // the accumulator columns of chunk c+1 are loaded while chunk c is processed
@@ -592,11 +650,10 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
 #pragma unroll 1
     for (int c = 0; c < NCH; ++c, ++g) {
       const int slot = g % SL;
-      uint8_t* b0 = ebuf + slot * T::ARR * 8192;
       const int n0 = tn * BN + c * CW;
       float v[CW];
 #pragma unroll
-      for (int j = 0; j < CW; ++j) v[j] = __uint_as_float(rn[j]);
+      for (int jj = 0; jj < CW; ++jj) v[jj] = __uint_as_float(rn[jj]);
       if (c + 1 < NCH) {
         tmem_ld_cols(tbase + uint32_t((c + 1) * CW), rn);
       } else if (leader) {
@@ -604,73 +661,17 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
         // barrier: the accumulator is drained, the pair's MMA may reuse it
         mbar_arrive_cluster(tempty_pair(acc));
       }
-      if constexpr (EPI == EPI_RESID || EPI == EPI_GELU_BWD) {
-        if (ok) ok = mbar_wait(lbar(slot), uint32_t((g / SL) & 1), p.err, 7);
-        float r[CW];
-        row_get<OutT>(b0, e, r);
-        if constexpr (EPI == EPI_RESID) {
-          if (ep.bias) {
-            float bb[CW];
-            bias_chunk<CW>(ep.bias, n0, p.N, bb);
-#pragma unroll
-            for (int j = 0; j < CW; ++j) r[j] += bb[j];
-          }
-#pragma unroll
-          for (int j = 0; j < CW; ++j) v[j] += r[j];
-        } else {
-#pragma unroll
-          for (int j = 0; j < CW; j += 2) gelu_bwd_pair(v[j], v[j + 1], r[j], r[j + 1]);
-        }
-        row_put<OutT>(b0, e, v);
-      } else if constexpr (EPI == EPI_GELU) {
-        static_assert(CW == 32, "bf16 GELU chunks");
-        float bb[CW];
-        bias_chunk<CW>(ep.bias, n0, p.N, bb);
-        uint32_t pre[CW / 2], act[CW / 2];
-        gelu_chunk32(v, bb, pre, act);
-        row_put_bits(b0, e, pre);
-        row_put_bits(b0 + 8192, e, act);
-      } else if constexpr (EPI == EPI_STORE) {
-        if (ep.bias) {
-          float bb[CW];
-          bias_chunk<CW>(ep.bias, n0, p.N, bb);
-#pragma unroll
-          for (int j = 0; j < CW; ++j) v[j] = v[j] * ep.alpha + bb[j];
-        } else {
-#pragma unroll
-          for (int j = 0; j < CW; ++j) v[j] *= ep.alpha;
-        }
-        row_put<OutT>(b0, e, v);
-      } else if constexpr (EPI == EPI_ACC) {
-        if (!p.ws) {  // split partial sums stay raw (alpha applied by the reduction)
-#pragma unroll
-          for (int j = 0; j < CW; ++j) v[j] *= ep.alpha;
-        }
-        row_put<OutT>(b0, e, v);
-      } else if constexpr (EPI == EPI_CE_GRAD) {
-        const float cs = ep.ce_scale, l2 = row_l * kLog2e;
-#pragma unroll
-        for (int j = 0; j < CW; ++j) v[j] = cs * ex2_hw(fmaf(v[j], kLog2e, -l2));
-        if (row_t >= n0 && row_t < n0 + CW) {  // the target column: - scale
-#pragma unroll
-          for (int j = 0; j < CW; ++j)
-            if (n0 + j == row_t) v[j] -= cs;
-        }
-        row_put<OutT>(b0, e, v);
-      }
+      chunk_apply<EPI, OutT, CW>(p, ebuf + slot * T::ARR * 8192, e, n0, v, row_l, row_t);
       fence_proxy_async();
       if (c + 1 < NCH) tmem_wait_cols(rn);
       if (c + 2 == NCH) tc_fence_before();  // last TMEM load of the tile waited for
-      if (leader) {
-        bulk_wait_read<T::WAITN>();
-        if (T::HAS_IN && next_load < total_chunks) issue_load();
-      }
+      if (leader) bulk_wait_read<T::WAITN>();
       epi_bar(bar_id);
       if (leader) {
         const uint32_t src = eb + slot * T::ARR * 8192;
         if (EPI == EPI_ACC && p.ws)  // split sp's partial: rows sp * M .. of [splits * M, N]
           tma_store_2d(mo, src, n0, m0 + sp * p.M);
-        else if (EPI == EPI_ACC && ep.accumulate)
+        else if (EPI == EPI_ACC && p.ep.accumulate)
           tma_reduce_add_2d(mo, src, n0, m0);
         else
           tma_store_2d(mo, src, n0, m0);
@@ -679,14 +680,126 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
       }
     }
   }
-  if (leader) {
-    bulk_wait_all();
-    // after an expired wait some fetched inputs were never waited for: let
-    // the last one of each buffer land before the CTA exits
-    if (!ok)
-      for (int gc = max(0, next_load - SL); gc < next_load; ++gc)
-        mbar_wait(lbar(gc % SL), uint32_t((gc / SL) & 1), p.err, 8);
+  if (leader) bulk_wait_all();
+}
+
+// Epilogue with an input (residual add, GELU backward), split in two roles
+// per warpgroup wg so that no TMA issue and no named barrier sits on the
+// warpgroup's per-chunk path:
+//   - the 128 threads of the warpgroup (thread e owns row 128 r + e of the
+//     pair's tile) wait for the chunk's input, load CW accumulator columns,
+//     apply the op, write the row over the input in the chunk's buffer, and
+//     each warp signals "chunk written" (rdy);
+//   - one issuer thread (lane 0 of warp 2 + wg, epilogue_issuer) issues the
+//     chunk's TMA store and, once that store has read the buffer, fetches
+//     the input of a later chunk into it.
+template <int BN, int EPI, typename OutT, int NBUF>
+__device__ __forceinline__ void epilogue_tma_split(const TcParams& p, uint8_t* ebuf, uint64_t* tb,
+                                                   uint32_t tmem_base, int wg) {
+  using T = TeCfg<EPI, OutT, NBUF>;
+  static_assert(T::HAS_IN && T::ARR == 1, "epilogues with an input");
+  constexpr int CW = T::CW, NCH = BN / CW, SL = T::SLOTS;
+  const int e = threadIdx.x - 128 - 128 * wg;
+  const int lane = e & 31;
+  const int q = e >> 5;  // TMEM lanes 32q .. 32q+31
+  auto tfull = [&](int a) { return smem_u32(tb + a); };
+  auto tempty_pair = [&](int a) { return mapa_shared(smem_u32(tb + 2 + a), 0); };
+  auto inb = [&](int s) { return smem_u32(tb + kEpiIn + 8 * wg + s); };
+  auto rdy = [&](int s) { return smem_u32(tb + kEpiRdy + 8 * wg + s); };
+  const EpiTiles et(p, wg);
+  // an expired wait (error word set) skips later waits; every arrival still happens
+  int g = 0;
+  bool ok = true;
+  for (int j = 0; j < et.my_tiles; ++j) {
+    const int t_local = wg + 2 * j;
+    int tm, tn, sp;
+    tile_coords(p, et.tile(j), tm, tn, sp);
+    const int acc = wg;
+    if (ok) ok = mbar_wait(tfull(acc), (t_local >> 1) & 1, p.err, 4);
+    tc_fence_after();
+    const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
+    // this warp's TMEM loads of the tile are complete: one of the pair's 8
+    // arrivals that let the MMA reuse the accumulator
+    auto drained = [&]() {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_pair(acc));
+    };
+    uint32_t rn[CW];
+    tmem_ld_cols(tbase, rn);
+    tmem_wait_cols(rn);
+    if (NCH == 1) drained();
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c, ++g) {
+      const int slot = g % SL;
+      float v[CW];
+#pragma unroll
+      for (int jj = 0; jj < CW; ++jj) v[jj] = __uint_as_float(rn[jj]);
+      if (c + 1 < NCH) tmem_ld_cols(tbase + uint32_t((c + 1) * CW), rn);
+      if (ok) ok = mbar_wait(inb(slot), uint32_t((g / SL) & 1), p.err, 7);
+      chunk_apply<EPI, OutT, CW>(p, ebuf + slot * 8192, e, tn * BN + c * CW, v, 0.f, -1);
+      // this thread's rows are written (generic proxy) before the store reads
+      // them (async proxy); the warp's arrival follows all its lanes' fences
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(rdy(slot));
+      if (c + 1 < NCH) {
+        tmem_wait_cols(rn);
+        if (c + 2 == NCH) drained();  // the tile's last TMEM load has completed
+      }
+    }
   }
+}
+
+// The issuer thread of warpgroup wg's chunks (epilogue_tma_split).  One
+// store group may still be reading its buffer when the next chunk is taken;
+// the input of chunk g + SLOTS - 1 goes into the buffer that chunk g - 1's
+// store has just released.
+template <int BN, int EPI, typename OutT, int NBUF>
+__device__ __forceinline__ void epilogue_issuer(const TcParams& p, const CUtensorMap* mo,
+                                                const CUtensorMap* mi, uint8_t* ebuf, uint64_t* tb,
+                                                int wg) {
+  using T = TeCfg<EPI, OutT, NBUF>;
+  static_assert(T::HAS_IN && T::ARR == 1, "epilogues with an input");
+  constexpr int CW = T::CW, NCH = BN / CW, SL = T::SLOTS, W = T::WAITN;
+  const int rank = int(cluster_ctarank());
+  const uint32_t eb = smem_u32(ebuf);
+  auto inb = [&](int s) { return smem_u32(tb + kEpiIn + 8 * wg + s); };
+  auto rdy = [&](int s) { return smem_u32(tb + kEpiRdy + 8 * wg + s); };
+  const EpiTiles et(p, wg);
+  const int total_chunks = et.my_tiles * NCH;
+  // global coordinates of chunk gc: column n0, first row m0 of this CTA's half
+  auto coords = [&](int gc, int& n0, int& m0) {
+    int tm, tn, sp;
+    tile_coords(p, et.tile(gc / NCH), tm, tn, sp);
+    n0 = tn * BN + (gc % NCH) * CW;
+    m0 = tm * BM2 + rank * BM;
+  };
+  int next_load = 0;  // next chunk whose input is to be fetched
+  auto issue_load = [&]() {
+    int n0, m0;
+    coords(next_load, n0, m0);
+    const int slot = next_load % SL;
+    mbar_expect_tx(inb(slot), 8192);
+    tma_load_2d(eb + slot * 8192, mi, inb(slot), n0, m0);
+    ++next_load;
+  };
+  while (next_load < min(SL, total_chunks)) issue_load();  // every buffer starts free
+  bool ok = true;
+  for (int g = 0; g < total_chunks; ++g) {
+    if (ok) ok = mbar_wait(rdy(g % SL), uint32_t((g / SL) & 1), p.err, 9);
+    int n0, m0;
+    coords(g, n0, m0);
+    tma_store_2d(mo, eb + (g % SL) * 8192, n0, m0);
+    bulk_commit();
+    bulk_wait_read<W>();  // the stores of chunks <= g - W have read their buffers
+    if (g >= W && next_load < total_chunks) issue_load();
+  }
+  bulk_wait_all();
+  // after an expired wait some fetched inputs may never have been waited
+  // for: let the last one of each buffer land before the CTA exits
+  for (int gc = max(0, next_load - SL); gc < next_load; ++gc)
+    mbar_wait(inb(gc % SL), uint32_t((gc / SL) & 1), p.err, 8);
 }
 
 template <int BN, int EPI, typename OutT, bool TE>
@@ -704,7 +817,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // [stages | epilogue area | barriers]; both CTAs of the pair use the same
   // offsets, which the pair's MMA and its multicast commits rely on
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cfg::STAGE + Cfg::EPI_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 20);
+  static_assert((2 * S + kTmemSlot + 1) * 8 <= Cfg::BAR_BYTES, "barrier area");
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + kTmemSlot);
   const uint32_t sbase = smem_u32(smem);
   auto full = [&](int s) { return smem_u32(bars + s); };
   auto empty = [&](int s) { return smem_u32(bars + S + s); };
@@ -721,9 +835,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull(a), 1);   // the pair's MMA commit
-      mbar_init(tempty(a), 2);  // even CTA: one arrival from each CTA's epilogue
+      // even CTA: the epilogue arrivals of both CTAs (one per warp when the
+      // epilogue has an input and TMA stores, else one per warpgroup)
+      mbar_init(tempty(a), (TE && epi_has_input<EPI>()) ? 8 : 2);
     }
-    for (int s = 0; s < 16; ++s) mbar_init(smem_u32(bars + 2 * S + 4 + s), 1);  // epilogue inputs
+    for (int s = 0; s < 16; ++s) {  // TMA epilogue slots of both warpgroups
+      mbar_init(smem_u32(bars + 2 * S + kEpiIn + s), 1);
+      mbar_init(smem_u32(bars + 2 * S + kEpiRdy + s), 4);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -832,13 +951,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int last = t_local - 1;
       mbar_wait(tfull(last & 1), uint32_t((last >> 1) & 1), p.err, 6);
     }
+  } else if ((warp == 2 || warp == 3) && lane == 0 && TE && epi_has_input<EPI>()) {
+    // ------------------------------------------------ TMA issuer of epilogue warpgroup warp - 2
+    const int wg = warp - 2;
+    if constexpr (TE && epi_has_input<EPI>())
+      epilogue_issuer<BN, EPI, OutT, Cfg::NBUF_WG>(
+          p, &tma_o, &tma_i, smem + S * Cfg::STAGE + wg * Cfg::WG_BYTES, bars + 2 * S, wg);
   } else if (warp >= 4 && TE) {
     // ------------------------------------------------ epilogue warpgroup (TMA stores)
-    // (instantiated for the staged configuration too, where it never runs)
     const int wg = (warp - 4) >> 2;  // warpgroup wg drains accumulator wg
-    epilogue_tma<BN, EPI, OutT, (TE ? Cfg::NBUF_WG : 4)>(
-        p, &tma_o, &tma_o2, &tma_i, smem + S * Cfg::STAGE + wg * Cfg::WG_BYTES, bars + 2 * S,
-        tmem_base, wg);
+    uint8_t* ebuf = smem + S * Cfg::STAGE + wg * Cfg::WG_BYTES;
+    if constexpr (TE && epi_has_input<EPI>())
+      epilogue_tma_split<BN, EPI, OutT, Cfg::NBUF_WG>(p, ebuf, bars + 2 * S, tmem_base, wg);
+    else if constexpr (TE)
+      epilogue_tma<BN, EPI, OutT, Cfg::NBUF_WG>(p, &tma_o, &tma_o2, ebuf, bars + 2 * S, tmem_base,
+                                                wg);
   } else if (warp >= 4) {
     // ------------------------------------------------ epilogue warpgroup
     // TMEM phase: thread e (= row 128 rank + e of the tile, TMEM lane e)
