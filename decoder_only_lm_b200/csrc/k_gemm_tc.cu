@@ -569,9 +569,21 @@ __device__ __forceinline__ void chunk_apply(const TcParams& p, uint8_t* b0, int 
     }
     row_put<OutT>(b0, e, v);
   } else if constexpr (EPI == EPI_CE_GRAD) {
-    const float cs = ep.ce_scale, l2 = row_l * kLog2e;
+    const float cs = ep.ce_scale;
+    if (cs > 0.f) {  // cs 2^x = 2^(x + log2 cs): one packed fma and one ex2 per element
+      const float b = log2f(cs) - row_l * kLog2e;
 #pragma unroll
-    for (int j = 0; j < CW; ++j) v[j] = cs * ex2_hw(fmaf(v[j], kLog2e, -l2));
+      for (int j = 0; j < CW; j += 2) {
+        float a0, a1;
+        fma2(a0, a1, v[j], v[j + 1], kLog2e, kLog2e, b, b);
+        v[j] = ex2_hw(a0);
+        v[j + 1] = ex2_hw(a1);
+      }
+    } else {
+      const float l2 = row_l * kLog2e;
+#pragma unroll
+      for (int j = 0; j < CW; ++j) v[j] = cs * ex2_hw(fmaf(v[j], kLog2e, -l2));
+    }
     if (row_t >= n0 && row_t < n0 + CW) {  // the target column: - scale
 #pragma unroll
       for (int j = 0; j < CW; ++j)
@@ -633,15 +645,16 @@ __device__ __forceinline__ void epilogue_tma(const TcParams& p, const CUtensorMa
     tile_coords(p, et.tile(j), tm, tn, sp);
     const int acc = wg;
     const int m0 = tm * BM2 + rank * BM;  // first row of this CTA's half
-    if (ok) ok = mbar_wait(tfull(acc), (t_local >> 1) & 1, p.err, 4);
-    tc_fence_after();
     const int m = m0 + e;
+    // the row's log-sum-exp and target are fetched while the MMAs still run
     float row_l = 0.f;
     int row_t = -1;
     if (EPI == EPI_CE_GRAD && m < p.M) {
       row_l = p.ep.lse[m];
       row_t = p.ep.tgt[m];
     }
+    if (ok) ok = mbar_wait(tfull(acc), (t_local >> 1) & 1, p.err, 4);
+    tc_fence_after();
     const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
     // the accumulator columns of chunk c+1 are loaded while chunk c is processed
     uint32_t rn[CW];
