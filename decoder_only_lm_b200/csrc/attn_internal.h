@@ -27,9 +27,6 @@ int launch_attn_bwd_ds(const bf16* dout, const bf16* qkv, const bf16* out, const
 int attn_bias_parts(int T);
 // whether launch_attn_bwd_ds with these arguments writes the partial sums
 bool attn_bias_parts_written(int B, int T, int C, int H, const bf16* ds);
-// out[c] (+)= sum over the `parts` rows of p[r * n + c], rows in a fixed order
-int launch_sum_parts(const float* p, int parts, int n, float* out, int accumulate,
-                     cudaStream_t st);
 // workspace of gpt2_attention_bwd: Delta (rounded up to 1 KB), then, for bf16
 // on the tcgen05 path, the score-gradient buffer
 size_t attn_bwd_workspace_total(int B, int T, int C, int H, bool bf16_path);

@@ -111,7 +111,16 @@ struct gpt2_handle {
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_join2 = nullptr;
   float* ws2 = nullptr;
   bf16* ads = nullptr;  // attention score gradients (bf16 tcgen05 path), one layer at a time
-  float* qkvb_parts = nullptr;  // per-block column sums of dqkv left by those kernels
+  // per-block column sums of dqkv left by those kernels, one buffer per layer
+  float* qkvb_parts = nullptr;
+  size_t qkvb_stride = 0;  // floats per layer
+  // partial sums of the vector gradients (LayerNorm gamma / beta, biases), one
+  // buffer per producer, summed in one launch at the end of the backward
+  float* ln_parts = nullptr;  // 2L + 1 LayerNorm backwards
+  size_t ln_stride = 0;       // floats per LayerNorm
+  float* cs_parts = nullptr;  // per layer: fc bias, then qkv bias (when not from attention)
+  size_t cs_stride = 0, cs_qkv_off = 0;
+  std::vector<RowSum> defer;
   void* ws_emb = nullptr;
   double* ws_norm = nullptr;
   DevStatus* status = nullptr;
@@ -648,10 +657,13 @@ int backward_t(gpt2_handle* h, float grad_scale) {
   {
     PROF(GPT2_PROF_LN_BWD, 0, lnb_bytes);
     H_CUDA(h, cudaMemsetAsync(h->dres, 0, M * C * sizeof(float), h->st));
+    h->defer.clear();
     // the residual gradient it leaves is the last layer's mlp.proj bias gradient
     H_TRY(h, (launch_layernorm_bwd<A, A>(dhf, h->res[2 * h->L], h->muf, h->rsf, P + h->off_lnfw,
                                           M, C, h->dres, copy, G + h->off_lnfw, G + h->off_lnfb,
-                                          G + h->lo[h->L - 1].fpb, acc, h->ws, h->st)));
+                                          G + h->lo[h->L - 1].fpb, acc,
+                                          h->ln_parts + 2 * h->L * h->ln_stride, h->st,
+                                          &h->defer)));
   }
   A* du = static_cast<A*>(h->du);
   A* dln = static_cast<A*>(h->dln);
@@ -692,7 +704,8 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     }
     {
       PROF(GPT2_PROF_OTHER, 0, a * M * F);
-      H_TRY(h, launch_colsum<A>(du, M, F, G + o.fcb, acc, sd.ws(), sd.st()));
+      H_TRY(h, launch_colsum<A>(du, M, F, G + o.fcb, acc, h->cs_parts + l * h->cs_stride,
+                                sd.st(), &h->defer));
       H_TRY(h, sd.join());
     }
     {
@@ -700,7 +713,9 @@ int backward_t(gpt2_handle* h, float grad_scale) {
       // ... and attn.proj's bias gradient: column sums of the residual gradient
       H_TRY(h, (launch_layernorm_bwd<A, A>(dln, h->res[2 * l + 1], h->mu2[l], h->rs2[l],
                                             P + o.ln2w, M, C, h->dres, copy, G + o.ln2w,
-                                            G + o.ln2b, G + o.projb, acc, h->ws, h->st)));
+                                            G + o.ln2b, G + o.projb, acc,
+                                            h->ln_parts + (2 * l + 1) * h->ln_stride, h->st,
+                                            &h->defer)));
     }
     {
       // attn.proj: h' = h + att Wp^T + b
@@ -715,13 +730,14 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     {
       PROF(GPT2_PROF_ATTN_BWD, attn_bwd_flops, a * 9.0 * M * C + 8.0 * M * Hh);
       if constexpr (std::is_same<A, bf16>::value) {
+        float* qp = h->qkvb_parts ? h->qkvb_parts + l * h->qkvb_stride : nullptr;
         H_TRY(h, launch_attn_bwd_ds(datt, static_cast<A*>(h->qkv[l]), static_cast<A*>(h->att[l]),
-                                    h->alse[l], B, T, C, Hh, dqkv, h->ws, h->ads, h->st,
-                                    h->qkvb_parts));
+                                    h->alse[l], B, T, C, Hh, dqkv, h->ws, h->ads, h->st, qp));
         // attn.qkv bias gradient from the kernels' per-block column sums
-        if (qkvb_fused)
-          H_TRY(h, launch_sum_parts(h->qkvb_parts, B * attn_bias_parts(T), 3 * C, G + o.qkvb, acc,
-                                    h->st));
+        if (qkvb_fused) {
+          const int parts = B * attn_bias_parts(T);
+          h->defer.push_back(RowSum{qp, G + o.qkvb, nullptr, nullptr, parts, 3 * C, 3 * C, acc});
+        }
       } else
         H_TRY(h, launch_attn_bwd<A>(datt, static_cast<A*>(h->qkv[l]), static_cast<A*>(h->att[l]),
                                     h->alse[l], B, T, C, Hh, dqkv, h->ws, h->st));
@@ -741,7 +757,9 @@ int backward_t(gpt2_handle* h, float grad_scale) {
     {
       PROF(GPT2_PROF_OTHER, 0, a * 3.0 * M * C);
       if (!qkvb_fused)
-        H_TRY(h, launch_colsum<A>(dqkv, M, 3 * C, G + o.qkvb, acc, sd.ws(), sd.st()));
+        H_TRY(h, launch_colsum<A>(dqkv, M, 3 * C, G + o.qkvb, acc,
+                                  h->cs_parts + l * h->cs_stride + h->cs_qkv_off, sd.st(),
+                                  &h->defer));
       H_TRY(h, sd.join());
     }
     {
@@ -749,11 +767,18 @@ int backward_t(gpt2_handle* h, float grad_scale) {
       // ... and the previous layer's mlp.proj bias gradient
       H_TRY(h, (launch_layernorm_bwd<A, A>(dln, h->res[2 * l], h->mu1[l], h->rs1[l], P + o.ln1w,
                                             M, C, h->dres, copy, G + o.ln1w, G + o.ln1b,
-                                            l > 0 ? G + h->lo[l - 1].fpb : nullptr, acc, h->ws,
-                                            h->st)));
+                                            l > 0 ? G + h->lo[l - 1].fpb : nullptr, acc,
+                                            h->ln_parts + 2 * l * h->ln_stride, h->st,
+                                            &h->defer)));
     }
     // layer l's weight matrices are final on st (every side-stream writer joined)
     H_TRY(h, bucket_ready(h, h->L - 1 - l));
+  }
+  {
+    // the vector gradients: every partial buffer above, summed in one launch
+    PROF(GPT2_PROF_OTHER, 0, 0.0);
+    H_TRY(h, launch_row_sums(h->defer.data(), int(h->defer.size()), h->st));
+    h->defer.clear();
   }
   {
     // embedding: both uses of the tied matrix add into one gradient [LECTURE]
@@ -863,11 +888,18 @@ int gpt2_create(const gpt2_config* cfg, gpt2_handle** out) {
   h->ws_bytes = ws;
   h->ws = static_cast<float*>(A(ws));
   h->ws2 = static_cast<float*>(A(ws));
+  auto r64 = [](size_t n) { return (n + 63) / 64 * 64; };  // floats, rounded to 256 bytes
   if (h->use_bf16 && attn_tc_supported(c.max_B, c.max_Tseq, int(C), H)) {
     h->ads = static_cast<bf16*>(A(attn_tc_ds_bytes(c.max_B, c.max_Tseq, H)));
-    h->qkvb_parts = static_cast<float*>(
-        A(size_t(c.max_B) * attn_bias_parts(c.max_Tseq) * 3 * C * sizeof(float)));
+    h->qkvb_stride = r64(size_t(c.max_B) * attn_bias_parts(c.max_Tseq) * 3 * C);
+    h->qkvb_parts = static_cast<float*>(A(size_t(h->L) * h->qkvb_stride * sizeof(float)));
   }
+  // (every buffer starts on a 256-byte boundary: the staged kernels want 16)
+  h->ln_stride = r64(layernorm_bwd_workspace(M, int(C)) / sizeof(float));
+  h->ln_parts = static_cast<float*>(A(size_t(2 * h->L + 1) * h->ln_stride * sizeof(float)));
+  h->cs_qkv_off = r64(colsum_workspace(M, int(F)) / sizeof(float));
+  h->cs_stride = h->cs_qkv_off + r64(colsum_workspace(M, int(3 * C)) / sizeof(float));
+  h->cs_parts = static_cast<float*>(A(size_t(h->L) * h->cs_stride * sizeof(float)));
   h->ws_emb = A(embed_bwd_workspace(M, int(C)));
   h->ws_norm = static_cast<double*>(A(gradnorm_workspace()));
   h->status = static_cast<DevStatus*>(A(sizeof(DevStatus)));

@@ -15,7 +15,6 @@
 
 #include <algorithm>
 
-#include "attn_internal.h"
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -611,11 +610,10 @@ __global__ void __launch_bounds__(kLnWarps * 32, 1) layernorm_bwd_staged_kernel(
 // out[c] (+)= sum_p ws[p][c] for c < n (c >= split goes to out1[c - split],
 // c >= 2 split to out2[c - 2 split]),
 // in a fixed order: 8 interleaved row slices per column, then the 8 slices.
-__global__ void __launch_bounds__(256) reduce_rows_kernel(const float* __restrict__ ws, int parts,
-                                                          int n, float* __restrict__ out0,
-                                                          float* __restrict__ out1, int split,
-                                                          int accumulate,
-                                                          float* __restrict__ out2 = nullptr) {
+__device__ __forceinline__ void reduce_rows_body(const float* __restrict__ ws, int parts, int n,
+                                                 float* __restrict__ out0,
+                                                 float* __restrict__ out1, int split,
+                                                 int accumulate, float* __restrict__ out2) {
   __shared__ float sh[8][33];
   const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + cx;
@@ -631,6 +629,24 @@ __global__ void __launch_bounds__(256) reduce_rows_kernel(const float* __restric
     float* o = c < split ? out0 + c : c < 2 * split ? out1 + (c - split) : out2 + (c - 2 * split);
     *o = accumulate ? *o + t : t;
   }
+}
+__global__ void __launch_bounds__(256) reduce_rows_kernel(const float* __restrict__ ws, int parts,
+                                                          int n, float* __restrict__ out0,
+                                                          float* __restrict__ out1, int split,
+                                                          int accumulate,
+                                                          float* __restrict__ out2 = nullptr) {
+  reduce_rows_body(ws, parts, n, out0, out1, split, accumulate, out2);
+}
+// Up to kRowSumMax such sums in one launch: blockIdx.y picks the sum, the
+// same arithmetic in the same order as reduce_rows_kernel.
+constexpr int kRowSumMax = 64;
+struct RowSumBatch {
+  RowSum s[kRowSumMax];
+};
+__global__ void __launch_bounds__(256) reduce_rows_batch_kernel(const __grid_constant__ RowSumBatch b) {
+  const RowSum& r = b.s[blockIdx.y];
+  if (int(blockIdx.x) * 32 >= r.n) return;  // the whole block: this sum has fewer columns
+  reduce_rows_body(r.p, r.parts, r.n, r.out0, r.out1, r.split, r.accumulate, r.out2);
 }
 
 // ------------------------------------------------------------ bias-gradient column sums
@@ -982,7 +998,8 @@ size_t layernorm_bwd_workspace(int64_t M, int C) {
 template <typename DyT, typename CopyT>
 int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const float* rstd,
                          const float* g, int64_t M, int C, float* dx, CopyT* dx_copy, float* dg,
-                         float* db, float* dsum, int accumulate, float* ws, cudaStream_t st) {
+                         float* db, float* dsum, int accumulate, float* ws, cudaStream_t st,
+                         std::vector<RowSum>* defer) {
   if (C > kLnMaxPerLane * 32) {
     gpt2_internal::set_error("layernorm: C above 1024");
     return GPT2_ERR_ARG;
@@ -1010,8 +1027,12 @@ int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const
       COUNT_LAUNCH(1);
     }
     const int n = (dsum ? 3 : 2) * C;
-    reduce_rows_kernel<<<cdiv(n, 32), 256, 0, st>>>(ws, nb, n, dg, db, C, accumulate, dsum);
-    COUNT_LAUNCH(1);
+    if (defer) {
+      defer->push_back(RowSum{ws, dg, db, dsum, nb, n, C, accumulate});
+    } else {
+      reduce_rows_kernel<<<cdiv(n, 32), 256, 0, st>>>(ws, nb, n, dg, db, C, accumulate, dsum);
+      COUNT_LAUNCH(1);
+    }
   } else {
     const int nb = int(cdiv64(M, kLnRowsPerBlock));
     if (nb > 0) {
@@ -1036,13 +1057,15 @@ int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const
 template int launch_layernorm_bwd<float, float>(const float*, const float*, const float*,
                                                 const float*, const float*, int64_t, int, float*,
                                                 float*, float*, float*, float*, int, float*,
-                                                cudaStream_t);
+                                                cudaStream_t, std::vector<RowSum>*);
 template int launch_layernorm_bwd<bf16, bf16>(const bf16*, const float*, const float*, const float*,
                                               const float*, int64_t, int, float*, bf16*, float*,
-                                              float*, float*, int, float*, cudaStream_t);
+                                              float*, float*, int, float*, cudaStream_t,
+                                              std::vector<RowSum>*);
 template int launch_layernorm_bwd<float, bf16>(const float*, const float*, const float*,
                                                const float*, const float*, int64_t, int, float*,
-                                               bf16*, float*, float*, float*, int, float*, cudaStream_t);
+                                               bf16*, float*, float*, float*, int, float*, cudaStream_t,
+                                               std::vector<RowSum>*);
 
 // Column sums over a slab of kColRows rows, 16 bytes per lane and row: a block
 // of 32 lanes x 8 row slices covers 32*VEC columns; lanes of a warp read one
@@ -1093,27 +1116,23 @@ __global__ void __launch_bounds__(256) colsum_vec_kernel(const InT* __restrict__
   }
 }
 
-int launch_sum_parts(const float* p, int parts, int n, float* out, int accumulate,
-                     cudaStream_t st) {
-  reduce_rows_kernel<<<cdiv(n, 32), 256, 0, st>>>(p, parts, n, out, nullptr, n, accumulate);
-  COUNT_LAUNCH(1);
-  GPT2_LAUNCH_CHECK();
-  return GPT2_OK;
-}
-
 size_t colsum_workspace(int64_t M, int N) { return size_t(cdiv64(M, kColRows)) * N * sizeof(float); }
 
 template <typename InT>
 int launch_colsum(const InT* in, int64_t M, int N, float* out, int accumulate, float* ws,
-                  cudaStream_t st) {
+                  cudaStream_t st, std::vector<RowSum>* defer) {
   const int parts = int(cdiv64(M, kColRows));
   constexpr int VEC = 16 / int(sizeof(InT));
   if (N % VEC == 0 && (reinterpret_cast<uintptr_t>(in) & 15) == 0) {
     dim3 grid(cdiv(N, 32 * VEC), parts);
     colsum_vec_kernel<InT><<<grid, 256, 0, st>>>(in, M, N, ws);
     COUNT_LAUNCH(1);
-    reduce_rows_kernel<<<cdiv(N, 32), 256, 0, st>>>(ws, parts, N, out, nullptr, N, accumulate);
-    COUNT_LAUNCH(1);
+    if (defer) {
+      defer->push_back(RowSum{ws, out, nullptr, nullptr, parts, N, N, accumulate});
+    } else {
+      reduce_rows_kernel<<<cdiv(N, 32), 256, 0, st>>>(ws, parts, N, out, nullptr, N, accumulate);
+      COUNT_LAUNCH(1);
+    }
   } else {
     dim3 grid(cdiv(N, kThreads), parts);
     colsum_partial_kernel<InT><<<grid, kThreads, 0, st>>>(in, M, N, ws);
@@ -1124,8 +1143,27 @@ int launch_colsum(const InT* in, int64_t M, int N, float* out, int accumulate, f
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;
 }
-template int launch_colsum<float>(const float*, int64_t, int, float*, int, float*, cudaStream_t);
-template int launch_colsum<bf16>(const bf16*, int64_t, int, float*, int, float*, cudaStream_t);
+template int launch_colsum<float>(const float*, int64_t, int, float*, int, float*, cudaStream_t,
+                                  std::vector<RowSum>*);
+template int launch_colsum<bf16>(const bf16*, int64_t, int, float*, int, float*, cudaStream_t,
+                                 std::vector<RowSum>*);
+
+int launch_row_sums(const RowSum* sums, int count, cudaStream_t st) {
+  for (int i0 = 0; i0 < count; i0 += kRowSumMax) {
+    const int k = std::min(kRowSumMax, count - i0);
+    RowSumBatch b{};
+    int max_n = 0;
+    for (int i = 0; i < k; ++i) {
+      b.s[i] = sums[i0 + i];
+      max_n = std::max(max_n, b.s[i].n);
+    }
+    if (max_n <= 0) continue;
+    reduce_rows_batch_kernel<<<dim3(cdiv(max_n, 32), k), 256, 0, st>>>(b);
+    COUNT_LAUNCH(1);
+    GPT2_LAUNCH_CHECK();
+  }
+  return GPT2_OK;
+}
 
 size_t gradnorm_workspace() { return kNormBlocks * sizeof(double); }
 

@@ -1,6 +1,8 @@
 // Host-side launchers of the library's kernels (internal, C++ linkage).
 #pragma once
 
+#include <vector>
+
 #include "common.cuh"
 
 // ---------------------------------------------------------------- GEMM
@@ -70,18 +72,31 @@ int launch_embed_bwd(const int32_t* x, const float* dh, int B, int T, int C, int
 template <typename OutT>
 int launch_layernorm_fwd(const float* x, const float* g, const float* b, OutT* y, float* mean,
                          float* rstd, int64_t M, int C, float eps, cudaStream_t st);
+// A fixed-order sum of the `parts` rows of the fp32 matrix p [parts, n]:
+// column c (+)= into out0[c] (c < split), out1[c - split] (c < 2 split) or
+// out2[c - 2 split].  The backward pass collects these (LayerNorm and bias
+// gradient partials, each in a buffer of its own) and runs them in one launch
+// at its end: only the optimizer reads the vectors they produce.
+struct RowSum {
+  const float* p;
+  float *out0, *out1, *out2;
+  int parts, n, split, accumulate;
+};
+int launch_row_sums(const RowSum* sums, int count, cudaStream_t st);
 size_t layernorm_bwd_workspace(int64_t M, int C);
 // dx (+)= LN backward; dg, db (+)= dgamma, dbeta; dsum (nullable) (+)= column
-// sums of the updated dx.
+// sums of the updated dx.  With `defer`, the final sum of the partial rows in
+// ws is appended there instead of launched (ws must then stay untouched until
+// launch_row_sums runs the list).
 template <typename DyT, typename CopyT>
 int launch_layernorm_bwd(const DyT* dy, const float* x, const float* mean, const float* rstd,
                          const float* g, int64_t M, int C, float* dx, CopyT* dx_copy,
                          float* dg, float* db, float* dsum, int accumulate, float* ws,
-                         cudaStream_t st);
+                         cudaStream_t st, std::vector<RowSum>* defer = nullptr);
 size_t colsum_workspace(int64_t M, int N);
 template <typename InT>
 int launch_colsum(const InT* in, int64_t M, int N, float* out, int accumulate, float* ws,
-                  cudaStream_t st);
+                  cudaStream_t st, std::vector<RowSum>* defer = nullptr);
 // gradient norm (deterministic two-stage, double accumulation) into *norm (device)
 size_t gradnorm_workspace();
 int launch_gradnorm(const float* g, int64_t n, double* ws, float* norm, cudaStream_t st);
