@@ -63,6 +63,28 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x for a pair on the FMA pipe: x = n + f with n the nearest integer (from
+// the 1.5 * 2^23 shift) and f in [-1/2, 1/2]; 2^f from a cubic fitted here to
+// 2^f on that interval (equal-ripple relative error, at most 7.5e-5, below the
+// bf16 rounding of the probabilities); 2^n added to the exponent field (the
+// shift's own bits drop out of bits(t) << 23).  Arguments below -126 give ~0.
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261113f, c3 = 0.05517167f;
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0 = x0, t1 = x1;
+  add2(t0, t1, kShift, kShift);  // n in the low mantissa bits of t
+  float n0 = t0, n1 = t1;
+  add2(n0, n1, -kShift, -kShift);
+  float f0, f1, p0, p1;
+  fma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);  // f = x - n (exact)
+  fma2(p0, p1, f0, f1, c3, c3, c2, c2);
+  fma2(p0, p1, p0, p1, f0, f1, c1, c1);
+  fma2(p0, p1, p0, p1, f0, f1, c0, c0);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -656,8 +678,12 @@ __global__ void __launch_bounds__(kThreads, 2)
           const float2 nl = *reinterpret_cast<const float2*>(sLD + qc);
           float t0, t1;
           fma2(t0, t1, __uint_as_float(sx[c]), __uint_as_float(sx[c + 1]), sl2, sl2, nl.x, nl.y);
-          pv[qc] = ex2(t0);
-          pv[qc + 1] = ex2(t1);
+          if (((qc >> 1) % 2 == 1)) {
+            ex2_poly2(t0, t1, pv[qc], pv[qc + 1]);
+          } else {
+            pv[qc] = ex2(t0);
+            pv[qc + 1] = ex2(t1);
+          }
         }
       }
       if (need_mask) {
