@@ -208,55 +208,78 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // ====================================================================== forward
+// Persistent: two CTAs per SM walk the (query block, head, batch) items,
+// listed longest first, one per round of grid-size items, every other round
+// in reverse CTA order (long and short items pair up).  Q and the O
+// accumulator are double-buffered per item (shared memory, TMEM) and every
+// barrier's phase follows a tile counter that runs across items, so the next
+// item's Q / K / V loads and first S MMAs overlap the current item's last
+// tiles and its output store.
 constexpr int NSF = 4;  // K/V stages (5 measured 0.7% slower)
-constexpr int kFwdSmem = kRowTile + NSF * 2 * kStrTile + 256 + 1024;
+constexpr int kFwdSmem = 2 * kRowTile + NSF * 2 * kStrTile + 256 + 1024;
 
 struct FwdParams {
   int T, C, H;
+  int nblk, n_items;  // query blocks per (batch, head); items = nblk * H * B
   bf16* out;
   float* lse;
   int* err;
 };
+// item i: query block nblk - 1 - i / (B H) (longest first), then (batch, head)
+struct FwdItem {
+  int qb, h, b;
+};
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int i, int BH) {
+  const int bh = i % BH;
+  return FwdItem{p.nblk - 1 - i / BH, bh % p.H, bh / p.H};
+}
 
 __global__ void __launch_bounds__(kThreads, 2)
     fa_tc_fwd_kernel(const __grid_constant__ CUtensorMap m128, const __grid_constant__ CUtensorMap m64,
                      const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  const uint32_t sQ = smem_u32(smem);
-  const uint32_t sK = sQ + kRowTile;             // NSF x 8 KB
-  const uint32_t sV = sK + NSF * kStrTile;       // NSF x 8 KB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRowTile + 2 * NSF * kStrTile);
-  // q_full | kv_full[NSF] | kv_empty[NSF] | s_full[2] | s_free[2] | p_full[2] | o_done[2] | slot
-  const uint32_t b_q = smem_u32(bars);
-  auto b_kvf = [&](int s) { return smem_u32(bars + 1 + s); };
-  auto b_kve = [&](int s) { return smem_u32(bars + 1 + NSF + s); };
-  auto b_sf = [&](int i) { return smem_u32(bars + 1 + 2 * NSF + i); };
-  auto b_sfr = [&](int i) { return smem_u32(bars + 3 + 2 * NSF + i); };
-  auto b_pf = [&](int i) { return smem_u32(bars + 5 + 2 * NSF + i); };
-  auto b_od = [&](int i) { return smem_u32(bars + 7 + 2 * NSF + i); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 2 * NSF);
+  const uint32_t sQ0 = smem_u32(smem);            // 2 x 16 KB
+  const uint32_t sK = sQ0 + 2 * kRowTile;         // NSF x 8 KB
+  const uint32_t sV = sK + NSF * kStrTile;        // NSF x 8 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kRowTile + 2 * NSF * kStrTile);
+  // q_full[2] | q_empty[2] | kv_full[NSF] | kv_empty[NSF] | s_full[2] | s_free[2] | p_full[2] |
+  // o_done[2] | o_empty[2] | slot
+  auto b_q = [&](int i) { return smem_u32(bars + i); };
+  auto b_qe = [&](int i) { return smem_u32(bars + 2 + i); };
+  auto b_kvf = [&](int s) { return smem_u32(bars + 4 + s); };
+  auto b_kve = [&](int s) { return smem_u32(bars + 4 + NSF + s); };
+  auto b_sf = [&](int i) { return smem_u32(bars + 4 + 2 * NSF + i); };
+  auto b_sfr = [&](int i) { return smem_u32(bars + 6 + 2 * NSF + i); };
+  auto b_pf = [&](int i) { return smem_u32(bars + 8 + 2 * NSF + i); };
+  auto b_od = [&](int i) { return smem_u32(bars + 10 + 2 * NSF + i); };
+  auto b_oe = [&](int i) { return smem_u32(bars + 12 + 2 * NSF + i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14 + 2 * NSF);
 
-  const WorkItem wi = work_item();
-  const int qb = gridDim.x - 1 - wi.step;
-  const int h = wi.h, b = wi.b;
-  const int T = p.T, C = p.C;
-  const int last_key = min(T, (qb + 1) * BR) - 1;
-  const int nkt = last_key / BS + 1;  // 64-key tiles 0 .. nkt-1
-  const int row_base = b * T;
+  const int T = p.T, C = p.C, BH = p.H * (p.n_items / (p.nblk * p.H));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // 64-key tiles of an item: keys 0 .. min(T, (qb + 1) BR) - 1
+  auto n_tiles = [&](int qb) { return (min(T, (qb + 1) * BR) - 1) / BS + 1; };
+  // this CTA's k-th item: one per round of gridDim.x items, the rounds taken
+  // in alternating directions so that long and short items pair up
+  auto item_of = [&](int k) {
+    const int G = int(gridDim.x), c = int(blockIdx.x);
+    return k * G + ((k & 1) ? G - 1 - c : c);
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(b_q, 1);
-    for (int s = 0; s < NSF; ++s) {
-      mbar_init(b_kvf(s), 1);
-      mbar_init(b_kve(s), 1);
-    }
     for (int i = 0; i < 2; ++i) {
+      mbar_init(b_q(i), 1);
+      mbar_init(b_qe(i), 1);
       mbar_init(b_sf(i), 1);
       mbar_init(b_sfr(i), 128);
       mbar_init(b_pf(i), 128);
       mbar_init(b_od(i), 1);
+      mbar_init(b_oe(i), 128);
+    }
+    for (int s = 0; s < NSF; ++s) {
+      mbar_init(b_kvf(s), 1);
+      mbar_init(b_kve(s), 1);
     }
     init_bar_fence();
   }
@@ -265,159 +288,190 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;  // S buffers at +0 and +64
+  const uint32_t tS = tmem;  // S buffers at +0 and +64; O buffers at +128 and +192
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ TMA
-    mbar_expect_tx(b_q, kRowTile);
-    tma_load_2d(sQ, &m128, b_q, h * D, row_base + qb * BR);
-    int issued = 0;
-    for (int j = 0; j < nkt; ++j) {
-      const int s = j % NSF;
-      if (!mbar_wait(b_kve(s), ((j / NSF) & 1) ^ 1, p.err, 11)) break;
-      mbar_expect_tx(b_kvf(s), 2 * kStrTile);
-      tma_load_2d(sK + s * kStrTile, &m64, b_kvf(s), C + h * D, row_base + j * BS);
-      tma_load_2d(sV + s * kStrTile, &m64, b_kvf(s), 2 * C + h * D, row_base + j * BS);
-      ++issued;
+    int g = 0, issued_q = 0;
+    bool ok = true;
+    for (int k = 0; ok && item_of(k) < p.n_items; ++k) {
+      const FwdItem w = fwd_item(p, item_of(k), BH);
+      const int row_base = w.b * T, nkt = n_tiles(w.qb), qbuf = k & 1;
+      // Q_k goes into the buffer item k - 2 used, once its last S MMA is done
+      if (!mbar_wait(b_qe(qbuf), ((k >> 1) & 1) ^ 1, p.err, 11)) break;
+      mbar_expect_tx(b_q(qbuf), kRowTile);
+      tma_load_2d(sQ0 + qbuf * kRowTile, &m128, b_q(qbuf), w.h * D, row_base + w.qb * BR);
+      ++issued_q;
+      for (int j = 0; j < nkt; ++j, ++g) {
+        const int s = g % NSF;
+        if (!mbar_wait(b_kve(s), ((g / NSF) & 1) ^ 1, p.err, 11)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(b_kvf(s), 2 * kStrTile);
+        tma_load_2d(sK + s * kStrTile, &m64, b_kvf(s), C + w.h * D, row_base + j * BS);
+        tma_load_2d(sV + s * kStrTile, &m64, b_kvf(s), 2 * C + w.h * D, row_base + j * BS);
+      }
     }
-    mbar_wait(b_q, 0, p.err, 15);
-    for (int q = 1; q <= min(issued, NSF); ++q) {
-      const int idx = issued - q;
-      mbar_wait(b_kvf(idx % NSF), uint32_t((idx / NSF) & 1), p.err, 15);
-    }
+    // every issued copy has landed before the CTA may exit
+    for (int q = max(0, issued_q - 2); q < issued_q; ++q)
+      mbar_wait(b_q(q & 1), uint32_t((q >> 1) & 1), p.err, 15);
+    for (int q = max(0, g - NSF); q < g; ++q)
+      mbar_wait(b_kvf(q % NSF), uint32_t((q / NSF) & 1), p.err, 15);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------ MMA
+    // per tile: S_g = Q K_g^T; then O += P_{g-1} V_{g-1} of the previous tile
+    // (possibly of the previous item), so the next S is queued before it
     const uint32_t id_s = idesc_bf16(BR, BS, 0, 0);
     const uint32_t id_o = idesc_bf16(BR, D, 0, 1);
-    // slice-0 descriptors, stage s adds s * kStrTile bytes
-    const uint64_t dQ = desc_kmajor(sQ, 0), dK = desc_kmajor(sK, 0), dVm = desc_mnmajor(sV, 0);
-    bool ok = mbar_wait(b_q, 0, p.err, 12);
-    int last_pv = -1;
-    for (int j = 0; ok && j <= nkt; ++j) {
-      if (j < nkt) {
-        const int s = j % NSF;
-        if (!mbar_wait(b_kvf(s), (j / NSF) & 1, p.err, 12) ||
-            !mbar_wait(b_sfr(j & 1), ((j >> 1) & 1) ^ 1, p.err, 12)) {
+    const uint64_t dK = desc_kmajor(sK, 0), dVm = desc_mnmajor(sV, 0);
+    struct Pending {
+      int g, k, j;  // tile counter, item number, tile within the item
+    } pv{-1, 0, 0};
+    bool ok = true;
+    auto issue_pv = [&](const Pending& t) -> bool {
+      if (!mbar_wait(b_pf(t.g & 1), (t.g >> 1) & 1, p.err, 13)) return false;
+      // the first P V of item k overwrites O buffer k & 1: item k - 2's output read
+      if (t.j == 0 && !mbar_wait(b_oe(t.k & 1), ((t.k >> 1) & 1) ^ 1, p.err, 13)) return false;
+      tc_fence_after();
+      // P sits in the first 32 columns of its score buffer (two bf16 per
+      // column); S_{g+2} reuses that buffer only after this MMA (issue order)
+      mma_ts4(tmem + 128 + 64 * (t.k & 1), tS + (t.g & 1) * BS,
+              desc_offset(dVm, (t.g % NSF) * kStrTile), id_o, 128, t.j > 0);
+      umma_commit(b_od(t.g & 1));
+      umma_commit(b_kve(t.g % NSF));
+      return true;
+    };
+    int g = 0;
+    for (int k = 0; ok && item_of(k) < p.n_items; ++k) {
+      const FwdItem w = fwd_item(p, item_of(k), BH);
+      const int nkt = n_tiles(w.qb), qbuf = k & 1;
+      if (!mbar_wait(b_q(qbuf), (k >> 1) & 1, p.err, 12)) break;
+      const uint64_t dQ = desc_kmajor(sQ0 + qbuf * kRowTile, 0);
+      for (int j = 0; j < nkt; ++j, ++g) {
+        const int s = g % NSF;
+        if (!mbar_wait(b_kvf(s), (g / NSF) & 1, p.err, 12) ||
+            !mbar_wait(b_sfr(g & 1), ((g >> 1) & 1) ^ 1, p.err, 12)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        mma_ss4(tS + (j & 1) * BS, dQ, desc_offset(dK, s * kStrTile), id_s, 2, 2, false);
-        umma_commit(b_sf(j & 1));
-      }
-      if (j >= 1) {
-        const int jj = j - 1, s = jj % NSF;
-        if (!mbar_wait(b_pf(jj & 1), (jj >> 1) & 1, p.err, 13)) {
+        mma_ss4(tS + (g & 1) * BS, dQ, desc_offset(dK, s * kStrTile), id_s, 2, 2, false);
+        umma_commit(b_sf(g & 1));
+        if (j == nkt - 1) umma_commit(b_qe(qbuf));  // Q_k read by its last S MMA
+        if (pv.g >= 0 && !issue_pv(pv)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        // P_jj sits in the first 32 columns of its score buffer (two bf16 per
-        // column); S_{jj+2} reuses that buffer only after this MMA (issue order)
-        mma_ts4(tO, tS + (jj & 1) * BS, desc_offset(dVm, s * kStrTile), id_o, 128, jj > 0);
-        umma_commit(b_od(jj & 1));
-        umma_commit(b_kve(s));
-        last_pv = jj;
+        pv = Pending{g, k, j};
       }
     }
-    if (last_pv >= 0) mbar_wait(b_od(last_pv & 1), uint32_t((last_pv >> 1) & 1), p.err, 16);
+    if (ok && pv.g >= 0) ok = issue_pv(pv);
+    // all issued MMAs complete before TMEM is released
+    if (pv.g >= 0) mbar_wait(b_od(pv.g & 1), uint32_t((pv.g >> 1) & 1), p.err, 16);
   } else if (warp >= 2) {
     // ------------------------------------------------ softmax warpgroup
     const int e = (warp & 3) * 32 + lane;  // query row in the block = TMEM lane
-    const int q = qb * BR + e;
     const uint32_t lo = uint32_t((warp & 3) * 32) << 16;
     const float sl2 = rsqrtf(float(D)) * kLog2e;
-    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkt; ++j) {
-      bool w = mbar_wait(b_sf(j & 1), (j >> 1) & 1, p.err, 14);
-      if (!__all_sync(0xffffffffu, w)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld32_async(tS + lo + (j & 1) * BS, r0);
-      tmem_ld32_async(tS + lo + (j & 1) * BS + 32, r1);
-      tmem_wait_ld(r0);
-      reg_after_wait(r1);
-      tc_fence_before();
-      mbar_arrive(b_sfr(j & 1));
-      const int key0 = j * BS;
-      const bool need_mask = key0 + BS - 1 > qb * BR || key0 + BS > T;
-      float x[64];  // raw scores; keys past the query or past T become -inf
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        x[i] = __uint_as_float(r0[i]);
-        x[32 + i] = __uint_as_float(r1[i]);
-      }
-      if (need_mask) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) x[i] = (key0 + i > q || key0 + i >= T) ? -INFINITY : x[i];
-      }
-      // running maximum in log2 units (scale > 0 commutes with max)
-      const float mn = fmaxf(m, max64(x) * sl2);
-      const bool resc = mn > m + kRescale;  // always on the first tile (m = -inf)
-      const float mu = resc ? mn : m;
-      const float corr = resc ? ex2(m - mn) : 1.f;
-      // p = 2^(x sl2 - mu): one packed FMA per pair, ex2 per element, packed sums
-      uint32_t pk[32];
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-      // branch-free (so the pairs interleave); masked scores are -inf and
-      // ex2.approx(-inf) is exactly 0
-#pragma unroll
-      for (int i = 0; i < 64; i += 2) {
-        float t0, t1;
-        fma2(t0, t1, x[i], x[i + 1], sl2, sl2, -mu, -mu);
-        const float p0 = ex2(t0), p1 = ex2(t1);
-        add2(sa[(i >> 1) & 3], sb[(i >> 1) & 3], p0, p1);
-        pk[i >> 1] = pack2(p0, p1);
-      }
-      const float rs = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
-      l = l * corr + rs;
-      m = mu;
-      if (j >= 1 && __any_sync(0xffffffffu, resc)) {
-        // O must hold P_{j-1} V_{j-1} before it is rescaled
-        w = mbar_wait(b_od((j - 1) & 1), ((j - 1) >> 1) & 1, p.err, 17);
-        if (!__all_sync(0xffffffffu, w)) {
+    int g = 0;
+    for (int k = 0; ok && item_of(k) < p.n_items; ++k) {
+      const FwdItem w = fwd_item(p, item_of(k), BH);
+      const int nkt = n_tiles(w.qb), row_base = w.b * T;
+      const int q = w.qb * BR + e;
+      const uint32_t tO = tmem + 128 + 64 * (k & 1);
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkt; ++j, ++g) {
+        bool wt = mbar_wait(b_sf(g & 1), (g >> 1) & 1, p.err, 14);
+        if (!__all_sync(0xffffffffu, wt)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t o0[32], o1[32];
-        tmem_ld32_async(tO + lo, o0);
-        tmem_ld32_async(tO + lo + 32, o1);
-        tmem_wait_ld(o0);
-        reg_after_wait(o1);
-        float f0[32], f1[32];
+        uint32_t r0[32], r1[32];
+        tmem_ld32_async(tS + lo + (g & 1) * BS, r0);
+        tmem_ld32_async(tS + lo + (g & 1) * BS + 32, r1);
+        tmem_wait_ld(r0);
+        reg_after_wait(r1);
+        tc_fence_before();
+        mbar_arrive(b_sfr(g & 1));
+        const int key0 = j * BS;
+        const bool need_mask = key0 + BS - 1 > w.qb * BR || key0 + BS > T;
+        float x[64];  // raw scores; keys past the query or past T become -inf
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          f0[i] = __uint_as_float(o0[i]) * corr;
-          f1[i] = __uint_as_float(o1[i]) * corr;
+          x[i] = __uint_as_float(r0[i]);
+          x[32 + i] = __uint_as_float(r1[i]);
         }
-        tmem_st32(tO + lo, f0);
-        tmem_st32(tO + lo + 32, f1);
+        if (need_mask) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) x[i] = (key0 + i > q || key0 + i >= T) ? -INFINITY : x[i];
+        }
+        // running maximum in log2 units (scale > 0 commutes with max)
+        const float mn = fmaxf(m, max64(x) * sl2);
+        const bool resc = mn > m + kRescale;  // always on the first tile (m = -inf)
+        const float mu = resc ? mn : m;
+        const float corr = resc ? ex2(m - mn) : 1.f;
+        // p = 2^(x sl2 - mu): one packed FMA per pair, ex2 per element, packed sums
+        uint32_t pk[32];
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        // branch-free (so the pairs interleave); masked scores are -inf and
+        // ex2.approx(-inf) is exactly 0
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          float t0, t1;
+          fma2(t0, t1, x[i], x[i + 1], sl2, sl2, -mu, -mu);
+          const float p0 = ex2(t0), p1 = ex2(t1);
+          add2(sa[(i >> 1) & 3], sb[(i >> 1) & 3], p0, p1);
+          pk[i >> 1] = pack2(p0, p1);
+        }
+        const float rs = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
+        l = l * corr + rs;
+        m = mu;
+        if (j >= 1 && __any_sync(0xffffffffu, resc)) {
+          // O must hold P_{g-1} V_{g-1} before it is rescaled
+          wt = mbar_wait(b_od((g - 1) & 1), ((g - 1) >> 1) & 1, p.err, 17);
+          if (!__all_sync(0xffffffffu, wt)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t o0[32], o1[32];
+          tmem_ld32_async(tO + lo, o0);
+          tmem_ld32_async(tO + lo + 32, o1);
+          tmem_wait_ld(o0);
+          reg_after_wait(o1);
+          float f0[32], f1[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            f0[i] = __uint_as_float(o0[i]) * corr;
+            f1[i] = __uint_as_float(o1[i]) * corr;
+          }
+          tmem_st32(tO + lo, f0);
+          tmem_st32(tO + lo + 32, f1);
+        }
+        // P_g (bf16) over the first 32 columns of S_g's buffer, the A operand of P_g V_g
+        tmem_st32_async(tS + lo + (g & 1) * BS, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(b_pf(g & 1));
       }
-      // P_j (bf16) over the first 32 columns of S_j's buffer, the A operand of P_j V_j
-      tmem_st32_async(tS + lo + (j & 1) * BS, pk);
-      tmem_wait_st();
+      if (!ok) break;
+      const int jl = g - 1;  // the item's last tile
+      bool wt = mbar_wait(b_od(jl & 1), (jl >> 1) & 1, p.err, 19);
+      if (!__all_sync(0xffffffffu, wt)) break;
+      tc_fence_after();
+      uint32_t o0[32], o1[32];
+      tmem_ld32_async(tO + lo, o0);
+      tmem_ld32_async(tO + lo + 32, o1);
+      tmem_wait_ld(o0);
+      reg_after_wait(o1);
       tc_fence_before();
-      mbar_arrive(b_pf(j & 1));
-    }
-    if (ok) {
-      const int jl = nkt - 1;
-      bool w = mbar_wait(b_od(jl & 1), (jl >> 1) & 1, p.err, 19);
-      if (__all_sync(0xffffffffu, w)) {
-        tc_fence_after();
-        uint32_t o0[32], o1[32];
-        tmem_ld32_async(tO + lo, o0);
-        tmem_ld32_async(tO + lo + 32, o1);
-        tmem_wait_ld(o0);
-        reg_after_wait(o1);
-        if (q < T) {
-          store_row64(p.out + (int64_t(row_base) + q) * C + h * D, o0, o1, 1.f / l);
-          p.lse[(int64_t(b) * p.H + h) * T + q] = (m + log2f(l)) / kLog2e;
-        }
+      mbar_arrive(b_oe(k & 1));  // the O buffer may take item k + 2
+      if (q < T) {
+        store_row64(p.out + (int64_t(row_base) + q) * C + w.h * D, o0, o1, 1.f / l);
+        p.lse[(int64_t(w.b) * p.H + w.h) * T + q] = (m + log2f(l)) / kLog2e;
       }
     }
   }
@@ -1132,8 +1186,11 @@ int launch_attn_tc_fwd(const bf16* qkv, int B, int T, int C, int H, bf16* out, f
     gpt2_internal::set_error("attention: tensor map encoding failed");
     return GPT2_ERR_CUDA;
   }
-  FwdParams p{T, C, H, out, lse, device_error_word()};
-  dim3 grid(cdiv(T, BR), H, B);
+  const int nblk = cdiv(T, BR);
+  const int64_t items = int64_t(nblk) * H * B;
+  if (items <= 0) return GPT2_OK;
+  FwdParams p{T, C, H, nblk, int(items), out, lse, device_error_word()};
+  const int grid = int(std::min<int64_t>(items, 2 * int64_t(gpt2_internal::sm_count())));
   fa_tc_fwd_kernel<<<grid, kThreads, kFwdSmem, st>>>(m128, m64, p);
   COUNT_LAUNCH(1);
   GPT2_LAUNCH_CHECK();
