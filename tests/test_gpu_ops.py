@@ -107,6 +107,30 @@ def test_attention(g, B, T, C, H, bf16):
     assert rel_l2(dq.float().cpu().numpy(), do) <= tol
 
 
+def test_attention_items_across_rounds(g):
+    """bf16, B=32, T=1024, C=256, H=4: 1024 (query block, head, batch) items,
+    more than the forward kernel's persistent CTAs (two per SM) take at once,
+    so every CTA runs several items in turn, on alternating Q and output
+    buffers with its barrier phases carried from item to item.  Three batch
+    elements, whose items fall in different rounds, against the oracle; the
+    backward (which reads the forward's log-sum-exp) as well."""
+    import torch
+    B, T, C, H = 32, 1024, 256, 4
+    rng = np.random.default_rng(1024)
+    q = torch.from_numpy(rng.normal(size=(B, T, 3 * C)).astype(np.float32)).cuda().bfloat16()
+    dout = torch.from_numpy(rng.normal(size=(B, T, C)).astype(np.float32)).cuda().bfloat16()
+    out, lse = g.attention_fwd(q, H)
+    dq = g.attention_bwd(dout, q, out, lse, H)
+    qr = q.float().cpu().numpy().astype(np.float64)
+    dr = dout.float().cpu().numpy().astype(np.float64)
+    for b in (0, 13, 31):
+        qb = np.ascontiguousarray(qr[b:b + 1])
+        assert rel_l2(out[b:b + 1].float().cpu().numpy(), oracle.attention(qb, H)) <= 3e-2, b
+        do = oracle.attention_bwd(np.ascontiguousarray(dr[b:b + 1]), qb, H)
+        assert rel_l2(dq[b:b + 1].float().cpu().numpy(), do) <= 3e-2, b
+    assert g.device_error() == 0
+
+
 @pytest.mark.parametrize("bf16", [False, True], ids=["fp32", "bf16"])
 def test_lmhead_ce_midsize(g, bf16):
     import torch
