@@ -236,7 +236,7 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int i, int BH) {
 
 __global__ void __launch_bounds__(kThreads, 2)
     fa_tc_fwd_kernel(const __grid_constant__ CUtensorMap m128, const __grid_constant__ CUtensorMap m64,
-                     const FwdParams p) {
+                     const __grid_constant__ CUtensorMap mo, const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sQ0 = smem_u32(smem);            // 2 x 16 KB
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t sV = sK + NSF * kStrTile;        // NSF x 8 KB
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kRowTile + 2 * NSF * kStrTile);
   // q_full[2] | q_empty[2] | kv_full[NSF] | kv_empty[NSF] | s_full[2] | s_free[2] | p_full[2] |
-  // o_done[2] | o_empty[2] | slot
+  // o_done[2] | o_empty[2] | o_staged[2] | slot
   auto b_q = [&](int i) { return smem_u32(bars + i); };
   auto b_qe = [&](int i) { return smem_u32(bars + 2 + i); };
   auto b_kvf = [&](int s) { return smem_u32(bars + 4 + s); };
@@ -254,12 +254,17 @@ __global__ void __launch_bounds__(kThreads, 2)
   auto b_pf = [&](int i) { return smem_u32(bars + 8 + 2 * NSF + i); };
   auto b_od = [&](int i) { return smem_u32(bars + 10 + 2 * NSF + i); };
   auto b_oe = [&](int i) { return smem_u32(bars + 12 + 2 * NSF + i); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14 + 2 * NSF);
+  auto b_ost = [&](int i) { return smem_u32(bars + 14 + 2 * NSF + i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16 + 2 * NSF);
 
   const int T = p.T, C = p.C, BH = p.H * (p.n_items / (p.nblk * p.H));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // 64-key tiles of an item: keys 0 .. min(T, (qb + 1) BR) - 1
   auto n_tiles = [&](int qb) { return (min(T, (qb + 1) * BR) - 1) / BS + 1; };
+  // whole query blocks leave their output tile in their Q buffer for one TMA
+  // store (a block that runs past T is stored row by row: a 2-D box would
+  // reach into the next sequence)
+  auto whole = [&](int qb) { return (qb + 1) * BR <= T; };
   // this CTA's k-th item: one per round of gridDim.x items, the rounds taken
   // in alternating directions so that long and short items pair up
   auto item_of = [&](int k) {
@@ -276,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(b_pf(i), 128);
       mbar_init(b_od(i), 1);
       mbar_init(b_oe(i), 128);
+      mbar_init(b_ost(i), 128);
     }
     for (int s = 0; s < NSF; ++s) {
       mbar_init(b_kvf(s), 1);
@@ -292,13 +298,28 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ TMA
-    int g = 0, issued_q = 0;
+    // item kk's output tile, staged by the softmax warpgroup in its Q buffer
+    auto store_out = [&](int kk) -> bool {
+      if (!mbar_wait(b_ost(kk & 1), uint32_t((kk >> 1) & 1), p.err, 18)) return false;
+      const FwdItem w = fwd_item(p, item_of(kk), BH);
+      if (whole(w.qb)) {
+        tma_store_2d(&mo, sQ0 + (kk & 1) * kRowTile, w.h * D, w.b * T + w.qb * BR);
+        bulk_commit();
+      }
+      return true;
+    };
+    int g = 0, issued_q = 0, k = 0;
     bool ok = true;
-    for (int k = 0; ok && item_of(k) < p.n_items; ++k) {
+    for (; ok && item_of(k) < p.n_items; ++k) {
       const FwdItem w = fwd_item(p, item_of(k), BH);
       const int row_base = w.b * T, nkt = n_tiles(w.qb), qbuf = k & 1;
       // Q_k goes into the buffer item k - 2 used, once its last S MMA is done
+      // and the output tile staged there has been read by its store
       if (!mbar_wait(b_qe(qbuf), ((k >> 1) & 1) ^ 1, p.err, 11)) break;
+      if (k >= 2) {
+        if (!store_out(k - 2)) break;
+        bulk_wait_read<0>();
+      }
       mbar_expect_tx(b_q(qbuf), kRowTile);
       tma_load_2d(sQ0 + qbuf * kRowTile, &m128, b_q(qbuf), w.h * D, row_base + w.qb * BR);
       ++issued_q;
@@ -313,7 +334,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         tma_load_2d(sV + s * kStrTile, &m64, b_kvf(s), 2 * C + w.h * D, row_base + j * BS);
       }
     }
-    // every issued copy has landed before the CTA may exit
+    // the last two items' outputs; every issued copy has landed (loads) or
+    // completed (stores) before the CTA may exit
+    if (ok)
+      for (int kk = max(0, k - 2); kk < k; ++kk)
+        if (!store_out(kk)) break;
+    bulk_wait_all();
     for (int q = max(0, issued_q - 2); q < issued_q; ++q)
       mbar_wait(b_q(q & 1), uint32_t((q >> 1) & 1), p.err, 15);
     for (int q = max(0, g - NSF); q < g; ++q)
@@ -469,10 +495,29 @@ __global__ void __launch_bounds__(kThreads, 2)
       reg_after_wait(o1);
       tc_fence_before();
       mbar_arrive(b_oe(k & 1));  // the O buffer may take item k + 2
-      if (q < T) {
-        store_row64(p.out + (int64_t(row_base) + q) * C + w.h * D, o0, o1, 1.f / l);
-        p.lse[(int64_t(w.b) * p.H + w.h) * T + q] = (m + log2f(l)) / kLog2e;
+      const float il = 1.f / l;
+      if (whole(w.qb)) {
+        // row e of the output tile into Q_k's buffer (every MMA that read Q_k
+        // is complete: they precede the P V whose completion was awaited), in
+        // the 128-byte swizzle of the tensor map: unit u of row e at
+        // e * 128 + 16 * (u ^ (e & 7))
+        uint8_t* row = smem + (k & 1) * kRowTile + e * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t* src = u < 4 ? o0 + 8 * u : o1 + 8 * (u - 4);
+          uint4 v;
+          v.x = pack2(__uint_as_float(src[0]) * il, __uint_as_float(src[1]) * il);
+          v.y = pack2(__uint_as_float(src[2]) * il, __uint_as_float(src[3]) * il);
+          v.z = pack2(__uint_as_float(src[4]) * il, __uint_as_float(src[5]) * il);
+          v.w = pack2(__uint_as_float(src[6]) * il, __uint_as_float(src[7]) * il);
+          *reinterpret_cast<uint4*>(row + ((u ^ (e & 7)) << 4)) = v;
+        }
+        fence_proxy_async();  // visible to the TMA store the producer issues
+      } else if (q < T) {
+        store_row64(p.out + (int64_t(row_base) + q) * C + w.h * D, o0, o1, il);
       }
+      mbar_arrive(b_ost(k & 1));
+      if (q < T) p.lse[(int64_t(w.b) * p.H + w.h) * T + q] = (m + log2f(l)) / kLog2e;
     }
   }
   tc_fence_before();
@@ -1181,8 +1226,10 @@ int launch_attn_tc_fwd(const bf16* qkv, int B, int T, int C, int H, bf16* out, f
   }
   CUtensorMap m128, m64;
   const int64_t rows = int64_t(B) * T;
+  CUtensorMap mo;
   if (!make_map_bf16(&m128, qkv, 3 * int64_t(C), rows, 3 * int64_t(C), BR) ||
-      !make_map_bf16(&m64, qkv, 3 * int64_t(C), rows, 3 * int64_t(C), BS)) {
+      !make_map_bf16(&m64, qkv, 3 * int64_t(C), rows, 3 * int64_t(C), BS) ||
+      !make_map_bf16(&mo, out, int64_t(C), rows, int64_t(C), BR)) {
     gpt2_internal::set_error("attention: tensor map encoding failed");
     return GPT2_ERR_CUDA;
   }
@@ -1191,7 +1238,7 @@ int launch_attn_tc_fwd(const bf16* qkv, int B, int T, int C, int H, bf16* out, f
   if (items <= 0) return GPT2_OK;
   FwdParams p{T, C, H, nblk, int(items), out, lse, device_error_word()};
   const int grid = int(std::min<int64_t>(items, 2 * int64_t(gpt2_internal::sm_count())));
-  fa_tc_fwd_kernel<<<grid, kThreads, kFwdSmem, st>>>(m128, m64, p);
+  fa_tc_fwd_kernel<<<grid, kThreads, kFwdSmem, st>>>(m128, m64, mo, p);
   COUNT_LAUNCH(1);
   GPT2_LAUNCH_CHECK();
   return GPT2_OK;
