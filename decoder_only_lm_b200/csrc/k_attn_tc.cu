@@ -5,8 +5,10 @@
 // probabilities never leave TMEM and registers; the backward may keep the
 // causal half of the score gradients (bf16) for its dQ step.
 //
-// Every kernel: one CTA of 192 threads per block of 128 rows (queries, or keys
-// in dK/dV) = the 128 TMEM lanes, streaming 64-row tiles of the other operand:
+// Every kernel: CTAs of 192 threads working on blocks of 128 rows (queries, or
+// keys in dK/dV) = the 128 TMEM lanes, streaming 64-row tiles of the other
+// operand (the forward's CTAs are persistent and take several blocks in turn,
+// the backward's take one each):
 //   warp 0, one lane   TMA loads (128-row tile once, 64-row tiles in a ring);
 //   warp 1             owns the TMEM allocation (256 columns); one lane issues
 //                      the tcgen05.mma instructions and commits;
@@ -27,6 +29,8 @@
 //   2^8 (probabilities are taken relative to the kept maximum, so they stay
 //   <= 256); P_j (bf16) is written back over its own score buffer in TMEM
 //   and O += P_j V_j reads it from there (A operand in TMEM, V MN-major).
+//   Q and O are double-buffered across a CTA's blocks; the normalised output
+//   tile goes through the block's Q buffer to one TMA store.
 // Backward, with Delta_i = dO_i . O_i and P = exp(S / sqrt(D) - lse):
 //   dK/dV kernel (per 128 keys, 64-query tiles i >= keys): S^T, dP^T = V dO^T,
 //   dS^T = P^T (dP^T - Delta); dV += P^T dO, dK += dS^T Q / sqrt(D);
@@ -36,7 +40,8 @@
 //   exponentials, no second S or dP); without one (the no-allocation entry
 //   point) the dQ kernel recomputes P and dS as above.  Both backward kernels
 //   may also leave per-block column sums of dq, dk, dv (the qkv bias gradient).
-// CTAs take the longest causal row blocks first (work_item).
+// CTAs take the longest causal row blocks first (work_item; the persistent
+// forward: one block per round of grid-size blocks, alternate rounds reversed).
 // Every output element is written by one CTA, no atomics (deterministic).
 // Every wait is bounded (2 s of global time) and reports a timeout in the
 // error word instead of hanging.
