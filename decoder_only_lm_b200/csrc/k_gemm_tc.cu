@@ -8,8 +8,10 @@
 //     128 x BN (BN = 256 or 128), m fastest so co-resident CTAs share B tiles;
 //   - warp-specialised: warp 0 issues TMA loads (one elected lane), warp 1
 //     issues tcgen05.mma (one elected lane), warp 2 owns the TMEM allocation,
-//     warps 4-7 (one warpgroup) drain the accumulator with tcgen05.ld and run
-//     the epilogue;
+//     warps 4-7 and 8-11 (two warpgroups, one per accumulator) drain the
+//     accumulator with tcgen05.ld and run the epilogue; for epilogues with an
+//     input (residual, GELU input) lane 0 of warp 2 / 3 issues the TMA copies
+//     of warpgroup 0 / 1;
 //   - STAGES-deep shared-memory ring of (A, B) k-blocks of 64 elements with
 //     128-byte swizzle, full/empty mbarriers; two TMEM accumulators so the
 //     epilogue of tile i overlaps the MMAs of tile i+1;
