@@ -601,7 +601,7 @@ template <bool KEEP>
 __global__ void __launch_bounds__(kThreads, 2)
     fa_tc_dkdv_kernel(const __grid_constant__ CUtensorMap q128, const __grid_constant__ CUtensorMap q64,
                       const __grid_constant__ CUtensorMap o64, const __grid_constant__ CUtensorMap ds_map,
-                      const BwdParams p) {
+                      const __grid_constant__ CUtensorMap dqkv_map, const BwdParams p) {
   constexpr int NSK = DkdvCfg<KEEP>::NSK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -848,6 +848,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     if (have) tc_fence_after();
     bf16* drow = p.dqkv + (int64_t(row_base) + key) * 3 * C + h * D;
+    // a whole key block leaves its dV and dK tiles in two 16 KB buffers of
+    // the Q/dO ring (idle now: every load has been consumed by an MMA that
+    // has completed; the column sums below use the K/V tiles) for two TMA
+    // stores; a block that runs past T is stored row by row (a 2-D box would
+    // reach into the next sequence)
+    const bool whole = (kb + 1) * BR <= T;
+    uint8_t* stage = smem + 40 * 1024;
     // dV then dK, one 64-column row each (and their column sums: every
     // thread of the warpgroup takes part, whatever the waits gave)
 #pragma unroll 1
@@ -858,7 +865,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_ld32_async((w2 ? tKd : tV) + lo + 32, a1);
         tmem_wait_ld(a0);
         reg_after_wait(a1);
-        if (key < T) store_row64(drow + (w2 ? C : 2 * C), a0, a1, w2 ? scale : 1.f);
+        const float f = w2 ? scale : 1.f;
+        if (whole) {
+          // row e in the 128-byte swizzle of the tensor map: unit u at e * 128 + 16 * (u ^ (e & 7))
+          uint8_t* row = stage + w2 * kRowTile + e * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t* src = u < 4 ? a0 + 8 * u : a1 + 8 * (u - 4);
+            uint4 v;
+            v.x = pack2(__uint_as_float(src[0]) * f, __uint_as_float(src[1]) * f);
+            v.y = pack2(__uint_as_float(src[2]) * f, __uint_as_float(src[3]) * f);
+            v.z = pack2(__uint_as_float(src[4]) * f, __uint_as_float(src[5]) * f);
+            v.w = pack2(__uint_as_float(src[6]) * f, __uint_as_float(src[7]) * f);
+            *reinterpret_cast<uint4*>(row + ((u ^ (e & 7)) << 4)) = v;
+          }
+          fence_proxy_async();  // visible to the TMA stores below
+        } else if (key < T) {
+          store_row64(drow + (w2 ? C : 2 * C), a0, a1, f);
+        }
       }
       if (p.bias_part) {
         // the K / V rows of the keys past T are excluded by selection (a
@@ -876,6 +900,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                     p.bias_part + (int64_t(b) * gridDim.x + kb) * 3 * C + (w2 ? C : 2 * C) +
                         h * D);
       }
+    }
+    wg_bar();  // every row of both tiles written
+    if (whole && have && e == 0) {
+      tma_store_2d(&dqkv_map, smem_u32(stage), 2 * C + h * D, row_base + kb * BR);             // dV
+      tma_store_2d(&dqkv_map, smem_u32(stage + kRowTile), C + h * D, row_base + kb * BR);  // dK
+      bulk_commit();
+      bulk_wait_read<0>();  // the shared memory is released with the CTA
     }
   }
   tc_fence_before();
@@ -1268,12 +1299,13 @@ int launch_attn_tc_bwd(const bf16* dout, const bf16* qkv, const float* lse, cons
     gpt2_internal::set_error("attention: score-gradient buffer misaligned or too large");
     return GPT2_ERR_ARG;
   }
-  CUtensorMap q128, q64, o128, o64;
+  CUtensorMap q128, q64, o128, o64, dmap;
   const int64_t rows = int64_t(B) * T;
   if (!make_map_bf16(&q128, qkv, 3 * int64_t(C), rows, 3 * int64_t(C), BR) ||
       !make_map_bf16(&q64, qkv, 3 * int64_t(C), rows, 3 * int64_t(C), BS) ||
       !make_map_bf16(&o128, dout, int64_t(C), rows, int64_t(C), BR) ||
-      !make_map_bf16(&o64, dout, int64_t(C), rows, int64_t(C), BS)) {
+      !make_map_bf16(&o64, dout, int64_t(C), rows, int64_t(C), BS) ||
+      !make_map_bf16(&dmap, dqkv, 3 * int64_t(C), rows, 3 * int64_t(C), BR)) {
     gpt2_internal::set_error("attention: tensor map encoding failed");
     return GPT2_ERR_CUDA;
   }
@@ -1287,11 +1319,13 @@ int launch_attn_tc_bwd(const bf16* dout, const bf16* qkv, const float* lse, cons
   BwdParams p{T, C, H, lse, delta, dqkv, ds, ntri, device_error_word(), ds ? bias_part : nullptr};
   dim3 grid(nqb, H, B);
   if (ds) {
-    fa_tc_dkdv_kernel<true><<<grid, kThreads, DkdvCfg<true>::kSmem, st>>>(q128, q64, o64, ds_st, p);
+    fa_tc_dkdv_kernel<true><<<grid, kThreads, DkdvCfg<true>::kSmem, st>>>(q128, q64, o64, ds_st, dmap,
+                                                                          p);
     COUNT_LAUNCH(1);
     fa_tc_dq_ds_kernel<<<grid, kThreads, kDqgSmem, st>>>(ds_ld, q64, p);
   } else {
-    fa_tc_dkdv_kernel<false><<<grid, kThreads, DkdvCfg<false>::kSmem, st>>>(q128, q64, o64, q64, p);
+    fa_tc_dkdv_kernel<false><<<grid, kThreads, DkdvCfg<false>::kSmem, st>>>(q128, q64, o64, q64,
+                                                                            dmap, p);
     COUNT_LAUNCH(1);
     fa_tc_dq_kernel<<<grid, kThreads, kDqSmem, st>>>(q128, q64, o128, p);
   }
