@@ -116,3 +116,28 @@ def test_null_arguments_are_refused(g):
     assert g.lib.gpt2_generate(None, buf, 1, 4, 4, 0.0, 0, 1.0, None, buf) == g.ERR_ARG
     assert g.lib.gpt2_generate_cached(None, buf, 1, 4, 4, 0.0, 0, 1.0, None, buf) == g.ERR_ARG
     assert g.lib.gpt2_logits_last(None, buf, 1, 4, 1, buf, 64) == g.ERR_ARG
+
+
+def test_attention_bwd_workspace_layout(g):
+    """gpt2_attention_bwd_workspace as the header states it: one float of Delta
+    per (batch, head, position); for bf16 with head size 64, after Delta at a
+    1 KB boundary, the causal half of the score gradients in bf16, B*H*n(n+1)/2
+    tiles of 128 x 128 with n = ceil(T/128) (226 MB at B=16, T=1024, H=12)."""
+    ws = C.c_size_t()
+
+    def size(B, T, Cc, H, dt):
+        assert g.lib.gpt2_attention_bwd_workspace(B, T, Cc, H, dt, C.byref(ws)) == g.OK
+        return ws.value
+
+    for B, T, Cc, H in [(16, 1024, 768, 12), (2, 130, 128, 2), (3, 1, 128, 2), (1, 2048, 1024, 16)]:
+        delta = B * H * T * 4
+        n = -(-T // 128)
+        assert size(B, T, Cc, H, g.F32) == delta
+        assert size(B, T, Cc, H, g.BF16) == -(-delta // 1024) * 1024 + B * H * n * (n + 1) // 2 * 128 * 128 * 2
+    assert size(16, 1024, 768, 12, g.BF16) - 16 * 12 * 1024 * 4 == 226_492_416
+    # other head sizes (the CUDA-core kernels) keep only Delta
+    assert size(2, 100, 64, 2, g.BF16) == 2 * 2 * 100 * 4
+    assert size(2, 100, 64, 4, g.BF16) == 2 * 4 * 100 * 4
+    # sizes are checked on the host
+    assert g.lib.gpt2_attention_bwd_workspace(0, 8, 128, 2, g.BF16, C.byref(ws)) == g.ERR_ARG
+    assert g.lib.gpt2_attention_bwd_workspace(1, 8, 128, 2, g.BF16, None) == g.ERR_ARG
