@@ -776,6 +776,8 @@ int backward_t(gpt2_handle* h, float grad_scale) {
   }
   {
     // the vector gradients: every partial buffer above, summed in one launch
+    // on st (the side stream's fc-bias partials were joined into st with the
+    // layer that wrote them); before the last bucket, which holds the vectors
     PROF(GPT2_PROF_OTHER, 0, 0.0);
     H_TRY(h, launch_row_sums(h->defer.data(), int(h->defer.size()), h->st));
     h->defer.clear();
